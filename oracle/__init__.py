@@ -1,0 +1,244 @@
+"""fp64 CPU oracle for exact scaled-dot-product attention (test infrastructure).
+
+Only the test suite, ``__graft_entry__.smoke()`` and the bench's CPU-baseline
+leg may import this package.  The CUDA library never calls it and shares no
+code with it; there is no CPU fallback anywhere in the product path.
+
+The arithmetic lives in ``attn_oracle.c`` (plain C, fp64, OpenMP over rows);
+this module only compiles it with gcc and marshals numpy arrays.
+
+Parity status of each function (what pins it, see ``tests/test_oracle_pins.py``):
+
+* ``fwd`` / ``probs`` -- pinned: the worked example [2, 5, 1, 4] of the
+  FlashAttention-2 tutorial (2.1.9), row sums, constant V, key permutation,
+  causal row 0, closed forms (one key, Q = 0), the fully masked row, and an
+  independent library witness (torch fp64 softmax) on small shapes.
+* ``bwd`` / ``bwd_sampled`` -- pinned: central finite differences of the
+  forward's loss on tiny shapes, gradient invariants (columns of dS sum to
+  zero, sum_j dV_j = sum_i dO_i), grouped-query equality to the sum of
+  per-head gradients, and a torch fp64 autograd witness.
+* ``online_row`` / ``merge`` -- pinned: the worked example's block statistics
+  (block A: m = 5, S = 1.0498; ratio 0.7312; block C = [10] rescale e^-5) and
+  brute-force equality with the one-pass softmax over every block split.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_SO = os.path.join(_BUILD, "libattn_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_ip = ctypes.POINTER(ctypes.c_int)
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library with gcc (fp64, OpenMP)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        tmp = _SO + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fopenmp", "-fno-fast-math",
+               "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(tmp, _SO)
+    return _SO
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            lib.oracle_set_threads.argtypes = [ctypes.c_int]
+            lib.oracle_get_threads.restype = ctypes.c_int
+            lib.oracle_fwd_head.argtypes = [_dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_double, ctypes.c_int, ctypes.c_int, _ip,
+                                            ctypes.c_int, _dp, _dp]
+            lib.oracle_probs_head.argtypes = [_dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_double, ctypes.c_int, ctypes.c_int, _dp, _dp]
+            lib.oracle_bwd_head.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, ctypes.c_double, ctypes.c_int,
+                                            ctypes.c_int, _dp, _dp, _dp]
+            lib.oracle_bwd_head_sampled.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
+                                                    ctypes.c_int, ctypes.c_double, ctypes.c_int,
+                                                    ctypes.c_int, _ip, ctypes.c_int, _ip,
+                                                    ctypes.c_int, _dp, _dp, _dp]
+            lib.oracle_online_row.argtypes = [_dp, _dp, ctypes.c_int, ctypes.c_int, _ip, ctypes.c_int,
+                                              _dp, _dp, _dp, _dp, _dp]
+            lib.oracle_merge.argtypes = [ctypes.c_double, ctypes.c_double, _dp, ctypes.c_double,
+                                         ctypes.c_double, _dp, ctypes.c_int, _dp, _dp, _dp]
+            _lib = lib
+    return _lib
+
+
+def set_threads(n: int) -> None:
+    _load().oracle_set_threads(int(n))
+
+
+def threads() -> int:
+    return int(_load().oracle_get_threads())
+
+
+def _f64(x) -> np.ndarray:
+    """fp64 C-contiguous copy; uint16 inputs are read as bf16 bit patterns."""
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        u = np.ascontiguousarray(x).astype(np.uint32) << np.uint32(16)
+        return u.view(np.float32).astype(np.float64)
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(_dp)
+
+
+def _pi(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(_ip)
+
+
+def _kv_len(k_lens, b, Lk):
+    return int(Lk if k_lens is None else k_lens[b])
+
+
+def fwd(Q, K, V, scale: float, causal: bool = False, k_lens=None, rows=None, heads=None):
+    """Forward of every (b, h) head, or of the listed ``heads`` [(b, h), ...].
+
+    Q [B,Hq,Lq,d]; K, V [B,Hkv,Lk,d] (fp64 or bf16 bits); query head h reads
+    key/value head h // (Hq // Hkv).  ``rows`` restricts the query rows.
+    Returns (O, LSE): O [B,Hq,R,d] fp64 and LSE [B,Hq,R] fp64 (R = len(rows) or
+    Lq); heads not listed are left at zero.
+    """
+    lib = _load()
+    B, Hq, Lq, d = np.shape(Q)
+    _, Hkv, Lk, _ = np.shape(K)
+    G = Hq // Hkv
+    rows_a = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
+    R = Lq if rows_a is None else len(rows_a)
+    O = np.zeros((B, Hq, R, d))
+    L = np.zeros((B, Hq, R))
+    todo = [(b, h) for b in range(B) for h in range(Hq)] if heads is None else list(heads)
+    for b, h in todo:
+        q = _f64(Q[b, h])
+        k = _f64(K[b, h // G])
+        v = _f64(V[b, h // G])
+        o = np.zeros((R, d))
+        lse = np.zeros(R)
+        lib.oracle_fwd_head(_p(q), _p(k), _p(v), Lq, Lk, d, float(scale), int(bool(causal)),
+                            _kv_len(k_lens, b, Lk), _pi(rows_a), R, _p(o), _p(lse))
+        O[b, h] = o
+        L[b, h] = lse
+    return O, L
+
+
+def probs(Q, K, scale: float, causal: bool = False, kv_len=None):
+    """Full probability matrix P [Lq,Lk] and LSE [Lq] of one head (Q [Lq,d], K [Lk,d])."""
+    lib = _load()
+    q = _f64(Q)
+    k = _f64(K)
+    Lq, d = q.shape
+    Lk = k.shape[0]
+    P = np.zeros((Lq, Lk))
+    lse = np.zeros(Lq)
+    lib.oracle_probs_head(_p(q), _p(k), Lq, Lk, d, float(scale), int(bool(causal)),
+                          int(Lk if kv_len is None else kv_len), _p(P), _p(lse))
+    return P, lse
+
+
+def bwd(Q, K, V, dO, scale: float, causal: bool = False, k_lens=None):
+    """Full backward: returns (dQ [B,Hq,Lq,d], dK [B,Hkv,Lk,d], dV [B,Hkv,Lk,d]) in fp64.
+
+    Grouped query heads accumulate into their shared key/value head."""
+    lib = _load()
+    B, Hq, Lq, d = np.shape(Q)
+    _, Hkv, Lk, _ = np.shape(K)
+    G = Hq // Hkv
+    dQ = np.zeros((B, Hq, Lq, d))
+    dK = np.zeros((B, Hkv, Lk, d))
+    dV = np.zeros((B, Hkv, Lk, d))
+    for b in range(B):
+        for hk in range(Hkv):
+            k = _f64(K[b, hk])
+            v = _f64(V[b, hk])
+            dk = np.zeros((Lk, d))
+            dv = np.zeros((Lk, d))
+            for h in range(hk * G, hk * G + G):
+                q = _f64(Q[b, h])
+                g = _f64(dO[b, h])
+                dq = np.zeros((Lq, d))
+                lib.oracle_bwd_head(_p(q), _p(k), _p(v), _p(g), Lq, Lk, d, float(scale),
+                                    int(bool(causal)), _kv_len(k_lens, b, Lk), _p(dq), _p(dk),
+                                    _p(dv))
+                dQ[b, h] = dq
+            dK[b, hk] = dk
+            dV[b, hk] = dv
+    return dQ, dK, dV
+
+
+def bwd_sampled(Q, K, V, dO, scale: float, causal: bool, k_lens, b: int, hk: int, qrows, kcols):
+    """Backward of key/value head (b, hk) at sampled outputs.
+
+    Returns (dQ [G,nq,d] for the G query heads of hk at rows ``qrows``,
+    dK [nk,d] and dV [nk,d] at key rows ``kcols``), all fp64."""
+    lib = _load()
+    B, Hq, Lq, d = np.shape(Q)
+    _, Hkv, Lk, _ = np.shape(K)
+    G = Hq // Hkv
+    qa = np.ascontiguousarray(qrows, dtype=np.int32)
+    ka = np.ascontiguousarray(kcols, dtype=np.int32)
+    k = _f64(K[b, hk])
+    v = _f64(V[b, hk])
+    dQs = np.zeros((G, len(qa), d))
+    dKs = np.zeros((len(ka), d))
+    dVs = np.zeros((len(ka), d))
+    for gi, h in enumerate(range(hk * G, hk * G + G)):
+        q = _f64(Q[b, h])
+        g = _f64(dO[b, h])
+        dq = np.zeros((len(qa), d))
+        lib.oracle_bwd_head_sampled(_p(q), _p(k), _p(v), _p(g), Lq, Lk, d, float(scale),
+                                    int(bool(causal)), _kv_len(k_lens, b, Lk), _pi(qa), len(qa),
+                                    _pi(ka), len(ka), _p(dq), _p(dKs), _p(dVs))
+        dQs[gi] = dq
+    return dQs, dKs, dVs
+
+
+def online_row(s, V, block_ends):
+    """Unnormalised online softmax over one score row; returns (O, m, l, m_trace, l_trace)."""
+    lib = _load()
+    s = _f64(s)
+    V = _f64(V)
+    n, d = V.shape
+    be = np.ascontiguousarray(block_ends, dtype=np.int32)
+    O = np.zeros(d)
+    m = np.zeros(1)
+    l = np.zeros(1)
+    mt = np.zeros(len(be))
+    lt = np.zeros(len(be))
+    lib.oracle_online_row(_p(s), _p(V), n, d, _pi(be), len(be), _p(O), _p(m), _p(l), _p(mt),
+                          _p(lt))
+    return O, float(m[0]), float(l[0]), mt, lt
+
+
+def merge(m_a, l_a, O_a, m_b, l_b, O_b):
+    """Normalised merge of two partial (m, l, O) results; returns (m, l, O)."""
+    lib = _load()
+    Oa = _f64(O_a)
+    Ob = _f64(O_b)
+    d = Oa.shape[0]
+    O = np.zeros(d)
+    m = np.zeros(1)
+    l = np.zeros(1)
+    lib.oracle_merge(float(m_a), float(l_a), _p(Oa), float(m_b), float(l_b), _p(Ob), d, _p(m),
+                     _p(l), _p(O))
+    return float(m[0]), float(l[0]), O

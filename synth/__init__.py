@@ -1,0 +1,111 @@
+"""Seeded synthetic inputs shared by the tests, the bench and the smoke check.
+
+This module holds no attention arithmetic.  It only turns a seed into
+reproducible bf16 tensors and integer key lengths, so that the fp64 oracle and
+the CUDA path see bit-identical inputs.
+
+Generator
+---------
+* counter-based splitmix64: element ``i`` of stream ``seed`` is
+  ``mix(seed * 2**32 + i + 1)`` where ``mix`` is Steele, Lea and Flood's
+  splitmix64 finaliser (multiply by the golden-ratio increment, then two
+  xor-shift-multiply rounds and a final xor-shift);
+* a normal draw uses two uniforms ``u1, u2 in (0, 1]`` (53-bit mantissas) and
+  the Box-Muller cosine branch ``sqrt(-2 ln u1) * cos(2 pi u2)``;
+* fp64 -> fp32 -> bf16, each step round-to-nearest-even.
+
+The workloads' tensors are i.i.d. N(0, 1) in bf16, laid out ``[B, H, L, d]``
+row-major; per-request key lengths are integers uniform in ``[lo, hi]``.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+_GOLDEN = np.uint64(0x9E3779B97F4A7C15)
+_M1 = np.uint64(0xBF58476D1CE4E5B9)
+_M2 = np.uint64(0x94D049BB133111EB)
+
+
+def _mix(x: np.ndarray) -> np.ndarray:
+    """splitmix64 output function applied to counters ``x`` (uint64, wraps mod 2**64)."""
+    with np.errstate(over="ignore"):
+        z = x * _GOLDEN
+        z = (z ^ (z >> np.uint64(30))) * _M1
+        z = (z ^ (z >> np.uint64(27))) * _M2
+        return z ^ (z >> np.uint64(31))
+
+
+def uniform_u64(seed: int, n: int, offset: int = 0) -> np.ndarray:
+    """``n`` raw 64-bit draws of stream ``seed`` starting at counter ``offset``."""
+    base = np.uint64((int(seed) & 0xFFFFFFFF) << 32)
+    ctr = np.arange(offset + 1, offset + n + 1, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        return _mix(base + ctr)
+
+
+def _unit(u: np.ndarray) -> np.ndarray:
+    """Map raw draws to doubles in (0, 1]."""
+    return ((u >> np.uint64(11)).astype(np.float64) + 1.0) * (2.0 ** -53)
+
+
+def normal_f64(seed: int, n: int) -> np.ndarray:
+    """``n`` N(0,1) doubles from stream ``seed`` (Box-Muller, cosine branch)."""
+    raw = uniform_u64(seed, 2 * n)
+    u1 = _unit(raw[0::2])
+    u2 = _unit(raw[1::2])
+    return np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
+
+
+def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """fp64 -> fp32 (RNE) -> bf16 (RNE); returns the bf16 bit patterns as uint16."""
+    f = np.ascontiguousarray(x, dtype=np.float64).astype(np.float32)
+    b = f.view(np.uint32).astype(np.uint64)
+    # round-to-nearest-even on the 16 dropped bits; NaN/Inf do not occur here
+    lsb = (b >> np.uint64(16)) & np.uint64(1)
+    b = (b + np.uint64(0x7FFF) + lsb) >> np.uint64(16)
+    return b.astype(np.uint16)
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns to fp64."""
+    u = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return u.view(np.float32).astype(np.float64)
+
+
+def normal_bf16(seed: int, shape) -> np.ndarray:
+    """i.i.d. N(0,1) tensor of the given shape, as bf16 bit patterns (uint16)."""
+    n = int(np.prod(shape)) if len(shape) else 1
+    return f64_to_bf16_bits(normal_f64(seed, n)).reshape(shape)
+
+
+def uniform_int(seed: int, n: int, lo: int, hi: int) -> np.ndarray:
+    """``n`` integers uniform in ``[lo, hi]`` (int32)."""
+    raw = uniform_u64(seed, n)
+    span = np.uint64(hi - lo + 1)
+    return (np.int64(lo) + (raw % span).astype(np.int64)).astype(np.int32)
+
+
+def to_torch_bf16(bits: np.ndarray):
+    """View bf16 bit patterns as a CPU ``torch.bfloat16`` tensor (no copy of values)."""
+    import torch
+
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+
+# Workload seeds: 46 * 100 + workload number; each tensor draws its own stream.
+def workload_seed(workload: int, tensor: str) -> int:
+    tags = {"q": 1, "k": 2, "v": 3, "do": 4, "klen": 5}
+    return (4600 + workload) * 16 + tags[tensor]
+
+
+__all__ = [
+    "uniform_u64",
+    "normal_f64",
+    "f64_to_bf16_bits",
+    "bf16_bits_to_f64",
+    "normal_bf16",
+    "uniform_int",
+    "to_torch_bf16",
+    "workload_seed",
+]

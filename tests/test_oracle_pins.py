@@ -1,0 +1,408 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+None of these compares the oracle with itself: each check is a value printed
+on the pages (the worked example of the FlashAttention-2 tutorial, 2.1.9), a
+closed form, an invariant of softmax attention, a special case that reduces to
+a simpler problem, brute force over block splits, central finite differences,
+or an independent library witness (torch fp64).
+"""
+
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "online_softmax_worked_example.txt")
+
+
+def _golden():
+    vals = {}
+    for line in open(GOLDEN):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        k, v = [t.strip() for t in line.split("=")]
+        nums = [float(x) for x in v.split()]
+        vals[k] = nums if len(nums) > 1 else nums[0]
+    return vals
+
+
+def _rand(seed, shape):
+    return synth.bf16_bits_to_f64(synth.normal_bf16(seed, shape))
+
+
+def _worked_qkv(scores, d=None):
+    """One query whose scaled scores against n = len(scores) keys are exactly
+    ``scores`` (scale 1, q = e_0, k_j = scores[j] e_0), head dimension d
+    (default n) and, when d == n, V = identity so that O = P."""
+    n = len(scores)
+    d = n if d is None else d
+    Q = np.zeros((1, 1, 1, d))
+    Q[0, 0, 0, 0] = 1.0
+    K = np.zeros((1, 1, n, d))
+    K[0, 0, :, 0] = scores
+    V = np.eye(n, d)[None, None]
+    return Q, K, V
+
+
+# ---------------------------------------------------------------- worked example
+
+
+def test_worked_example_one_pass():
+    g = _golden()
+    Q, K, V = _worked_qkv(g["scores"])
+    O, L = oracle.fwd(Q, K, V, scale=1.0)
+    p = O[0, 0, 0]
+    assert np.all(np.abs(p - np.array(g["probs"])) <= g["tol"])
+    # LSE = max + ln(sum of shifted exponentials), from the printed max and sum
+    assert abs(L[0, 0, 0] - (g["max"] + math.log(g["sum"]))) <= g["tol_sum"] / g["sum"] + 1e-12
+    # the exponentials relative to the max and their sum
+    P, lse = oracle.probs(Q[0, 0], K[0, 0], 1.0)
+    e = P[0] * math.exp(lse[0] - g["max"])
+    assert np.all(np.abs(e - np.array(g["exps"])) <= g["tol"])
+    assert abs(e.sum() - g["sum"]) <= g["tol_sum"]
+    assert abs(P[0].sum() - 1.0) <= 1e-15
+
+
+def test_worked_example_two_blocks_unnormalised():
+    g = _golden()
+    n = len(g["scores"])
+    O, m, l, mt, lt = oracle.online_row(g["scores"], np.eye(n), [int(x) for x in g["block_ends"]])
+    assert np.all(np.abs(O - np.array(g["probs"])) <= g["tol"])
+    assert mt[0] == g["blockA_max"] and m == g["max"]
+    assert abs(lt[0] - g["blockA_sum"]) <= g["tol"]
+    assert abs(lt[1] - g["sum"]) <= g["tol_sum"]
+    assert abs((lt[1] - lt[0]) - g["blockB_sum"]) <= g["tol"]
+
+
+def test_worked_example_two_blocks_normalised_merge():
+    g = _golden()
+    s = np.array(g["scores"])
+    n = len(s)
+    # each block on its own: (m, l, O) with O normalised inside the block
+    Oa, ma, la, _, _ = oracle.online_row(s[:2], np.eye(n)[:2], [2])
+    Ob, mb, lb, _, _ = oracle.online_row(s[2:], np.eye(n)[2:], [2])
+    assert np.all(np.abs(Oa[:2] - np.array(g["blockA_probs"])) <= g["tol"])
+    m, l, O = oracle.merge(ma, la, Oa, mb, lb, Ob)
+    assert np.all(np.abs(O - np.array(g["probs"])) <= g["tol"])
+    # weight that carries the block-A probabilities into the merged row
+    ratio = math.exp(ma - m) * la / l
+    assert abs(ratio - g["old_over_new"]) <= g["tol_ratio"]
+    # block B's unnormalised weights relative to the running max 5
+    wb = np.exp(s[2:] - m)
+    assert np.all(np.abs(wb - np.array(g["blockB_weights"])) <= g["tol"])
+
+
+def test_worked_example_block_c_rescale():
+    """A third block [10] raises the max from 5 to 10: the history is scaled by e^-5."""
+    g = _golden()
+    s = np.array(list(g["scores"]) + [g["blockC"]])
+    n = len(s)
+    O, m, l, mt, lt = oracle.online_row(s, np.eye(n), [2, 4, 5])
+    assert mt[1] == g["max"] and mt[2] == g["blockC"] and m == g["blockC"]
+    factor = math.exp(g["blockC_factor_exponent"])
+    assert abs(lt[2] - (lt[1] * factor + 1.0)) <= 1e-15
+    # and the result is the one-pass softmax of all five scores
+    Q, K, V = _worked_qkv(s)
+    O1, _ = oracle.fwd(Q, K, V, scale=1.0)
+    assert np.max(np.abs(O - O1[0, 0, 0])) <= 1e-15
+
+
+# ---------------------------------------------------------------- invariants
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_rows_sum_to_one_and_masked_zero(causal):
+    Q = _rand(11, (37, 16))
+    K = _rand(12, (53, 16))
+    P, lse = oracle.probs(Q, K, 0.25, causal=causal, kv_len=41)
+    vis = P > 0
+    assert np.all(np.abs(P.sum(axis=1) - 1.0) <= 1e-14)
+    i = np.arange(37)[:, None]
+    j = np.arange(53)[None, :]
+    allowed = (j < 41) & ((~np.bool_(causal)) | (j <= i + (53 - 37)))
+    assert not np.any(vis & ~allowed)
+
+
+def test_constant_v_gives_v():
+    Q = _rand(21, (1, 2, 19, 8))
+    K = _rand(22, (1, 2, 23, 8))
+    v = _rand(23, (8,))
+    V = np.broadcast_to(v, (1, 2, 23, 8)).copy()
+    for causal in (False, True):
+        O, _ = oracle.fwd(Q, K, V, 0.3, causal=causal)
+        assert np.max(np.abs(O - v)) <= 1e-14 * max(1.0, np.max(np.abs(v)))
+
+
+def test_key_permutation_invariance_non_causal():
+    Q = _rand(31, (1, 1, 9, 8))
+    K = _rand(32, (1, 1, 14, 8))
+    V = _rand(33, (1, 1, 14, 8))
+    perm = np.random.default_rng(0).permutation(14)
+    O1, L1 = oracle.fwd(Q, K, V, 0.35)
+    O2, L2 = oracle.fwd(Q, K[:, :, perm], V[:, :, perm], 0.35)
+    assert np.max(np.abs(O1 - O2)) <= 1e-13
+    assert np.max(np.abs(L1 - L2)) <= 1e-13
+
+
+def test_causal_row_zero_is_v0():
+    Q = _rand(41, (1, 1, 12, 16))
+    K = _rand(42, (1, 1, 12, 16))
+    V = _rand(43, (1, 1, 12, 16))
+    O, L = oracle.fwd(Q, K, V, 0.25, causal=True)
+    assert np.array_equal(O[0, 0, 0], V[0, 0, 0])
+    s00 = float(np.dot(Q[0, 0, 0], K[0, 0, 0])) * 0.25
+    assert abs(L[0, 0, 0] - s00) <= 1e-13
+
+
+def test_single_key_closed_form():
+    Q = _rand(51, (2, 2, 7, 8))
+    K = _rand(52, (2, 2, 1, 8))
+    V = _rand(53, (2, 2, 1, 8))
+    O, L = oracle.fwd(Q, K, V, 0.5)
+    assert np.array_equal(O, np.broadcast_to(V, O.shape))
+    s = np.einsum("bhid,bhjd->bhi", Q, K) * 0.5
+    assert np.max(np.abs(L - s)) <= 1e-13
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_query_gives_mean_of_visible(causal):
+    Lq, Lk, kl = 6, 10, 8
+    Q = np.zeros((1, 1, Lq, 4))
+    K = _rand(61, (1, 1, Lk, 4))
+    V = _rand(62, (1, 1, Lk, 4))
+    O, L = oracle.fwd(Q, K, V, 1.0, causal=causal, k_lens=[kl])
+    for i in range(Lq):
+        hi = min(kl, i + (Lk - Lq) + 1) if causal else kl
+        assert np.max(np.abs(O[0, 0, i] - V[0, 0, :hi].mean(axis=0))) <= 1e-14
+        assert abs(L[0, 0, i] - math.log(hi)) <= 1e-14
+
+
+def test_fully_masked_rows():
+    Q = _rand(71, (2, 1, 5, 4))
+    K = _rand(72, (2, 1, 3, 4))
+    V = _rand(73, (2, 1, 3, 4))
+    # k_len = 0 masks every key of sequence 0
+    O, L = oracle.fwd(Q, K, V, 1.0, k_lens=[0, 3])
+    assert np.all(O[0] == 0.0) and np.all(L[0] == -np.inf)
+    assert np.all(np.isfinite(L[1]))
+    # bottom-right causal with Lq > Lk: row i sees keys j <= i - 2
+    O, L = oracle.fwd(Q, K, V, 1.0, causal=True, k_lens=[3, 3])
+    assert np.all(O[:, :, :2] == 0.0) and np.all(L[:, :, :2] == -np.inf)
+    assert np.array_equal(O[:, :, 2], V[:, :, 0])
+
+
+def test_padding_equals_truncated_problem():
+    """A key length k reduces to the unmasked problem on the first k keys."""
+    Q = _rand(81, (1, 2, 11, 8))
+    K = _rand(82, (1, 2, 17, 8))
+    V = _rand(83, (1, 2, 17, 8))
+    O1, L1 = oracle.fwd(Q, K, V, 0.3, k_lens=[9])
+    O2, L2 = oracle.fwd(Q, K[:, :, :9], V[:, :, :9], 0.3)
+    assert np.max(np.abs(O1 - O2)) <= 1e-15 and np.max(np.abs(L1 - L2)) <= 1e-15
+    # causal + padding: bottom-right causality is defined against the full Lk
+    O3, _ = oracle.fwd(Q, K, V, 0.3, causal=True, k_lens=[9])
+    for i in range(11):
+        hi = min(9, i + (17 - 11) + 1)
+        Oi, _ = oracle.fwd(Q[:, :, i:i + 1], K[:, :, :hi], V[:, :, :hi], 0.3)
+        assert np.max(np.abs(O3[:, :, i] - Oi[:, :, 0])) <= 1e-14
+
+
+def test_gqa_reads_shared_head():
+    Q = _rand(91, (1, 4, 5, 8))
+    K = _rand(92, (1, 2, 6, 8))
+    V = _rand(93, (1, 2, 6, 8))
+    O, L = oracle.fwd(Q, K, V, 0.3)
+    Ke = np.repeat(K, 2, axis=1)
+    Ve = np.repeat(V, 2, axis=1)
+    O2, L2 = oracle.fwd(Q, Ke, Ve, 0.3)
+    assert np.array_equal(O, O2) and np.array_equal(L, L2)
+
+
+def test_rows_subset_matches_full():
+    Q = _rand(95, (1, 1, 40, 8))
+    K = _rand(96, (1, 1, 40, 8))
+    V = _rand(97, (1, 1, 40, 8))
+    O, L = oracle.fwd(Q, K, V, 0.3, causal=True)
+    rows = [0, 7, 39, 21]
+    Os, Ls = oracle.fwd(Q, K, V, 0.3, causal=True, rows=rows)
+    assert np.array_equal(Os[0, 0], O[0, 0, rows]) and np.array_equal(Ls[0, 0], L[0, 0, rows])
+
+
+# ---------------------------------------------------------------- blockwise == one pass
+
+
+def _compositions(n):
+    """Every split of range(n) into consecutive non-empty blocks, as block right ends."""
+    for cuts in itertools.product([0, 1], repeat=n - 1):
+        ends = [i + 1 for i, c in enumerate(cuts) if c] + [n]
+        yield ends
+
+
+@pytest.mark.parametrize("n,d,seed", [(1, 2, 1), (3, 2, 2), (5, 3, 3), (8, 4, 4)])
+def test_online_equals_one_pass_every_split(n, d, seed):
+    s = _rand(100 + seed, (n,)) * 3.0
+    V = _rand(200 + seed, (n, d))
+    Q, K, _ = _worked_qkv(s, d)
+    O1, L1 = oracle.fwd(Q, K, V[None, None], 1.0)
+    for ends in _compositions(n):
+        O, m, l, _, _ = oracle.online_row(s, V, ends)
+        assert np.max(np.abs(O - O1[0, 0, 0])) <= 1e-12
+        assert abs(m + math.log(l) - L1[0, 0, 0]) <= 1e-12
+        # normalised merge applied block by block gives the same row
+        mm, ll, OO = -np.inf, 0.0, np.zeros(d)
+        start = 0
+        for e in ends:
+            Ob, mb, lb, _, _ = oracle.online_row(s[start:e], V[start:e], [e - start])
+            mm, ll, OO = oracle.merge(mm, ll, OO, mb, lb, Ob)
+            start = e
+        assert np.max(np.abs(OO - O1[0, 0, 0])) <= 1e-12
+
+
+def test_online_with_masked_entries():
+    s = np.array([-np.inf, 1.0, -np.inf, 2.5, 0.5, -np.inf])
+    V = _rand(301, (6, 3))
+    ends_all = list(_compositions(6))
+    ref = None
+    for ends in ends_all:
+        O, m, l, _, _ = oracle.online_row(s, V, ends)
+        ref = O if ref is None else ref
+        assert np.max(np.abs(O - ref)) <= 1e-14
+    w = np.exp(np.array([1.0, 2.5, 0.5]) - 2.5)
+    exp_O = (w[:, None] * V[[1, 3, 4]]).sum(0) / w.sum()
+    assert np.max(np.abs(ref - exp_O)) <= 1e-14
+
+
+# ---------------------------------------------------------------- library witness
+
+
+@pytest.mark.parametrize("causal,klen", [(False, None), (True, None), (True, 19), (False, 5)])
+def test_torch_fp64_witness_forward(causal, klen):
+    import torch
+
+    Q = _rand(401, (2, 4, 13, 16))
+    K = _rand(402, (2, 2, 23, 16))
+    V = _rand(403, (2, 2, 23, 16))
+    kl = None if klen is None else [klen, 23]
+    O, L = oracle.fwd(Q, K, V, 0.25, causal=causal, k_lens=kl)
+    q = torch.from_numpy(Q)
+    k = torch.from_numpy(np.repeat(K, 2, axis=1))
+    v = torch.from_numpy(np.repeat(V, 2, axis=1))
+    s = q @ k.transpose(-1, -2) * 0.25
+    i = torch.arange(13)[:, None]
+    j = torch.arange(23)[None, :]
+    for b in range(2):
+        keep = torch.ones(13, 23, dtype=torch.bool)
+        if causal:
+            keep &= j <= i + 10
+        if kl is not None:
+            keep &= j < kl[b]
+        s[b] = s[b].masked_fill(~keep, float("-inf"))
+    ref_L = torch.logsumexp(s, dim=-1)
+    ref_O = torch.softmax(s, dim=-1) @ v
+    assert np.max(np.abs(O - ref_O.numpy())) <= 1e-13
+    assert np.max(np.abs(L - ref_L.numpy())) <= 1e-13
+
+
+# ---------------------------------------------------------------- backward
+
+
+def _loss(Q, K, V, dO, scale, causal, k_lens):
+    O, _ = oracle.fwd(Q, K, V, scale, causal=causal, k_lens=k_lens)
+    return float(np.sum(O * dO))
+
+
+@pytest.mark.parametrize("causal,k_lens,Hq,Hkv", [(False, None, 1, 1), (True, None, 1, 1),
+                                                   (True, [4], 2, 1), (False, [2], 2, 2)])
+def test_backward_central_differences(causal, k_lens, Hq, Hkv):
+    rng = np.random.default_rng(7)
+    Lq, Lk, d = 3, 5, 2
+    Q = rng.standard_normal((1, Hq, Lq, d))
+    K = rng.standard_normal((1, Hkv, Lk, d))
+    V = rng.standard_normal((1, Hkv, Lk, d))
+    dO = rng.standard_normal((1, Hq, Lq, d))
+    scale = 0.7
+    dQ, dK, dV = oracle.bwd(Q, K, V, dO, scale, causal=causal, k_lens=k_lens)
+    h = 1e-5
+    for X, G in ((Q, dQ), (K, dK), (V, dV)):
+        num = np.zeros_like(X)
+        for idx in np.ndindex(X.shape):
+            old = X[idx]
+            X[idx] = old + h
+            fp = _loss(Q, K, V, dO, scale, causal, k_lens)
+            X[idx] = old - h
+            fm = _loss(Q, K, V, dO, scale, causal, k_lens)
+            X[idx] = old
+            num[idx] = (fp - fm) / (2 * h)
+        err = np.max(np.abs(num - G)) / max(1e-12, np.max(np.abs(G)))
+        assert err <= 1e-6, err
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_invariants(causal):
+    Q = _rand(501, (1, 2, 17, 8))
+    K = _rand(502, (1, 2, 21, 8))
+    V = _rand(503, (1, 2, 21, 8))
+    dO = _rand(504, (1, 2, 17, 8))
+    dQ, dK, dV = oracle.bwd(Q, K, V, dO, 0.3, causal=causal)
+    # every row of dS sums to zero, so the key gradients sum to zero
+    assert np.max(np.abs(dK.sum(axis=2))) <= 1e-12
+    # every visible row of P sums to one, so sum_j dV_j = sum_i dO_i
+    assert np.max(np.abs(dV.sum(axis=2) - dO.sum(axis=2))) <= 1e-12
+
+
+def test_backward_gqa_is_sum_of_heads():
+    Q = _rand(511, (1, 4, 9, 8))
+    K = _rand(512, (1, 2, 11, 8))
+    V = _rand(513, (1, 2, 11, 8))
+    dO = _rand(514, (1, 4, 9, 8))
+    dQ, dK, dV = oracle.bwd(Q, K, V, dO, 0.3, causal=True)
+    Ke = np.repeat(K, 2, axis=1)
+    Ve = np.repeat(V, 2, axis=1)
+    dQe, dKe, dVe = oracle.bwd(Q, Ke, Ve, dO, 0.3, causal=True)
+    assert np.max(np.abs(dQ - dQe)) <= 1e-13
+    assert np.max(np.abs(dK - dKe.reshape(1, 2, 2, 11, 8).sum(2))) <= 1e-13
+    assert np.max(np.abs(dV - dVe.reshape(1, 2, 2, 11, 8).sum(2))) <= 1e-13
+
+
+def test_backward_sampled_matches_full():
+    Q = _rand(521, (1, 4, 33, 8))
+    K = _rand(522, (1, 2, 40, 8))
+    V = _rand(523, (1, 2, 40, 8))
+    dO = _rand(524, (1, 4, 33, 8))
+    dQ, dK, dV = oracle.bwd(Q, K, V, dO, 0.3, causal=True, k_lens=[37])
+    qr = [0, 5, 32, 17]
+    kc = [0, 36, 39, 12]
+    dQs, dKs, dVs = oracle.bwd_sampled(Q, K, V, dO, 0.3, True, [37], 0, 1, qr, kc)
+    assert np.max(np.abs(dQs - dQ[0, 2:4][:, qr])) <= 1e-13
+    assert np.max(np.abs(dKs - dK[0, 1, kc])) <= 1e-13
+    assert np.max(np.abs(dVs - dV[0, 1, kc])) <= 1e-13
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_torch_fp64_autograd_witness_backward(causal):
+    import torch
+
+    Q = _rand(531, (1, 2, 12, 8))
+    K = _rand(532, (1, 2, 15, 8))
+    V = _rand(533, (1, 2, 15, 8))
+    dO = _rand(534, (1, 2, 12, 8))
+    dQ, dK, dV = oracle.bwd(Q, K, V, dO, 0.3, causal=causal)
+    q = torch.tensor(Q, requires_grad=True)
+    k = torch.tensor(K, requires_grad=True)
+    v = torch.tensor(V, requires_grad=True)
+    s = q @ k.transpose(-1, -2) * 0.3
+    if causal:
+        i = torch.arange(12)[:, None]
+        j = torch.arange(15)[None, :]
+        s = s.masked_fill(~(j <= i + 3), float("-inf"))
+    o = torch.softmax(s, dim=-1) @ v
+    o.backward(torch.from_numpy(dO))
+    assert np.max(np.abs(dQ - q.grad.numpy())) <= 1e-12
+    assert np.max(np.abs(dK - k.grad.numpy())) <= 1e-12
+    assert np.max(np.abs(dV - v.grad.numpy())) <= 1e-12
