@@ -1,0 +1,208 @@
+"""Python binding of the B200 exact-attention C library (``libattn.so``).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI of ``include/attn.h``.  PyTorch provides device
+memory and the stream.  There is no CPU or library fallback: if the compiled
+library is missing, every call raises.
+
+The functions carry the C entry points' names:
+
+* ``attn_fwd(Q, K, V, ...) -> (O, LSE)``
+* ``attn_fwd_splitkv_decode(Q, Kcache, Vcache, k_lens, ...) -> (O, LSE)``
+* ``attn_bwd(Q, K, V, O, dO, LSE, ...) -> (dQ, dK, dV)``
+* the ``*_workspace_size`` queries and the device-status helpers.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn.so")
+
+ATTN_OK, ATTN_ERR_INVALID, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT = range(5)
+ATTN_MASK_NONE, ATTN_MASK_CAUSAL = 0, 1
+ATTN_DEV_BAD_KLEN, ATTN_DEV_TIMEOUT = 1, 2
+
+_lock = threading.Lock()
+_lib = None
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+_f = ctypes.c_float
+
+#: exported symbol -> (restype, argtypes); mirrors include/attn.h
+SIGNATURES = {
+    "attn_status_string": (ctypes.c_char_p, [_i]),
+    "attn_num_sms": (_i, []),
+    "attn_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _vp, _sz,
+                      _vp]),
+    "attn_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "attn_fwd_splitkv_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _vp,
+                                     _sz, _vp]),
+    "attn_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "attn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f,
+                      _i, _vp, _vp, _sz, _vp]),
+    "attn_read_device_status": (_i, [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]),
+    "attn_clear_device_status": (_i, [_vp, _vp]),
+}
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} ({code})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"CUDA library not built: {LIB_PATH} is missing "
+                    "(run `python -m exact_io_aware_46_b200.build`); there is no fallback")
+            L = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(L, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    try:
+        return lib().attn_status_string(int(code)).decode()
+    except RuntimeError:
+        return "library not loaded"
+
+
+def _check(code: int, where: str) -> None:
+    if code != ATTN_OK:
+        raise AttnError(code, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _bf16(t, name):
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA bfloat16 tensor")
+
+
+def _workspace(nbytes: int, device, stream):
+    ws = torch.empty(max(256, int(nbytes)), dtype=torch.uint8, device=device)
+    _check(lib().attn_clear_device_status(_ptr(ws), _stream(stream)), "attn_clear_device_status")
+    return ws
+
+
+def attn_num_sms() -> int:
+    return int(lib().attn_num_sms())
+
+
+def attn_fwd_workspace_size(B, Hq, Hkv, Lq, Lk, d) -> int:
+    return int(lib().attn_fwd_workspace_size(B, Hq, Hkv, Lq, Lk, d))
+
+
+def attn_decode_workspace_size(B, Hq, Hkv, Lmax, d) -> int:
+    return int(lib().attn_decode_workspace_size(B, Hq, Hkv, Lmax, d))
+
+
+def attn_bwd_workspace_size(B, Hq, Hkv, Lq, Lk, d) -> int:
+    return int(lib().attn_bwd_workspace_size(B, Hq, Hkv, Lq, Lk, d))
+
+
+def attn_read_device_status(workspace, stream=None) -> tuple[int, int]:
+    bits = ctypes.c_int32(0)
+    code = lib().attn_read_device_status(_ptr(workspace), _stream(stream), ctypes.byref(bits))
+    return int(code), int(bits.value)
+
+
+def attn_clear_device_status(workspace, stream=None) -> None:
+    _check(lib().attn_clear_device_status(_ptr(workspace), _stream(stream)),
+           "attn_clear_device_status")
+
+
+def attn_fwd(Q, K, V, scale=None, causal=False, k_lens=None, O=None, lse=None, workspace=None,
+             stream=None, want_lse=True):
+    """Forward attention.  Q [B,Hq,Lq,d], K/V [B,Hkv,Lk,d] bf16 on the GPU.
+
+    Returns (O, LSE) with O bf16 [B,Hq,Lq,d] and LSE fp32 [B,Hq,Lq] (None if
+    ``want_lse`` is False)."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _bf16(t, n)
+    B, Hq, Lq, d = Q.shape
+    Hkv, Lk = K.shape[1], K.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if O is None:
+        O = torch.empty_like(Q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=Q.device)
+    if workspace is None:
+        workspace = _workspace(attn_fwd_workspace_size(B, Hq, Hkv, Lq, Lk, d), Q.device, stream)
+    code = lib().attn_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse), B, Hq, Hkv, Lq, Lk, d,
+                          float(scale), ATTN_MASK_CAUSAL if causal else ATTN_MASK_NONE,
+                          _ptr(k_lens), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(code, "attn_fwd")
+    return O, lse
+
+
+def attn_fwd_splitkv_decode(Q, Kc, Vc, k_lens, scale=None, O=None, lse=None, workspace=None,
+                            stream=None, want_lse=True):
+    """Split-KV decode.  Q [B,Hq,1,d]; Kc/Vc [B,Hkv,Lmax,d] bf16; k_lens int32 [B] (device)."""
+    for t, n in ((Q, "Q"), (Kc, "Kcache"), (Vc, "Vcache")):
+        _bf16(t, n)
+    B, Hq, _, d = Q.shape
+    Hkv, Lmax = Kc.shape[1], Kc.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if O is None:
+        O = torch.empty_like(Q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=Q.device)
+    if workspace is None:
+        workspace = _workspace(attn_decode_workspace_size(B, Hq, Hkv, Lmax, d), Q.device, stream)
+    code = lib().attn_fwd_splitkv_decode(_ptr(Q), _ptr(Kc), _ptr(Vc), _ptr(O), _ptr(lse), B, Hq,
+                                         Hkv, Lmax, d, float(scale), _ptr(k_lens),
+                                         _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(code, "attn_fwd_splitkv_decode")
+    return O, lse
+
+
+def attn_bwd(Q, K, V, O, dO, lse, scale=None, causal=False, k_lens=None, dQ=None, dK=None,
+             dV=None, workspace=None, stream=None):
+    """Backward.  Returns (dQ, dK, dV) bf16."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V"), (O, "O"), (dO, "dO")):
+        _bf16(t, n)
+    B, Hq, Lq, d = Q.shape
+    Hkv, Lk = K.shape[1], K.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dQ = torch.empty_like(Q) if dQ is None else dQ
+    dK = torch.empty_like(K) if dK is None else dK
+    dV = torch.empty_like(V) if dV is None else dV
+    if workspace is None:
+        workspace = _workspace(attn_bwd_workspace_size(B, Hq, Hkv, Lq, Lk, d), Q.device, stream)
+    code = lib().attn_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(lse), _ptr(dQ),
+                          _ptr(dK), _ptr(dV), B, Hq, Hkv, Lq, Lk, d, float(scale),
+                          ATTN_MASK_CAUSAL if causal else ATTN_MASK_NONE, _ptr(k_lens),
+                          _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(code, "attn_bwd")
+    return dQ, dK, dV

@@ -1,0 +1,258 @@
+// attn_api.cu -- the C ABI (include/attn.h): argument validation, tensor-map
+// encoding, grid planning and kernel launches on the caller's stream.  It
+// allocates no memory and never synchronises (attn_read_device_status aside).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "bwd_kernel.cuh"
+#include "decode_kernel.cuh"
+#include "fwd_kernel.cuh"
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;  // status word + scheduler counters, 256-byte aligned
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 view [heads][rows][d] of a [B, H, L, d] tensor, boxes of
+// 64 columns x `box_rows` rows x 1 head, 128-byte swizzle.
+bool make_tmap(CUtensorMap* m, const void* base, int d, int L, long long heads, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L > 0 ? L : 1),
+                        static_cast<cuuint64_t>(heads)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(d) * 2 * static_cast<cuuint64_t>(L > 0 ? L : 1)};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+bool shapes_ok(int B, int Hq, int Hkv, int Lq, int Lk) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 0 || Lk < 0) return false;
+  if (Hq % Hkv != 0) return false;
+  // every element index must fit the kernels' 64-bit offsets and the tensor
+  // maps' 32-bit coordinates
+  if (static_cast<long long>(B) * Hq > (1LL << 30)) return false;
+  if (Lq > (1 << 30) || Lk > (1 << 30)) return false;
+  return true;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_string(attn_status_t s) {
+  switch (s) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported";
+    case ATTN_ERR_CUDA: return "cuda error";
+    case ATTN_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+int attn_num_sms(void) { return device_sms(); }
+
+// ------------------------------------------------------------------ forward
+
+size_t attn_fwd_workspace_size(int, int, int, int, int, int) { return kStatusBytes; }
+
+attn_status_t attn_fwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf16_t* V,
+                       attn_bf16_t* O, float* lse, int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                       float scale, int mask_flags, const int32_t* k_lens, void* workspace,
+                       size_t ws_bytes, void* stream) {
+  if (!shapes_ok(B, Hq, Hkv, Lq, Lk)) return ATTN_ERR_INVALID;
+  if (!Q || !K || !V || !O || !workspace) return ATTN_ERR_INVALID;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) ||
+      (lse && !aligned16(lse)) || (k_lens && !aligned16(k_lens)) || !aligned256(workspace))
+    return ATTN_ERR_INVALID;
+  if (!(std::isfinite(scale) && scale > 0.f)) return ATTN_ERR_INVALID;
+  if (mask_flags != ATTN_MASK_NONE && mask_flags != ATTN_MASK_CAUSAL) return ATTN_ERR_INVALID;
+  if (ws_bytes < attn_fwd_workspace_size(B, Hq, Hkv, Lq, Lk, d)) return ATTN_ERR_INVALID;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (Lq == 0) return ATTN_OK;
+
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, Q, d, Lq, static_cast<long long>(B) * Hq, 128) ||
+      !make_tmap(&tk, K, d, Lk, static_cast<long long>(B) * Hkv, 128) ||
+      !make_tmap(&tv, V, d, Lk, static_cast<long long>(B) * Hkv, 128))
+    return ATTN_ERR_CUDA;
+
+  attn_fwd_impl::Params p;
+  p.O = reinterpret_cast<__nv_bfloat16*>(O);
+  p.lse = lse;
+  p.k_lens = k_lens;
+  p.status = reinterpret_cast<int*>(workspace);
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Lq = Lq;
+  p.Lk = Lk;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = (mask_flags & ATTN_MASK_CAUSAL) ? 1 : 0;
+  p.n_pairs = (Lq + 2 * attn_fwd_impl::BM - 1) / (2 * attn_fwd_impl::BM);
+  p.n_items = B * Hq * p.n_pairs;
+  const int sms = device_sms();
+  if (sms <= 0) return ATTN_ERR_CUDA;
+  const int grid = p.n_items < sms ? p.n_items : sms;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (d == 128) {
+    constexpr int smem = attn_fwd_impl::Cfg<128>::SMEM_BYTES;
+    e = set_smem(attn_fwd_impl::fwd_kernel<128>, smem);
+    if (e == cudaSuccess)
+      attn_fwd_impl::fwd_kernel<128><<<grid, attn_fwd_impl::NTHREADS, smem, s>>>(tq, tk, tv, p);
+  } else {
+    constexpr int smem = attn_fwd_impl::Cfg<64>::SMEM_BYTES;
+    e = set_smem(attn_fwd_impl::fwd_kernel<64>, smem);
+    if (e == cudaSuccess)
+      attn_fwd_impl::fwd_kernel<64><<<grid, attn_fwd_impl::NTHREADS, smem, s>>>(tq, tk, tv, p);
+  }
+  if (e != cudaSuccess) return ATTN_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ decode
+
+size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d) {
+  return kStatusBytes + attn_decode_impl::partials_bytes(B, Hq, Hkv, Lmax, d);
+}
+
+attn_status_t attn_fwd_splitkv_decode(const attn_bf16_t* Q, const attn_bf16_t* Kc,
+                                      const attn_bf16_t* Vc, attn_bf16_t* O, float* lse, int B,
+                                      int Hq, int Hkv, int Lmax, int d, float scale,
+                                      const int32_t* k_lens, void* workspace, size_t ws_bytes,
+                                      void* stream) {
+  if (!shapes_ok(B, Hq, Hkv, 1, Lmax)) return ATTN_ERR_INVALID;
+  if (!Q || !Kc || !Vc || !O || !k_lens || !workspace) return ATTN_ERR_INVALID;
+  if (!aligned16(Q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(O) ||
+      (lse && !aligned16(lse)) || !aligned16(k_lens) || !aligned256(workspace))
+    return ATTN_ERR_INVALID;
+  if (!(std::isfinite(scale) && scale > 0.f)) return ATTN_ERR_INVALID;
+  if (ws_bytes < attn_decode_workspace_size(B, Hq, Hkv, Lmax, d)) return ATTN_ERR_INVALID;
+  if (d != 128 && d != 64) return ATTN_ERR_UNSUPPORTED;
+  if (!attn_decode_impl::supported_group(Hq / Hkv)) return ATTN_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = device_sms();
+  if (sms <= 0) return ATTN_ERR_CUDA;
+  cudaError_t e = attn_decode_impl::launch(
+      reinterpret_cast<const __nv_bfloat16*>(Q), reinterpret_cast<const __nv_bfloat16*>(Kc),
+      reinterpret_cast<const __nv_bfloat16*>(Vc), reinterpret_cast<__nv_bfloat16*>(O), lse, B, Hq,
+      Hkv, Lmax, d, scale, k_lens, reinterpret_cast<int*>(workspace),
+      reinterpret_cast<uint8_t*>(workspace) + kStatusBytes, sms, s);
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ backward
+
+size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d) {
+  return kStatusBytes + attn_bwd_impl::scratch_bytes(B, Hq, Hkv, Lq, Lk, d);
+}
+
+attn_status_t attn_bwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf16_t* V,
+                       const attn_bf16_t* O, const attn_bf16_t* dO, const float* lse,
+                       attn_bf16_t* dQ, attn_bf16_t* dK, attn_bf16_t* dV, int B, int Hq, int Hkv,
+                       int Lq, int Lk, int d, float scale, int mask_flags, const int32_t* k_lens,
+                       void* workspace, size_t ws_bytes, void* stream) {
+  if (!shapes_ok(B, Hq, Hkv, Lq, Lk)) return ATTN_ERR_INVALID;
+  if (!Q || !K || !V || !O || !dO || !lse || !dQ || !dK || !dV || !workspace)
+    return ATTN_ERR_INVALID;
+  const void* ptrs[] = {Q, K, V, O, dO, lse, dQ, dK, dV};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return ATTN_ERR_INVALID;
+  if ((k_lens && !aligned16(k_lens)) || !aligned256(workspace)) return ATTN_ERR_INVALID;
+  if (!(std::isfinite(scale) && scale > 0.f)) return ATTN_ERR_INVALID;
+  if (mask_flags != ATTN_MASK_NONE && mask_flags != ATTN_MASK_CAUSAL) return ATTN_ERR_INVALID;
+  if (ws_bytes < attn_bwd_workspace_size(B, Hq, Hkv, Lq, Lk, d)) return ATTN_ERR_INVALID;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (Lq == 0 && Lk == 0) return ATTN_OK;
+  const int sms = device_sms();
+  if (sms <= 0) return ATTN_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  attn_bwd_impl::Args a;
+  a.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
+  a.K = reinterpret_cast<const __nv_bfloat16*>(K);
+  a.V = reinterpret_cast<const __nv_bfloat16*>(V);
+  a.O = reinterpret_cast<const __nv_bfloat16*>(O);
+  a.dO = reinterpret_cast<const __nv_bfloat16*>(dO);
+  a.lse = lse;
+  a.dQ = reinterpret_cast<__nv_bfloat16*>(dQ);
+  a.dK = reinterpret_cast<__nv_bfloat16*>(dK);
+  a.dV = reinterpret_cast<__nv_bfloat16*>(dV);
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Lq = Lq;
+  a.Lk = Lk;
+  a.d = d;
+  a.scale = scale;
+  a.causal = (mask_flags & ATTN_MASK_CAUSAL) ? 1 : 0;
+  a.k_lens = k_lens;
+  a.status = reinterpret_cast<int*>(workspace);
+  a.scratch = reinterpret_cast<uint8_t*>(workspace) + kStatusBytes;
+  a.sms = sms;
+  return attn_bwd_impl::launch(a, s);
+}
+
+// ------------------------------------------------------------------ status
+
+attn_status_t attn_read_device_status(const void* workspace, void* stream, int32_t* bits) {
+  if (!workspace) return ATTN_ERR_INVALID;
+  int32_t v = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (bits) *bits = v;
+  if (v & ATTN_DEV_TIMEOUT) return ATTN_ERR_TIMEOUT;
+  if (v & ATTN_DEV_BAD_KLEN) return ATTN_ERR_INVALID;
+  return ATTN_OK;
+}
+
+attn_status_t attn_clear_device_status(void* workspace, void* stream) {
+  if (!workspace) return ATTN_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return cudaMemsetAsync(workspace, 0, kStatusBytes, s) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,423 @@
+// decode_kernel.cuh -- split-KV decode (one query token per sequence).
+//
+// Decode is the "short query scans a long history" case of "FlashAttention and
+// long context: three ledgers" (prefill vs decode): per step the whole cache
+// row range [0, k_len) is read once and the arithmetic per byte is tiny
+// (4 FLOP/B with 4 query heads per key/value head), so the kernel is bound by
+// HBM bandwidth, not by the tensor core.  It therefore runs on CUDA cores:
+//
+//  * split kernel: one CTA per (sequence, key/value head, chunk of CH keys).
+//    A producer thread streams the chunk's K and V rows (contiguous in the
+//    cache) with 1-D bulk copies into a ring of shared-memory stages; four
+//    compute warps each own 16 rows of every stage.  A half-warp covers one
+//    key row (16 lanes x d/16 elements), forms partial dot products with all
+//    query heads of the group (packed fp32x2 FMA), and a transpose-reduction
+//    across the 16 lanes leaves every lane with one complete (row, head)
+//    score.  The online softmax of page 1 runs per warp with a stale-max
+//    rescale threshold; warps are merged at the end and the chunk's
+//    normalised output and log2-sum-exp are written as a partial.
+//  * combine kernel: merges a sequence's partials with the normalised rule of
+//    the FlashAttention-2 tutorial, 2.1.3.  Writing each partial as
+//    (O_c, LSE_c) with e^{LSE_c} = e^{m_c} l_c gives exactly that rule's
+//    weights: O = sum_c e^{LSE_c - M} O_c / sum_c e^{LSE_c - M}.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace attn_decode_impl {
+
+constexpr int CH = 1024;  // keys per split
+constexpr int SR = 64;    // key rows per shared-memory stage
+constexpr int NST = 3;    // stages
+constexpr int NCW = 4;    // compute warps
+constexpr int NTHREADS = (NCW + 1) * 32;
+
+inline bool supported_group(int G) { return G == 1 || G == 2 || G == 4 || G == 8; }
+
+inline int n_split_max(int Lmax) { return Lmax > 0 ? (Lmax + CH - 1) / CH : 1; }
+
+inline size_t partials_bytes(int B, int Hq, int, int Lmax, int d) {
+  const size_t n = static_cast<size_t>(B) * Hq * n_split_max(Lmax);
+  size_t bytes = n * d * 4 + n * 4;
+  return (bytes + 255) & ~static_cast<size_t>(255);
+}
+
+template <int D>
+constexpr int smem_bytes() {
+  return NST * SR * D * 2 * 2 + 256;
+}
+
+struct SplitParams {
+  const __nv_bfloat16* Q;
+  const __nv_bfloat16* K;
+  const __nv_bfloat16* V;
+  const int* k_lens;
+  int* status;
+  float* part_o;    // [B*Hq][nsm][D] normalised chunk outputs
+  float* part_lse;  // [B*Hq][nsm] log2-sum-exp of the chunk (scaled scores)
+  int B, Hq, Hkv, G, Lmax, nsm;
+  float scale_log2;
+};
+
+__device__ __forceinline__ int valid_klen(const int* k_lens, int b, int Lmax, int* status,
+                                          bool report) {
+  int kl = __ldg(k_lens + b);
+  if (kl < 0 || kl > Lmax) {
+    if (report) atomicOr(status, 1);
+    kl = 0;
+  }
+  return kl;
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          sm100::smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(sm100::smem_u32(bar))
+      : "memory");
+}
+
+// bf16x2 word -> two floats (exact widening)
+__device__ __forceinline__ float2 bf2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// One stage of the transpose-reduction: lanes whose bit `O` is clear keep the
+// lower half of their N values, the others the upper half; each adds the half
+// its partner (lane ^ O) gives away.
+template <int O, int N>
+__device__ __forceinline__ void tr_stage(float (&v)[16], bool upper) {
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) {
+    const float send = upper ? v[i] : v[i + N / 2];
+    const float keep = upper ? v[i + N / 2] : v[i];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+  }
+}
+
+// Transpose-reduction of 16 values per lane across the 16 lanes of a
+// half-warp (15 shuffles instead of 64): afterwards lane hl holds the full sum
+// of value index hl.
+__device__ __forceinline__ float transpose_reduce16(float (&v)[16], int hl) {
+  tr_stage<8, 16>(v, (hl & 8) != 0);
+  tr_stage<4, 8>(v, (hl & 4) != 0);
+  tr_stage<2, 4>(v, (hl & 2) != 0);
+  tr_stage<1, 2>(v, (hl & 1) != 0);
+  return v[0];
+}
+
+// GP: query heads per key/value head, padded to 4 or 8 (heads >= G are inert).
+template <int D, int GP>
+__global__ void __launch_bounds__(NTHREADS, 2) decode_split_kernel(const SplitParams p) {
+  constexpr int EPL = D / 16;    // elements of a row per lane
+  constexpr int R = 16 / GP;     // rows per half-warp per step
+  constexpr int STEP = 2 * R;    // rows per warp per step
+  constexpr int WROWS = SR / NCW;
+  constexpr int ROWB = D * 2;    // bytes per row
+  constexpr int STAGE = SR * ROWB;  // bytes of K (or V) per stage
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + NST * STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + 2 * NST * STAGE);
+  uint64_t* empty = full + NST;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NST);
+
+  const int chunk = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
+  const int kl = valid_klen(p.k_lens, b, p.Lmax, p.status, chunk == 0 && hkv == 0 && threadIdx.x == 0);
+  const int k0 = chunk * CH;
+  if (k0 >= kl) return;
+  const int rows = min(CH, kl - k0);
+  const int nstages = (rows + SR - 1) / SR;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NST; ++i) {
+      sm100::mbar_init(&full[i], 1);
+      sm100::mbar_init(&empty[i], NCW);
+    }
+    *abort_flag = 0;
+    sm100::fence_barrier_init();
+  }
+  __syncthreads();
+
+  const size_t head_row0 = (static_cast<size_t>(b) * p.Hkv + hkv) * p.Lmax + k0;
+  if (warp == NCW) {
+    if (lane == 0) {
+      const uint8_t* gK = reinterpret_cast<const uint8_t*>(p.K) + head_row0 * ROWB;
+      const uint8_t* gV = reinterpret_cast<const uint8_t*>(p.V) + head_row0 * ROWB;
+      for (int s = 0; s < nstages; ++s) {
+        const int slot = s % NST;
+        if (!sm100::mbar_wait(&empty[slot], ((s / NST) & 1) ^ 1, abort_flag, p.status)) break;
+        const int n = min(SR, rows - s * SR);
+        const uint32_t bytes = static_cast<uint32_t>(n * ROWB);
+        sm100::mbar_arrive_expect_tx(&full[slot], 2 * bytes);
+        bulk_g2s(sK + slot * STAGE, gK + static_cast<size_t>(s) * STAGE, bytes, &full[slot]);
+        bulk_g2s(sV + slot * STAGE, gV + static_cast<size_t>(s) * STAGE, bytes, &full[slot]);
+      }
+    }
+    return;  // the producer takes no part in the merge below
+  }
+
+  // ---------------------------------------------------------------- compute warps
+  const int half = lane >> 4, hl = lane & 15;
+  const int g_own = hl % GP;        // head of this lane's score
+  const int i_own = hl / GP;        // row (within the half's R rows) of this lane's score
+
+  // q of every head in the group, pre-scaled by scale * log2(e)
+  float2 q2[GP][EPL / 2];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    if (g < p.G) {
+      const __nv_bfloat16* qp =
+          p.Q + (static_cast<size_t>(b) * p.Hq + hkv * p.G + g) * D + hl * EPL;
+      const uint32_t* qw = reinterpret_cast<const uint32_t*>(qp);
+#pragma unroll
+      for (int c = 0; c < EPL / 2; ++c) {
+        const float2 f = bf2(__ldg(qw + c));
+        q2[g][c] = make_float2(f.x * p.scale_log2, f.y * p.scale_log2);
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < EPL / 2; ++c) q2[g][c] = make_float2(0.f, 0.f);
+    }
+  }
+
+  float2 o2[GP][EPL / 2];
+#pragma unroll
+  for (int g = 0; g < GP; ++g)
+#pragma unroll
+    for (int c = 0; c < EPL / 2; ++c) o2[g][c] = make_float2(0.f, 0.f);
+  float m_run = -INFINITY, l_lane = 0.f;
+  bool ok = true;
+
+  for (int s = 0; s < nstages && ok; ++s) {
+    const int slot = s % NST;
+    if (!(ok = sm100::mbar_wait(&full[slot], (s / NST) & 1, abort_flag, p.status))) break;
+    const int n = min(SR, rows - s * SR);
+    const uint8_t* kst = sK + slot * STAGE;
+    const uint8_t* vst = sV + slot * STAGE;
+#pragma unroll 1
+    for (int rb = warp * WROWS; rb < warp * WROWS + WROWS; rb += STEP) {
+      if (rb >= n) break;
+      // ---- scores: partial dots of this lane's d-slice, then transpose-reduce
+      float part[16];
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        const int row = rb + half * R + i;
+        uint32_t kw[EPL / 2];
+        if (row < n) {
+          if constexpr (EPL == 8) {
+            const uint4 t = *reinterpret_cast<const uint4*>(kst + row * ROWB + hl * 16);
+            kw[0] = t.x; kw[1] = t.y; kw[2] = t.z; kw[3] = t.w;
+          } else {
+            const uint2 t = *reinterpret_cast<const uint2*>(kst + row * ROWB + hl * 8);
+            kw[0] = t.x; kw[1] = t.y;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < EPL / 2; ++c) kw[c] = 0u;
+        }
+        float2 kf[EPL / 2];
+#pragma unroll
+        for (int c = 0; c < EPL / 2; ++c) kf[c] = bf2(kw[c]);
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int c = 0; c < EPL / 2; ++c) acc = __ffma2_rn(q2[g][c], kf[c], acc);
+          part[i * GP + g] = acc.x + acc.y;
+        }
+      }
+      const float sc = transpose_reduce16(part, hl);
+      const int my_row = rb + half * R + i_own;
+      const float s2 = (my_row < n && g_own < p.G) ? sc : -INFINITY;
+
+      // ---- online softmax for this step's rows (per head: lanes sharing g_own)
+      float m_blk = s2;
+#pragma unroll
+      for (int o = GP; o < 32; o <<= 1) m_blk = fmaxf(m_blk, __shfl_xor_sync(0xffffffffu, m_blk, o));
+      const bool need = m_blk > m_run + 8.0f;
+      if (__any_sync(0xffffffffu, need)) {
+        const float m_new = fmaxf(m_run, m_blk);
+        const float alpha = (m_run == -INFINITY) ? 0.f : sm100::ex2(m_run - m_new);
+        l_lane *= alpha;
+        m_run = m_new;
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          const float a = __shfl_sync(0xffffffffu, alpha, g);
+          const float2 a2 = make_float2(a, a);
+#pragma unroll
+          for (int c = 0; c < EPL / 2; ++c) o2[g][c] = __fmul2_rn(o2[g][c], a2);
+        }
+      }
+      const float pv = (s2 == -INFINITY) ? 0.f : sm100::ex2(s2 - m_run);
+      l_lane += pv;
+
+      // ---- o += p V for this half's rows
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        const int row = rb + half * R + i;
+        uint32_t vw[EPL / 2];
+        if (row < n) {
+          if constexpr (EPL == 8) {
+            const uint4 t = *reinterpret_cast<const uint4*>(vst + row * ROWB + hl * 16);
+            vw[0] = t.x; vw[1] = t.y; vw[2] = t.z; vw[3] = t.w;
+          } else {
+            const uint2 t = *reinterpret_cast<const uint2*>(vst + row * ROWB + hl * 8);
+            vw[0] = t.x; vw[1] = t.y;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < EPL / 2; ++c) vw[c] = 0u;
+        }
+        float2 vf[EPL / 2];
+#pragma unroll
+        for (int c = 0; c < EPL / 2; ++c) vf[c] = bf2(vw[c]);
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          const float pg = __shfl_sync(0xffffffffu, pv, half * 16 + i * GP + g);
+          const float2 p2 = make_float2(pg, pg);
+#pragma unroll
+          for (int c = 0; c < EPL / 2; ++c) o2[g][c] = __ffma2_rn(p2, vf[c], o2[g][c]);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) sm100::mbar_arrive(&empty[slot]);
+  }
+
+  // ---------------------------------------------------------------- merge warps
+  // per head: l over the lanes sharing g_own; o over the two half-warps
+#pragma unroll
+  for (int o = GP; o < 32; o <<= 1) l_lane += __shfl_xor_sync(0xffffffffu, l_lane, o);
+#pragma unroll
+  for (int g = 0; g < GP; ++g)
+#pragma unroll
+    for (int c = 0; c < EPL / 2; ++c) {
+      o2[g][c].x += __shfl_xor_sync(0xffffffffu, o2[g][c].x, 16);
+      o2[g][c].y += __shfl_xor_sync(0xffffffffu, o2[g][c].y, 16);
+    }
+  // all stages are consumed: reuse the K ring for the per-warp partials
+  sm100::named_bar_sync(1, NCW * 32);
+  float* wm = reinterpret_cast<float*>(sK);        // [NCW][GP]
+  float* wl = wm + NCW * GP;                       // [NCW][GP]
+  float* wo = wl + NCW * GP;                       // [NCW][GP][D]
+  if (lane < GP) {  // lane g (half 0, row 0) owns head g's statistics
+    wm[warp * GP + lane] = ok ? m_run : -INFINITY;
+    wl[warp * GP + lane] = ok ? l_lane : 0.f;
+  }
+  if (half == 0) {
+#pragma unroll
+    for (int g = 0; g < GP; ++g)
+#pragma unroll
+      for (int c = 0; c < EPL / 2; ++c) {
+        wo[(warp * GP + g) * D + hl * EPL + 2 * c] = o2[g][c].x;
+        wo[(warp * GP + g) * D + hl * EPL + 2 * c + 1] = o2[g][c].y;
+      }
+  }
+  sm100::named_bar_sync(1, NCW * 32);
+  for (int e = threadIdx.x; e < p.G * D; e += NCW * 32) {
+    const int g = e / D, dd = e % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NCW; ++w) M = fmaxf(M, wm[w * GP + g]);
+    float lsum = 0.f, acc = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NCW; ++w) {
+        const float mw = wm[w * GP + g];
+        const float f = (mw == -INFINITY) ? 0.f : sm100::ex2(mw - M);
+        lsum += f * wl[w * GP + g];
+        acc += f * wo[(w * GP + g) * D + dd];
+      }
+    }
+    const size_t ph = (static_cast<size_t>(b) * p.Hq + hkv * p.G + g) * p.nsm + chunk;
+    p.part_o[ph * D + dd] = lsum > 0.f ? acc / lsum : 0.f;
+    if (dd == 0) p.part_lse[ph] = lsum > 0.f ? M + log2f(lsum) : -INFINITY;
+  }
+}
+
+struct CombineParams {
+  const float* part_o;
+  const float* part_lse;
+  const int* k_lens;
+  int* status;
+  __nv_bfloat16* O;
+  float* lse;
+  int Hq, Lmax, nsm;
+};
+
+template <int D>
+__global__ void __launch_bounds__(D) decode_combine_kernel(const CombineParams p) {
+  const int bh = blockIdx.x;
+  const int b = bh / p.Hq;
+  const int kl = valid_klen(p.k_lens, b, p.Lmax, p.status, false);
+  const int n = (kl + CH - 1) / CH;
+  const float* lp = p.part_lse + static_cast<size_t>(bh) * p.nsm;
+  float M = -INFINITY;
+  for (int c = 0; c < n; ++c) M = fmaxf(M, lp[c]);
+  float wsum = 0.f, acc = 0.f;
+  if (M != -INFINITY) {
+    const float* op = p.part_o + static_cast<size_t>(bh) * p.nsm * D + threadIdx.x;
+    for (int c = 0; c < n; ++c) {
+      const float w = (lp[c] == -INFINITY) ? 0.f : sm100::ex2(lp[c] - M);
+      wsum += w;
+      acc += w * op[static_cast<size_t>(c) * D];
+    }
+  }
+  p.O[static_cast<size_t>(bh) * D + threadIdx.x] = __float2bfloat16_rn(wsum > 0.f ? acc / wsum : 0.f);
+  if (threadIdx.x == 0 && p.lse)
+    p.lse[bh] = wsum > 0.f ? (M + log2f(wsum)) * 0.69314718055994531f : -INFINITY;
+}
+
+template <int D, int GP>
+cudaError_t launch_t(const SplitParams& sp, const CombineParams& cp, cudaStream_t s) {
+  constexpr int smem = smem_bytes<D>();
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, GP>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(sp.nsm, sp.Hkv, sp.B);
+  decode_split_kernel<D, GP><<<grid, NTHREADS, smem, s>>>(sp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  decode_combine_kernel<D><<<sp.B * sp.Hq, D, 0, s>>>(cp);
+  return cudaGetLastError();
+}
+
+inline cudaError_t launch(const __nv_bfloat16* Q, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                          __nv_bfloat16* O, float* lse, int B, int Hq, int Hkv, int Lmax, int d,
+                          float scale, const int* k_lens, int* status, uint8_t* scratch, int,
+                          cudaStream_t s) {
+  SplitParams sp;
+  sp.Q = Q;
+  sp.K = K;
+  sp.V = V;
+  sp.k_lens = k_lens;
+  sp.status = status;
+  sp.nsm = n_split_max(Lmax);
+  const size_t n = static_cast<size_t>(B) * Hq * sp.nsm;
+  sp.part_o = reinterpret_cast<float*>(scratch);
+  sp.part_lse = reinterpret_cast<float*>(scratch + n * d * 4);
+  sp.B = B;
+  sp.Hq = Hq;
+  sp.Hkv = Hkv;
+  sp.G = Hq / Hkv;
+  sp.Lmax = Lmax;
+  sp.scale_log2 = scale * 1.4426950408889634f;
+  CombineParams cp;
+  cp.part_o = sp.part_o;
+  cp.part_lse = sp.part_lse;
+  cp.k_lens = k_lens;
+  cp.status = status;
+  cp.O = O;
+  cp.lse = lse;
+  cp.Hq = Hq;
+  cp.Lmax = Lmax;
+  cp.nsm = sp.nsm;
+  const bool wide = sp.G > 4;
+  if (d == 128) return wide ? launch_t<128, 8>(sp, cp, s) : launch_t<128, 4>(sp, cp, s);
+  return wide ? launch_t<64, 8>(sp, cp, s) : launch_t<64, 4>(sp, cp, s);
+}
+
+}  // namespace attn_decode_impl

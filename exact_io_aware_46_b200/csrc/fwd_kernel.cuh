@@ -1,0 +1,420 @@
+// fwd_kernel.cuh -- forward attention on sm_100a.
+//
+// Computes O = softmax((Q K^T + M) * scale) V and the per-row log-sum-exp with
+// the online softmax of "FlashAttention and long context: three ledgers"
+// (section "the key of FlashAttention is online softmax"): per query row keep
+// the running max m, the sum l relative to m and the unnormalised output o;
+// for each key/value tile rescale l and o by e^{m - m'} and add the tile's
+// e^{S - m'} and e^{S - m'} V; finally O = o / l.  Tiles of Q, K and V are
+// staged on chip (the tiling of the FlashAttention-2 tutorial, 2.1.2), so the
+// score and probability tiles live only in tensor memory and registers.
+//
+// B200 design (not the A100/Hopper designs the pages describe):
+//  * persistent CTAs, one per SM, walking a heaviest-first list of work items;
+//    an item is a pair of 128-row query tiles of one (batch, head);
+//  * warp 8 streams K and V tiles with TMA (128-byte swizzle) into a ring of
+//    shared-memory slots; the two query tiles are loaded once per item;
+//  * warp 9 owns tensor memory and one elected thread issues every tcgen05.mma:
+//    S_t = Q_t K_j^T (both operands in shared memory) into TMEM, and
+//    O_t += P_t V_j with P_t read from TMEM where the softmax wrote it over S_t;
+//  * warps 0-3 and 4-7 are two softmax warpgroups, one per query tile, so the
+//    tensor core computes one tile's scores while the other tile's softmax
+//    runs (ping-pong).  Each thread owns one query row (= one TMEM lane).
+//  * the running max is kept in the log2 domain and is only moved when a row's
+//    new max exceeds it by more than 8 (a factor 256): o and l only need a
+//    common reference max, so a stale max is exact, and the O rescale in TMEM
+//    becomes rare.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace attn_fwd_impl {
+
+constexpr int BM = 128;        // query rows per tile (= TMEM lanes)
+constexpr int BN = 128;        // keys per key/value tile
+constexpr int NTHREADS = 320;  // 8 softmax warps + load warp + MMA warp
+constexpr int CHUNK_BYTES = 128 * 128;  // one 128-row x 64-column bf16 swizzle panel
+constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+
+template <int D>
+struct Cfg {
+  static constexpr int CHUNKS = D / 64;
+  static constexpr int TILE_BYTES = BM * D * 2;
+  static constexpr int NS = (D == 128) ? 4 : 8;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_KV = 2 * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_KV + NS * TILE_BYTES;
+  static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;  // barriers + alignment slack
+  // TMEM columns: S_0, S_1 (128 fp32 columns each; P_t overwrites the first
+  // 64 columns of S_t as packed bf16 pairs), then O_0, O_1 (D columns each)
+  __device__ static constexpr uint32_t s_col(int t) { return t * 128u; }
+  __device__ static constexpr uint32_t o_col(int t) { return 256u + t * D; }
+  static constexpr uint32_t IDESC_S = sm100::idesc_bf16_f32(128, BN, false, false);
+  static constexpr uint32_t IDESC_PV = sm100::idesc_bf16_f32(128, D, false, true);
+};
+
+struct Params {
+  __nv_bfloat16* O;
+  float* lse;
+  const int* k_lens;
+  int* status;
+  int B, Hq, Hkv, Lq, Lk;
+  float scale_log2;  // scale * log2(e)
+  int causal;
+  int n_pairs;  // ceil(Lq / 256)
+  int n_items;  // B * Hq * n_pairs
+};
+
+struct Item {
+  int b, h, row0;  // row0: first query row of tile 0; tile 1 starts at row0 + BM
+  int kv_len;
+  int n[2];  // key/value tiles each query tile visits
+  int nmax;
+};
+
+__device__ __forceinline__ int tiles_for(const Params& p, int row0, int kv_len) {
+  if (row0 >= p.Lq) return 0;
+  const int last = min(row0 + BM - 1, p.Lq - 1);
+  int hi = kv_len;
+  if (p.causal) hi = min(hi, last + (p.Lk - p.Lq) + 1);
+  return hi <= 0 ? 0 : (hi + BN - 1) / BN;
+}
+
+__device__ __forceinline__ Item get_item(const Params& p, int w, bool* bad) {
+  Item it;
+  const int BH = p.B * p.Hq;
+  const int pair = p.n_pairs - 1 - w / BH;  // latest rows first: heaviest under a causal mask
+  const int bh = w % BH;
+  it.b = bh / p.Hq;
+  it.h = bh % p.Hq;
+  it.row0 = pair * 2 * BM;
+  int kl = p.Lk;
+  if (p.k_lens) {
+    kl = __ldg(p.k_lens + it.b);
+    if (kl < 0 || kl > p.Lk) {
+      if (bad) *bad = true;
+      kl = 0;
+    }
+  }
+  it.kv_len = kl;
+  it.n[0] = tiles_for(p, it.row0, kl);
+  it.n[1] = tiles_for(p, it.row0 + BM, kl);
+  it.nmax = max(it.n[0], it.n[1]);
+  return it;
+}
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the 128-byte swizzle panels
+  const uint32_t raw_addr = sm100::smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+  const uint32_t sbase = sm100::smem_u32(smem);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = bars + C::NS;
+  uint64_t* q_full = bars + 2 * C::NS;
+  uint64_t* q_empty = q_full + 1;
+  uint64_t* s_full = q_full + 2;   // [2]
+  uint64_t* p_full = q_full + 4;   // [2]
+  uint64_t* o_full = q_full + 6;   // [2]
+  uint64_t* o_empty = q_full + 8;  // [2]
+  uint64_t* drain = q_full + 10;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 11);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NS; ++i) {
+      sm100::mbar_init(&kv_full[i], 1);
+      sm100::mbar_init(&kv_empty[i], 1);
+    }
+    sm100::mbar_init(q_full, 1);
+    sm100::mbar_init(q_empty, 1);
+    for (int t = 0; t < 2; ++t) {
+      sm100::mbar_init(&s_full[t], 1);
+      sm100::mbar_init(&p_full[t], 128);
+      sm100::mbar_init(&o_full[t], 1);
+      sm100::mbar_init(&o_empty[t], 128);
+    }
+    sm100::mbar_init(drain, 1);
+    *abort_flag = 0;
+    sm100::fence_barrier_init();
+  }
+  if (warp == 8 && sm100::lane_id() == 0) {
+    sm100::prefetch_tmap(&tmQ);
+    sm100::prefetch_tmap(&tmK);
+    sm100::prefetch_tmap(&tmV);
+  }
+  if (warp == 9) {
+    sm100::tmem_alloc(tmem_slot, 512);
+    sm100::tmem_relinquish();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (sm100::lane_id() == 0) {
+      uint32_t use = 0, qk = 0;
+      for (int w = blockIdx.x; w < p.n_items; w += gridDim.x, ++qk) {
+        const Item it = get_item(p, w, nullptr);
+        if (!sm100::mbar_wait(q_empty, (qk & 1) ^ 1, abort_flag, p.status)) break;
+        sm100::mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
+        const int qh = it.b * p.Hq + it.h;
+        for (int t = 0; t < 2; ++t)
+          for (int c = 0; c < C::CHUNKS; ++c)
+            sm100::tma_load_3d(&tmQ, q_full,
+                               smem + C::OFF_Q + t * C::TILE_BYTES + c * CHUNK_BYTES, c * 64,
+                               it.row0 + t * BM, qh);
+        const int kvh = it.b * p.Hkv + it.h / (p.Hq / p.Hkv);
+        bool ok = true;
+        for (int j = 0; j < it.nmax && ok; ++j) {
+          for (int kv = 0; kv < 2; ++kv, ++use) {
+            const int slot = use % C::NS;
+            if (!sm100::mbar_wait(&kv_empty[slot], ((use / C::NS) & 1) ^ 1, abort_flag,
+                                  p.status)) {
+              ok = false;
+              break;
+            }
+            sm100::mbar_arrive_expect_tx(&kv_full[slot], C::TILE_BYTES);
+            for (int c = 0; c < C::CHUNKS; ++c)
+              sm100::tma_load_3d(kv == 0 ? &tmK : &tmV, &kv_full[slot],
+                                 smem + C::OFF_KV + slot * C::TILE_BYTES + c * CHUNK_BYTES,
+                                 c * 64, j * BN, kvh);
+          }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (sm100::lane_id() == 0) {
+      uint32_t use = 0, qk = 0;
+      uint32_t sp_cnt[2] = {0, 0};  // P tiles consumed per query tile
+      bool ok = true;
+      const uint32_t q_addr = sbase + C::OFF_Q;
+      const uint32_t kv_addr = sbase + C::OFF_KV;
+
+      auto issue_s = [&](int t, int slot) {
+        const uint32_t qa = q_addr + t * C::TILE_BYTES;
+        const uint32_t ka = kv_addr + slot * C::TILE_BYTES;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * CHUNK_BYTES + (k & 3) * 32;
+          sm100::mma_ss(tmem + C::s_col(t), sm100::sdesc_sw128(qa + off, 16, 1024),
+                        sm100::sdesc_sw128(ka + off, 16, 1024), C::IDESC_S, k > 0);
+        }
+      };
+      auto issue_pv = [&](int t, int slot, bool acc) {
+        const uint32_t va = kv_addr + slot * C::TILE_BYTES;
+#pragma unroll
+        for (int k = 0; k < BN / 16; ++k) {
+          sm100::mma_ts(tmem + C::o_col(t), tmem + C::s_col(t) + k * 8,
+                        sm100::sdesc_sw128(va + k * 2048, CHUNK_BYTES, 1024), C::IDESC_PV,
+                        (acc || k > 0) ? 1u : 0u);
+        }
+      };
+
+      for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x, ++qk) {
+        const Item it = get_item(p, w, nullptr);
+        if (!(ok = sm100::mbar_wait(q_full, qk & 1, abort_flag, p.status))) break;
+        sm100::tc_fence_after();
+        const uint32_t oe_par = (qk & 1) ^ 1;
+        if (it.nmax > 0) {
+          const int ks = use % C::NS;
+          if (!(ok = sm100::mbar_wait(&kv_full[ks], (use / C::NS) & 1, abort_flag, p.status)))
+            break;
+          sm100::tc_fence_after();
+          for (int t = 0; t < 2; ++t)
+            if (it.n[t] > 0) {
+              issue_s(t, ks);
+              sm100::tc_commit(&s_full[t]);
+            }
+          sm100::tc_commit(&kv_empty[ks]);
+        }
+        for (int j = 0; j < it.nmax && ok; ++j) {
+          const uint32_t vuse = use + 2 * j + 1;
+          const int vs = vuse % C::NS;
+          const uint32_t kuse = vuse + 1;
+          const int ks = kuse % C::NS;
+          bool k_ready = false;
+          if (!(ok = sm100::mbar_wait(&kv_full[vs], (vuse / C::NS) & 1, abort_flag, p.status)))
+            break;
+          sm100::tc_fence_after();
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (j < it.n[t]) {
+              if (j == 0 && !(ok = sm100::mbar_wait(&o_empty[t], oe_par, abort_flag, p.status)))
+                break;
+              if (!(ok = sm100::mbar_wait(&p_full[t], sp_cnt[t] & 1, abort_flag, p.status)))
+                break;
+              ++sp_cnt[t];
+              sm100::tc_fence_after();
+              issue_pv(t, vs, j > 0);
+              if (j == it.n[t] - 1) sm100::tc_commit(&o_full[t]);
+            }
+            if (j + 1 < it.n[t]) {
+              if (!k_ready) {
+                if (!(ok = sm100::mbar_wait(&kv_full[ks], (kuse / C::NS) & 1, abort_flag,
+                                            p.status)))
+                  break;
+                sm100::tc_fence_after();
+                k_ready = true;
+              }
+              issue_s(t, ks);
+              sm100::tc_commit(&s_full[t]);
+            }
+          }
+          if (!ok) break;
+          if (k_ready) sm100::tc_commit(&kv_empty[ks]);
+          sm100::tc_commit(&kv_empty[vs]);
+        }
+        if (!ok) break;
+        for (int t = 0; t < 2; ++t)
+          if (it.n[t] == 0) {
+            if (!(ok = sm100::mbar_wait(&o_empty[t], oe_par, abort_flag, p.status))) break;
+            sm100::tc_commit(&o_full[t]);
+          }
+        sm100::tc_commit(q_empty);
+        use += 2 * it.nmax;
+      }
+      // all issued tensor-core work (and its commits) must land before TMEM is freed
+      sm100::tc_commit(drain);
+      sm100::mbar_wait(drain, 0, abort_flag, p.status);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int t = warp >> 2;            // query tile of this warpgroup
+    const int r = threadIdx.x & 127;    // row within the tile = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_addr = tmem + lane_base + C::s_col(t);
+    const uint32_t o_addr = tmem + lane_base + C::o_col(t);
+    const float sl2 = p.scale_log2;
+    uint32_t s_cnt = 0, qk = 0;
+    bool ok = true;
+
+    for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x, ++qk) {
+      bool bad = false;
+      const Item it = get_item(p, w, &bad);
+      if (bad && threadIdx.x == 0) atomicOr(p.status, 1);
+      const int row0 = it.row0 + t * BM;
+      const int row = row0 + r;
+      const int diag = row + (p.Lk - p.Lq);  // last visible key under the causal mask
+      float m_use = -INFINITY, l = 0.f;
+      for (int j = 0; j < it.n[t]; ++j) {
+        if (!(ok = sm100::mbar_wait(&s_full[t], s_cnt & 1, abort_flag, p.status))) break;
+        ++s_cnt;
+        sm100::tc_fence_after();
+        uint32_t s[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          sm100::tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
+        sm100::tmem_ld_wait();
+
+        const int k0 = j * BN;
+        const bool need_mask =
+            (k0 + BN > it.kv_len) || (p.causal && (k0 + BN - 1 > row0 + (p.Lk - p.Lq)));
+        if (need_mask) {
+          const int lim = p.causal ? min(it.kv_len - 1, diag) : it.kv_len - 1;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (k0 + c > lim) s[c] = __float_as_uint(-INFINITY);
+        }
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          mx0 = fmaxf(mx0, __uint_as_float(s[c]));
+          mx1 = fmaxf(mx1, __uint_as_float(s[c + 1]));
+        }
+        const float m_new = fmaxf(mx0, mx1) * sl2;
+        const bool need = m_new > m_use + RESCALE_THRESHOLD;
+        if (__any_sync(0xffffffffu, need)) {
+          const float m_upd = fmaxf(m_use, m_new);
+          const float alpha = (m_use == -INFINITY) ? 0.f : sm100::ex2(m_use - m_upd);
+          l *= alpha;
+          if (j > 0) {
+            // O holds PV of the previous tiles (complete: S of this tile was
+            // committed after them); rescale it in place
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              sm100::tmem_ld32(o_addr + c * 32, o);
+              sm100::tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              sm100::tmem_st32(o_addr + c * 32, o);
+            }
+          }
+          m_use = m_upd;
+        }
+        const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
+        float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float p0 = sm100::ex2(fmaf(__uint_as_float(s[2 * c]), sl2, -m_sub));
+          const float p1 = sm100::ex2(fmaf(__uint_as_float(s[2 * c + 1]), sl2, -m_sub));
+          l0 += p0;
+          l1 += p1;
+          s[c] = sm100::pack_bf16x2(p0, p1);
+        }
+        l += l0 + l1;
+        sm100::tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        sm100::tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+        sm100::tmem_st_wait();
+        sm100::tc_fence_before();
+        sm100::mbar_arrive(&p_full[t]);
+      }
+      if (!ok) break;
+      // ---------------- epilogue: O = o / l (bf16), LSE = ln(2) * (m + log2 l)
+      if (!(ok = sm100::mbar_wait(&o_full[t], qk & 1, abort_flag, p.status))) break;
+      sm100::tc_fence_after();
+      const bool live = row < p.Lq;
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      __nv_bfloat16* orow =
+          p.O + ((static_cast<size_t>(it.b) * p.Hq + it.h) * p.Lq + (live ? row : 0)) * D;
+      if (it.n[t] > 0) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          sm100::tmem_ld32(o_addr + c * 32, o);
+          sm100::tmem_ld_wait();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = sm100::pack_bf16x2(__uint_as_float(o[2 * e]) * inv,
+                                       __uint_as_float(o[2 * e + 1]) * inv);
+          if (live) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+      } else if (live) {
+        uint4* dst = reinterpret_cast<uint4*>(orow);
+        for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0, 0, 0, 0);
+      }
+      if (live && p.lse)
+        p.lse[(static_cast<size_t>(it.b) * p.Hq + it.h) * p.Lq + row] =
+            (l > 0.f) ? (m_use + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      sm100::tc_fence_before();
+      sm100::mbar_arrive(&o_empty[t]);
+    }
+  }
+
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace attn_fwd_impl

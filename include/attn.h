@@ -1,0 +1,156 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) exact-attention library (libattn.so).
+ *
+ * The library computes exact dense scaled-dot-product attention
+ *
+ *     O = softmax((Q K^T + M) * scale) V
+ *
+ * ("FlashAttention and long context: three ledgers", section on why standard
+ * attention is not only a FLOP problem) tile by tile with the online softmax of
+ * the same page ("the key of FlashAttention is online softmax"), so the
+ * L_q x L_k score and probability matrices never reach device memory.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Element types: bf16 tensors are passed as `attn_bf16_t` (the raw 16-bit
+ *   bfloat16 pattern); statistics are IEEE fp32.
+ * - Layout: every tensor is contiguous row-major [batch, heads, length, d]
+ *   (the [batch, heads, n, d] layout of the FlashAttention-2 tutorial, 2.1.1).
+ *   Q, O, dO, dQ: [B, Hq, Lq, d]; K, V, dK, dV: [B, Hkv, Lk, d];
+ *   LSE: [B, Hq, Lq] fp32.  Query head h reads key/value head h / (Hq / Hkv)
+ *   (grouped-query attention; Hq must be a multiple of Hkv).
+ * - d (head dimension) must be 64 or 128; anything else returns
+ *   ATTN_ERR_UNSUPPORTED.  There is no fallback path of any kind.
+ * - All device pointers must be 16-byte aligned (the tensor-memory-accelerator
+ *   copies require it) and must not alias one another (except where stated).
+ * - Masks: `mask_flags` = ATTN_MASK_NONE or ATTN_MASK_CAUSAL.  Causal is
+ *   bottom-right aligned: key j is visible to query i iff j <= i + (Lk - Lq).
+ *   Key padding is selected by passing `k_lens` (device int32 [B]): key j of
+ *   sequence b is visible iff j < k_lens[b].  Both combine by AND.  A query row
+ *   with no visible key gets O = 0, LSE = -inf and zero gradients.
+ * - LSE is the natural-log log-sum-exp of the row's scaled, masked scores: the
+ *   per-row statistic the backward recomputes from (page 1: the backward keeps
+ *   small row statistics and recomputes score blocks).
+ * - Ownership: the caller allocates and owns every buffer, including the
+ *   workspace, and the stream.  The library never allocates, frees or
+ *   synchronises, except attn_read_device_status (which synchronises `stream`).
+ * - Asynchrony: every compute call enqueues kernels on `stream` (a
+ *   cudaStream_t; NULL = legacy default stream) and returns at once.
+ * - Errors: argument errors are detected on the host before anything is
+ *   launched and return ATTN_ERR_INVALID or ATTN_ERR_UNSUPPORTED.  A failed
+ *   launch returns ATTN_ERR_CUDA.  Errors found on the device (a k_lens entry
+ *   outside [0, Lk], an internal wait that timed out) set bits of a status
+ *   word kept in the first 16 bytes of the workspace; the affected work units
+ *   write zeros.  The word is sticky: read it with attn_read_device_status and
+ *   clear it with attn_clear_device_status (a fresh workspace must be cleared
+ *   once before first use).
+ * - Workspace: each call has an *_workspace_size query; pass at least that
+ *   many bytes, 256-byte aligned.  Calls that overlap in time on the device
+ *   must not share a workspace.
+ */
+#ifndef ATTN_H_
+#define ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t attn_bf16_t;
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID = 1,     /* bad pointer, size, alignment, or workspace too small */
+  ATTN_ERR_UNSUPPORTED = 2, /* valid request outside what the kernels implement */
+  ATTN_ERR_CUDA = 3,        /* a CUDA runtime/driver call or launch failed */
+  ATTN_ERR_TIMEOUT = 4      /* (device status) a bounded internal wait expired */
+} attn_status_t;
+
+enum { ATTN_MASK_NONE = 0, ATTN_MASK_CAUSAL = 1 };
+
+/* Device status bits (first int32 of every workspace). */
+enum { ATTN_DEV_BAD_KLEN = 1, ATTN_DEV_TIMEOUT = 2 };
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* attn_status_string(attn_status_t s);
+
+/* ------------------------------------------------------------------ forward
+ * Prefill / training forward.  Defined by the attention formula and the online
+ * softmax of page 1 (m' = max(m, max S_j); l' = e^{m-m'} l + sum e^{S_j-m'};
+ * o' = e^{m-m'} o + sum e^{S_j-m'} V_j; O = o / l), with the tiling of the
+ * FlashAttention-2 tutorial, 2.1.2.
+ *
+ *   Q [B,Hq,Lq,d], K/V [B,Hkv,Lk,d] bf16 (read only); O [B,Hq,Lq,d] bf16 and
+ *   lse [B,Hq,Lq] fp32 (written; lse may be NULL when not needed).
+ *   scale: multiplies Q K^T (the pages use 1/sqrt(d)); must be finite and > 0.
+ *   k_lens: device int32 [B] or NULL (no padding).
+ *   Lq, Lk >= 0 (Lq == 0 is a no-op).  B, Hq, Hkv >= 1.
+ */
+size_t attn_fwd_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d);
+attn_status_t attn_fwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf16_t* V,
+                       attn_bf16_t* O, float* lse, int B, int Hq, int Hkv, int Lq, int Lk,
+                       int d, float scale, int mask_flags, const int32_t* k_lens,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ decode
+ * Split-KV decode (one query token per sequence over a contiguous KV cache):
+ * the "short query scans a long history" case of page 1 (prefill vs decode).
+ * The cache rows [0, k_lens[b]) of each sequence are split into chunks; each
+ * chunk yields a partial (m, l, O) and the partials are combined with the
+ * normalised merge of the FlashAttention-2 tutorial, 2.1.3:
+ *   m = max(m_a, m_b); l = e^{m_a-m} l_a + e^{m_b-m} l_b;
+ *   O = (e^{m_a-m} l_a / l) O_a + (e^{m_b-m} l_b / l) O_b.
+ *
+ *   Q [B,Hq,1,d] bf16; Kcache/Vcache [B,Hkv,Lmax,d] bf16; k_lens device int32
+ *   [B], required, each in [0, Lmax] (no causal mask inside the cache).
+ *   O [B,Hq,1,d] bf16 and lse [B,Hq] fp32 (lse may be NULL).
+ *   The workspace holds the fp32 partials; its size depends on Lmax.
+ */
+size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d);
+attn_status_t attn_fwd_splitkv_decode(const attn_bf16_t* Q, const attn_bf16_t* Kcache,
+                                      const attn_bf16_t* Vcache, attn_bf16_t* O, float* lse,
+                                      int B, int Hq, int Hkv, int Lmax, int d, float scale,
+                                      const int32_t* k_lens, void* workspace, size_t ws_bytes,
+                                      void* stream);
+
+/* ------------------------------------------------------------------ backward
+ * Backward by recomputation: page 1 says the backward keeps only small row
+ * statistics and recomputes the score blocks it needs.  From the saved LSE
+ * (and D_i = sum_d dO_id O_id) each score tile is rebuilt as
+ * P = exp(S * scale - LSE), and
+ *   dV = P^T dO; dP = dO V^T; dS = P o (dP - D); dQ = scale dS K;
+ *   dK = scale dS^T Q  (summed over the Hq / Hkv query heads of a KV head).
+ *
+ *   Q, O, dO [B,Hq,Lq,d] bf16; K, V [B,Hkv,Lk,d] bf16; lse [B,Hq,Lq] fp32 as
+ *   written by attn_fwd for the same arguments.  dQ [B,Hq,Lq,d], dK, dV
+ *   [B,Hkv,Lk,d] bf16 are written.  Same mask arguments as attn_fwd.
+ *   The workspace holds fp32 accumulators for dQ and D.
+ */
+size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d);
+attn_status_t attn_bwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf16_t* V,
+                       const attn_bf16_t* O, const attn_bf16_t* dO, const float* lse,
+                       attn_bf16_t* dQ, attn_bf16_t* dK, attn_bf16_t* dV, int B, int Hq, int Hkv,
+                       int Lq, int Lk, int d, float scale, int mask_flags, const int32_t* k_lens,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ status
+ * Reads (after synchronising `stream`) the device status word of `workspace`:
+ * ATTN_OK when clear, ATTN_ERR_TIMEOUT if any wait expired, ATTN_ERR_INVALID
+ * if a k_lens entry was out of range.  *bits (may be NULL) receives the raw
+ * ATTN_DEV_* bits.  Returns ATTN_ERR_CUDA if the copy itself fails. */
+attn_status_t attn_read_device_status(const void* workspace, void* stream, int32_t* bits);
+
+/* Enqueues a clear of the status word on `stream`. */
+attn_status_t attn_clear_device_status(void* workspace, void* stream);
+
+/* Number of streaming multiprocessors the persistent kernels size their grids
+ * for (the current device's count); 0 when no device is visible. */
+int attn_num_sms(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H_ */

@@ -109,3 +109,46 @@ __all__ = [
     "to_torch_bf16",
     "workload_seed",
 ]
+
+
+# ---------------------------------------------------------------- device-side generation
+# The same counter-based splitmix64 + Box-Muller recipe written with torch
+# tensor ops, for workloads too large to draw on the host (the decode cache is
+# 8.6 GB).  The device's fp64 log/cos may differ from numpy's in the last ulp,
+# so the two generators agree except in rare rounding ties; tests of large
+# workloads therefore always hand the oracle the bits that were actually used
+# (copied back from the device).
+
+
+def _t_mix(x):
+    import torch
+
+    def srl(z, k):  # logical right shift of int64 bit patterns
+        return (z >> k) & ((1 << (64 - k)) - 1)
+
+    def c64(v):  # uint64 constant as a wrapped int64
+        return v - (1 << 64) if v >= (1 << 63) else v
+
+    z = x * c64(0x9E3779B97F4A7C15)
+    z = (z ^ srl(z, 30)) * c64(0xBF58476D1CE4E5B9)
+    z = (z ^ srl(z, 27)) * c64(0x94D049BB133111EB)
+    return z ^ srl(z, 31)
+
+
+def normal_bf16_device(seed: int, shape, device, chunk: int = 1 << 25):
+    """Device twin of :func:`normal_bf16`: returns a ``torch.bfloat16`` tensor."""
+    import torch
+
+    n = int(np.prod(shape)) if len(shape) else 1
+    out = torch.empty(n, dtype=torch.bfloat16, device=device)
+    base = (int(seed) & 0xFFFFFFFF) << 32
+    base = base - (1 << 64) if base >= (1 << 63) else base
+    for s in range(0, n, chunk):
+        m = min(chunk, n - s)
+        ctr = torch.arange(2 * s + 1, 2 * (s + m) + 1, dtype=torch.int64, device=device)
+        z = _t_mix(ctr + base)
+        u = (((z >> 11) & ((1 << 53) - 1)).to(torch.float64) + 1.0) * (2.0 ** -53)
+        u1, u2 = u[0::2], u[1::2]
+        x = torch.sqrt(-2.0 * torch.log(u1)) * torch.cos(2.0 * np.pi * u2)
+        out[s:s + m] = x.to(torch.float32).to(torch.bfloat16)
+    return out.view(*shape)

@@ -1,0 +1,105 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol,
+and rejects bad arguments on the host before launching anything."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from exact_io_aware_46_b200 import build
+
+    build.build()
+    import exact_io_aware_46_b200 as attn
+
+    return attn.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    import exact_io_aware_46_b200 as attn
+
+    names = _declared()
+    assert names, "no declarations parsed"
+    for n in names:
+        assert hasattr(lib, n), f"{n} missing from libattn.so"
+        assert n in attn.SIGNATURES, f"{n} has no binding signature"
+
+
+def test_workspace_sizes_are_closed_forms(lib):
+    import exact_io_aware_46_b200 as attn
+
+    assert attn.attn_fwd_workspace_size(4, 16, 16, 4096, 4096, 128) == 256
+    # decode: fp32 partial output and log-sum-exp per (sequence, head, 1024-key chunk)
+    n = 64 * 32 * 32
+    assert attn.attn_decode_workspace_size(64, 32, 8, 32768, 128) == 256 + ((n * 128 * 4 + n * 4 + 255) // 256) * 256
+    # backward: fp32 dQ accumulator and D per query row; nothing of size Lq x Lk
+    rows = 2 * 16 * 8192
+    assert attn.attn_bwd_workspace_size(2, 16, 16, 8192, 8192, 128) == 256 + ((rows * 128 * 4 + rows * 4 + 255) // 256) * 256
+
+
+def test_status_strings(lib):
+    import exact_io_aware_46_b200 as attn
+
+    assert attn.status_string(0) == "ok"
+    assert attn.status_string(2) == "unsupported"
+
+
+# Host-side validation happens before any CUDA call, so these run without a GPU.
+P = ctypes.c_void_p(256 * 1024)  # a 256-byte aligned non-null stand-in, never dereferenced
+
+
+def _fwd(lib, **kw):
+    a = dict(Q=P, K=P, V=P, O=P, lse=None, B=1, Hq=2, Hkv=1, Lq=8, Lk=8, d=128, scale=0.1,
+             mask=0, k_lens=None, ws=P, ws_bytes=256, stream=None)
+    a.update(kw)
+    return lib.attn_fwd(a["Q"], a["K"], a["V"], a["O"], a["lse"], a["B"], a["Hq"], a["Hkv"],
+                        a["Lq"], a["Lk"], a["d"], a["scale"], a["mask"], a["k_lens"], a["ws"],
+                        a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Q=None), 1), (dict(ws=None), 1), (dict(Hq=3, Hkv=2), 1), (dict(B=0), 1),
+    (dict(Lq=-1), 1), (dict(scale=0.0), 1), (dict(scale=float("nan")), 1), (dict(mask=7), 1),
+    (dict(ws_bytes=16), 1), (dict(Q=ctypes.c_void_p(256 * 1024 + 8)), 1),
+    (dict(ws=ctypes.c_void_p(256 * 1024 + 16)), 1),
+    (dict(d=96), 2), (dict(d=256), 2), (dict(Lq=0), 0),
+])
+def test_fwd_rejects_on_host(lib, kw, code):
+    assert _fwd(lib, **kw) == code
+
+
+def test_decode_and_bwd_reject_on_host(lib):
+    # decode: k_lens are required; G = 3 is not a supported group size
+    assert lib.attn_fwd_splitkv_decode(P, P, P, P, None, 1, 4, 1, 64, 128, 0.1, None, P,
+                                       1 << 20, None) == 1
+    assert lib.attn_fwd_splitkv_decode(P, P, P, P, None, 1, 3, 1, 64, 128, 0.1, P, P,
+                                       1 << 20, None) == 2
+    assert lib.attn_fwd_splitkv_decode(P, P, P, P, None, 1, 4, 1, 64, 72, 0.1, P, P,
+                                       1 << 20, None) == 2
+    # bwd: lse is required; d must be 64 or 128
+    assert lib.attn_bwd(P, P, P, P, P, None, P, P, P, 1, 1, 1, 8, 8, 128, 0.1, 0, None, P,
+                        1 << 20, None) == 1
+    assert lib.attn_bwd(P, P, P, P, P, P, P, P, P, 1, 1, 1, 8, 8, 80, 0.1, 0, None, P,
+                        1 << 20, None) == 2
+
+
+def test_product_path_does_not_touch_oracle():
+    """The CUDA binding must neither import nor load anything from oracle/."""
+    pkg = os.path.join(ROOT, "exact_io_aware_46_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt, f
+                assert "attn_oracle" not in txt, f

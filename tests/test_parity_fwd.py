@@ -1,0 +1,174 @@
+"""Forward parity: the CUDA kernel (through the C ABI) against the fp64 oracle."""
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests._util import (assert_lse_close, assert_out_close, bits, dev_bf16, to_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+def _lib():
+    import exact_io_aware_46_b200 as attn
+
+    return attn
+
+
+def _inputs(seed, B, Hq, Hkv, Lq, Lk, d):
+    Q = synth.normal_bf16(seed * 16 + 1, (B, Hq, Lq, d))
+    K = synth.normal_bf16(seed * 16 + 2, (B, Hkv, Lk, d))
+    V = synth.normal_bf16(seed * 16 + 3, (B, Hkv, Lk, d))
+    return Q, K, V
+
+
+def _run(Q, K, V, causal, k_lens=None, scale=None):
+    import torch
+
+    attn = _lib()
+    kl = None if k_lens is None else torch.tensor(k_lens, dtype=torch.int32, device="cuda")
+    O, L = attn.attn_fwd(dev_bf16(Q), dev_bf16(K), dev_bf16(V), scale=scale, causal=causal,
+                         k_lens=kl)
+    torch.cuda.synchronize()
+    return to_f64(O), to_f64(L)
+
+
+CASES = [
+    # B, Hq, Hkv, Lq, Lk, d, causal, k_lens
+    (1, 2, 2, 256, 256, 64, False, None),        # the tiny workload
+    (2, 3, 3, 421, 421, 128, True, None),        # several tiles, ragged tail
+    (1, 4, 2, 300, 300, 128, True, None),        # grouped-query heads
+    (2, 2, 2, 333, 333, 128, False, [200, 77]),  # key padding
+    (2, 2, 1, 333, 333, 64, True, [333, 129]),   # causal + padding, d = 64
+    (1, 2, 2, 100, 300, 128, True, None),        # Lq < Lk, bottom-right causal
+    (1, 2, 2, 300, 100, 128, True, None),        # Lq > Lk: leading rows see no key
+    (1, 1, 1, 1, 1, 128, False, None),           # single query, single key
+    (1, 2, 1, 129, 513, 64, False, None),        # one row past a tile, 4+ KV tiles
+    (1, 1, 1, 700, 700, 128, True, [0]),         # k_len = 0: every row empty
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,d,causal,k_lens", CASES)
+def test_fwd_matches_oracle(B, Hq, Hkv, Lq, Lk, d, causal, k_lens):
+    Q, K, V = _inputs(7 + Lq + Lk + d, B, Hq, Hkv, Lq, Lk, d)
+    scale = 1.0 / math.sqrt(d)
+    O, L = _run(Q, K, V, causal, k_lens, scale)
+    Oref, Lref = oracle.fwd(Q, K, V, scale, causal=causal, k_lens=k_lens)
+    assert_out_close(O, Oref)
+    assert_lse_close(L, Lref)
+
+
+def _scores_qkv(Lk, d, placed):
+    """One query whose scores (scale 1) against Lk keys are -1000 except at the
+    positions of ``placed`` {key index: score}; V row j = one-hot(j mod d)."""
+    Q = np.zeros((1, 1, 1, d))
+    Q[0, 0, 0, 0] = 1.0
+    K = np.zeros((1, 1, Lk, d))
+    K[0, 0, :, 0] = -1000.0
+    for j, s in placed.items():
+        K[0, 0, j, 0] = s
+    V = np.zeros((1, 1, Lk, d))
+    V[0, 0, np.arange(Lk), np.arange(Lk) % d] = 1.0
+    tobits = lambda x: synth.f64_to_bf16_bits(x)
+    return tobits(Q), tobits(K), tobits(V)
+
+
+def test_worked_example_across_two_key_tiles():
+    """Scores [2,5 | 1,4] of the FlashAttention-2 tutorial (2.1.9), with block A
+    in the first 128-key tile and block B in the second."""
+    placed = {126: 2.0, 127: 5.0, 128: 1.0, 129: 4.0}
+    Q, K, V = _scores_qkv(256, 128, placed)
+    O, L = _run(Q, K, V, False, scale=1.0)
+    p = O[0, 0, 0, [126 % 128, 127 % 128, 128 % 128, 129 % 128]]
+    assert np.max(np.abs(p - np.array([0.0347, 0.6964, 0.0128, 0.2562]))) <= 4e-3
+    Oref, Lref = oracle.fwd(Q, K, V, 1.0)
+    assert_out_close(O, Oref)
+    assert_lse_close(L, Lref)
+
+
+@pytest.mark.parametrize("c", [10.0, 20.0])
+def test_max_jump_in_third_tile(c):
+    """A later tile whose score jumps the running max (block C of 2.1.9): by 5
+    (stale-max path, under the rescale threshold) and by 15 (rescale path)."""
+    placed = {126: 2.0, 127: 5.0, 128: 1.0, 129: 4.0, 300: c}
+    Q, K, V = _scores_qkv(384, 128, placed)
+    O, L = _run(Q, K, V, False, scale=1.0)
+    Oref, Lref = oracle.fwd(Q, K, V, 1.0)
+    assert_out_close(O, Oref)
+    assert_lse_close(L, Lref)
+
+
+def test_fwd_deterministic():
+    import torch
+
+    attn = _lib()
+    Q, K, V = _inputs(99, 1, 2, 2, 600, 600, 128)
+    q, k, v = dev_bf16(Q), dev_bf16(K), dev_bf16(V)
+    O1, L1 = attn.attn_fwd(q, k, v, causal=True)
+    O2, L2 = attn.attn_fwd(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(O1, O2) and torch.equal(L1, L2)
+
+
+def test_bad_k_len_sets_status_and_zeroes():
+    import torch
+
+    attn = _lib()
+    Q, K, V = _inputs(5, 2, 1, 1, 130, 130, 64)
+    kl = torch.tensor([131, 50], dtype=torch.int32, device="cuda")
+    ws = torch.zeros(attn.attn_fwd_workspace_size(2, 1, 1, 130, 130, 64), dtype=torch.uint8,
+                     device="cuda")
+    O, L = attn.attn_fwd(dev_bf16(Q), dev_bf16(K), dev_bf16(V), k_lens=kl, workspace=ws)
+    code, st = attn.attn_read_device_status(ws)
+    assert code == attn.ATTN_ERR_INVALID and st & attn.ATTN_DEV_BAD_KLEN
+    assert torch.all(O[0] == 0) and torch.all(torch.isneginf(L[0]))
+    Oref, Lref = oracle.fwd(Q[1:], K[1:], V[1:], 1 / 8, k_lens=[50])
+    assert_out_close(to_f64(O[1:]), Oref)
+
+
+# ------------------------------------------------------------- full-size workloads (sampled)
+
+
+def _sample_rows(L, n, seed):
+    rng = np.random.default_rng(seed)
+    rows = set(range(min(128, L))) | set(range(max(0, L - 128), L))
+    rows |= set(rng.choice(L, size=min(n, L), replace=False).tolist())
+    return np.array(sorted(rows), dtype=np.int32)
+
+
+def _full_size_check(seed, B, Hq, Hkv, L, d, causal, k_lens, heads):
+    import torch
+
+    attn = _lib()
+    q = synth.normal_bf16_device(seed * 16 + 1, (B, Hq, L, d), "cuda")
+    k = synth.normal_bf16_device(seed * 16 + 2, (B, Hkv, L, d), "cuda")
+    v = synth.normal_bf16_device(seed * 16 + 3, (B, Hkv, L, d), "cuda")
+    kl = None if k_lens is None else torch.tensor(k_lens, dtype=torch.int32, device="cuda")
+    O, Lse = attn.attn_fwd(q, k, v, causal=causal, k_lens=kl)
+    torch.cuda.synchronize()
+    rows = _sample_rows(L, 64, seed)
+    G = Hq // Hkv
+    for b, h in heads:
+        Qh = bits(q[b:b + 1, h:h + 1])
+        Kh = bits(k[b:b + 1, h // G:h // G + 1])
+        Vh = bits(v[b:b + 1, h // G:h // G + 1])
+        kb = None if k_lens is None else [k_lens[b]]
+        Oref, Lref = oracle.fwd(Qh, Kh, Vh, 1 / math.sqrt(d), causal=causal, k_lens=kb,
+                                rows=rows)
+        assert_out_close(to_f64(O[b, h, rows]), Oref[0, 0], f"O[{b},{h}]")
+        assert_lse_close(to_f64(Lse[b, h, rows]), Lref[0, 0])
+
+
+def test_causal_prefill_full_size_sampled():
+    """B=4, H=16, L=4096, d=128, causal: sampled rows of sampled heads."""
+    _full_size_check(4602, 4, 16, 16, 4096, 128, True, None, [(0, 0), (1, 7), (3, 15), (2, 3)])
+
+
+@pytest.mark.parametrize("padded", [False, True])
+def test_long_context_gqa_full_size_sampled(padded):
+    """B=1, Hq=32, Hkv=8, L=16384, d=128, causal (+ a key-padding variant)."""
+    k_lens = [int(synth.uniform_int(4603 * 16 + 5, 1, 8192, 16384)[0])] if padded else None
+    _full_size_check(4603, 1, 32, 8, 16384, 128, True, k_lens, [(0, 0), (0, 13), (0, 31)])
