@@ -1,0 +1,479 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path on B200.
+
+Headline: causal prefill forward (B=4, H=16, L=4096, d=128, bf16) in TFLOP/s
+(causal FLOPs counted as half: 4 * d * visible (query, key) pairs) and its
+fraction of the measured dense bf16 tensor peak.  The same JSON line carries
+the split-KV decode leg (B=64, Hq=32, Hkv=8, cache 32768 x 128, k_len ~
+U[1024, 32768]) in HBM GB/s and, once available, the causal backward leg
+(B=2, H=16, L=8192, d=128) in TFLOP/s.
+
+Contract: ``python bench.py --gpus N --steps K --warmup W [--impl reference]``;
+under torchrun each rank runs an independent replica of the workload (no
+collective on the data path), the step time is the max over ranks and rank 0
+prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import signal
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "fwd attention TFLOP/s & % of BF16 tensor peak; decode KV-scan HBM GB/s"
+FWD = dict(B=4, Hq=16, Hkv=16, L=4096, d=128, causal=True)
+DEC = dict(B=64, Hq=32, Hkv=8, Lmax=32768, d=128, klo=1024)
+BWD = dict(B=2, Hq=16, Hkv=16, L=8192, d=128, causal=True)
+L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
+
+
+def causal_pairs(Lq, Lk, causal, k_len=None):
+    """Number of visible (query, key) pairs of one head."""
+    kl = Lk if k_len is None else k_len
+    if not causal:
+        return Lq * kl
+    off = Lk - Lq
+    i = np.arange(Lq, dtype=np.int64)
+    return int(np.clip(np.minimum(i + off + 1, kl), 0, None).sum())
+
+
+def fwd_flops(c):
+    return 4.0 * c["d"] * causal_pairs(c["L"], c["L"], c["causal"]) * c["B"] * c["Hq"]
+
+
+def bwd_flops(c):
+    return 10.0 * c["d"] * causal_pairs(c["L"], c["L"], c["causal"]) * c["B"] * c["Hq"]
+
+
+def peaks():
+    p = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+         "source": "fallback"}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        p.update({k: float(m[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")})
+        p["source"] = "measured"
+    except Exception:
+        pass
+    return p
+
+
+class Clocks:
+    """nvidia-smi sampler running during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.send_signal(signal.SIGTERM)
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) >= 9 and f[1].replace(".", "").isdigit():
+                    rows.append(f)
+        except Exception:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k] == "Active"})
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(rows[0][2]),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit()),
+                "samples": len(rows), "reasons": reasons}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+
+def dist_setup(n_gpus):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    import torch
+
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ legs
+
+
+def timed_loop(fn, steps, warmup, stream, flush_buf):
+    """Runs fn() warmup + steps times; each timed call is bracketed by CUDA events
+    on ``stream`` and preceded by an L2 flush.  Returns per-step ms list."""
+    import torch
+
+    for _ in range(warmup):
+        flush_buf.fill_(1)
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for s, e in ev:
+        flush_buf.fill_(1)
+        s.record(stream)
+        fn()
+        e.record(stream)
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in ev]
+
+
+def fwd_leg(steps, warmup, world, flush):
+    import torch
+
+    import exact_io_aware_46_b200 as attn
+
+    c = FWD
+    dev = torch.device("cuda")
+    q = synth.normal_bf16_device(synth.workload_seed(2, "q"), (c["B"], c["Hq"], c["L"], c["d"]), dev)
+    k = synth.normal_bf16_device(synth.workload_seed(2, "k"), (c["B"], c["Hkv"], c["L"], c["d"]), dev)
+    v = synth.normal_bf16_device(synth.workload_seed(2, "v"), (c["B"], c["Hkv"], c["L"], c["d"]), dev)
+    O = torch.empty_like(q)
+    lse = torch.empty((c["B"], c["Hq"], c["L"]), dtype=torch.float32, device=dev)
+    ws = torch.zeros(attn.attn_fwd_workspace_size(c["B"], c["Hq"], c["Hkv"], c["L"], c["L"], c["d"]),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    call = lambda: attn.attn_fwd(q, k, v, causal=True, O=O, lse=lse, workspace=ws, stream=stream)
+    barrier(world)
+    ms = timed_loop(call, steps, warmup, stream, flush)
+    st = attn.attn_read_device_status(ws)
+    if st[0] != attn.ATTN_OK:
+        raise RuntimeError(f"device status {st}")
+
+    # end to end: pinned host inputs -> device -> kernel -> host outputs, every step
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+    hL = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+    def e2e_call():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        call()
+        hO.copy_(O, non_blocking=True)
+        hL.copy_(lse, non_blocking=True)
+
+    barrier(world)
+    ms_e2e = timed_loop(e2e_call, max(3, steps // 2), 2, stream, flush)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = hO.numel() * hO.element_size() + hL.numel() * hL.element_size()
+    return ms, ms_e2e, h2d, d2h
+
+
+def decode_leg(steps, warmup, world, flush):
+    import torch
+
+    import exact_io_aware_46_b200 as attn
+
+    c = DEC
+    dev = torch.device("cuda")
+    k_lens = synth.uniform_int(synth.workload_seed(4, "klen"), c["B"], c["klo"], c["Lmax"])
+    q = synth.normal_bf16_device(synth.workload_seed(4, "q"), (c["B"], c["Hq"], 1, c["d"]), dev)
+    kc = synth.normal_bf16_device(synth.workload_seed(4, "k"), (c["B"], c["Hkv"], c["Lmax"], c["d"]), dev)
+    vc = synth.normal_bf16_device(synth.workload_seed(4, "v"), (c["B"], c["Hkv"], c["Lmax"], c["d"]), dev)
+    kl = torch.from_numpy(k_lens).to(dev)
+    O = torch.empty_like(q)
+    lse = torch.empty((c["B"], c["Hq"]), dtype=torch.float32, device=dev)
+    ws = torch.zeros(attn.attn_decode_workspace_size(c["B"], c["Hq"], c["Hkv"], c["Lmax"], c["d"]),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    call = lambda: attn.attn_fwd_splitkv_decode(q, kc, vc, kl, O=O, lse=lse, workspace=ws,
+                                                stream=stream)
+    barrier(world)
+    ms = timed_loop(call, steps, warmup, stream, flush)
+    st = attn.attn_read_device_status(ws)
+    if st[0] != attn.ATTN_OK:
+        raise RuntimeError(f"device status {st}")
+    kv_bytes = float(np.sum(k_lens.astype(np.int64))) * c["Hkv"] * c["d"] * 2 * 2
+    del kc, vc
+    torch.cuda.empty_cache()
+    return ms, kv_bytes, k_lens
+
+
+def bwd_leg(steps, warmup, world, flush):
+    import torch
+
+    import exact_io_aware_46_b200 as attn
+
+    c = BWD
+    dev = torch.device("cuda")
+    shp_q = (c["B"], c["Hq"], c["L"], c["d"])
+    shp_k = (c["B"], c["Hkv"], c["L"], c["d"])
+    q = synth.normal_bf16_device(synth.workload_seed(5, "q"), shp_q, dev)
+    k = synth.normal_bf16_device(synth.workload_seed(5, "k"), shp_k, dev)
+    v = synth.normal_bf16_device(synth.workload_seed(5, "v"), shp_k, dev)
+    do = synth.normal_bf16_device(synth.workload_seed(5, "do"), shp_q, dev)
+    O, lse = attn.attn_fwd(q, k, v, causal=True)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.zeros(attn.attn_bwd_workspace_size(c["B"], c["Hq"], c["Hkv"], c["L"], c["L"], c["d"]),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    call = lambda: attn.attn_bwd(q, k, v, O, do, lse, causal=True, dQ=dq, dK=dk, dV=dv,
+                                 workspace=ws, stream=stream)
+    try:
+        call()
+    except attn.AttnError as e:
+        if e.code == attn.ATTN_ERR_UNSUPPORTED:
+            return None
+        raise
+    barrier(world)
+    ms = timed_loop(call, steps, warmup, stream, flush)
+    st = attn.attn_read_device_status(ws)
+    if st[0] != attn.ATTN_OK:
+        raise RuntimeError(f"device status {st}")
+    return ms
+
+
+# ------------------------------------------------------------------ CPU baseline (oracle)
+
+
+def cpu_baseline(budget_s=12.0):
+    """The fp64 oracle on the host cores, on a bounded sample of the forward
+    workload: every 16th query row of head (0, 0), scaled by visible pairs."""
+    import oracle
+
+    c = FWD
+    L, d = c["L"], c["d"]
+    Q = synth.normal_bf16(synth.workload_seed(2, "q") ^ 0x55, (1, 1, L, d))
+    K = synth.normal_bf16(synth.workload_seed(2, "k") ^ 0x55, (1, 1, L, d))
+    V = synth.normal_bf16(synth.workload_seed(2, "v") ^ 0x55, (1, 1, L, d))
+    stride = 16
+    done_flops, t_used, reps = 0.0, 0.0, 0
+    while t_used < budget_s and reps < 64:
+        rows = np.arange(reps % stride, L, stride, dtype=np.int32)
+        t0 = time.perf_counter()
+        oracle.fwd(Q, K, V, 1 / math.sqrt(d), causal=True, rows=rows)
+        t_used += time.perf_counter() - t0
+        done_flops += 4.0 * d * float(np.sum(rows + 1))
+        reps += 1
+    return {"value": done_flops / t_used / 1e12, "unit": "TFLOP/s", "cores": oracle.threads(),
+            "kind": "oracle",
+            "sample": f"{reps} x {L // stride} query rows (every {stride}th) of one "
+                      f"(b,h) head of the causal B4 H16 L4096 d128 forward, fp64, "
+                      f"{t_used:.1f} s of CPU time"}
+
+
+def reference_arm(args, rank, world):
+    """--impl reference: the oracle, as it stands, on this machine's host cores."""
+    if rank != 0:
+        return
+    steps, warmup = args.steps, args.warmup
+    import oracle
+
+    c = FWD
+    L, d = c["L"], c["d"]
+    Q = synth.normal_bf16(synth.workload_seed(2, "q") ^ 0x55, (1, 1, L, d))
+    K = synth.normal_bf16(synth.workload_seed(2, "k") ^ 0x55, (1, 1, L, d))
+    V = synth.normal_bf16(synth.workload_seed(2, "v") ^ 0x55, (1, 1, L, d))
+    stride = 64
+    times, flops = [], []
+    for it in range(warmup + steps):
+        rows = np.arange(it % stride, L, stride, dtype=np.int32)
+        t0 = time.perf_counter()
+        oracle.fwd(Q, K, V, 1 / math.sqrt(d), causal=True, rows=rows)
+        dt = time.perf_counter() - t0
+        if it >= warmup:
+            times.append(dt)
+            flops.append(4.0 * d * float(np.sum(rows + 1)))
+    val = sum(flops) / sum(times) / 1e12
+    sample = (f"each step: {L // stride} query rows (every {stride}th) of one head of the causal "
+              f"B4 H16 L4096 d128 forward, fp64 oracle")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": steps, "warmup": warmup,
+        "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "causal prefill forward B4 H16 L4096 d128 (sampled rows)"},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": oracle.threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ------------------------------------------------------------------ main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--legs", default="fwd,decode,bwd")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        reference_arm(args, rank, world)
+        return
+
+    import torch
+
+    import exact_io_aware_46_b200 as attn
+
+    attn.lib()  # fail loudly if the CUDA library is missing
+    rank, world, local = dist_setup(args.gpus)
+    pk = peaks()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    legs = args.legs.split(",")
+    out = {}
+
+    gpu_idx = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]
+                  if os.environ.get("CUDA_VISIBLE_DEVICES") else local)
+    with Clocks(gpu_idx) as clk:
+        ms, ms_e2e, h2d, d2h = fwd_leg(args.steps, args.warmup, world, flush)
+        if "decode" in legs:
+            dms, kv_bytes, _ = decode_leg(args.steps, args.warmup, world, flush)
+        if "bwd" in legs:
+            bms = bwd_leg(max(3, args.steps // 2), args.warmup, world, flush)
+        else:
+            bms = None
+    clocks = clk.summary()
+
+    flops = fwd_flops(FWD)
+    t_step = max_over_ranks(float(np.mean(ms)), world)
+    t_e2e = max_over_ranks(float(np.mean(ms_e2e)), world)
+    value = world * flops / (t_step * 1e-3) / 1e12
+    achieved = flops / (float(np.mean(ms)) * 1e-3) / 1e12
+    launches = args.steps  # one persistent forward kernel per step
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "causal prefill forward B4 H16 L4096 d128 (bf16 in, fp32 "
+                               "accumulate, O bf16 + LSE fp32)",
+                   "B": FWD["B"], "H": FWD["Hq"], "L": FWD["L"], "d": FWD["d"], "causal": True,
+                   "flops_per_step": flops, "flop_count": "4*d*visible pairs (causal = half)",
+                   "l2": "flushed (256 MB write) before every timed call",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                     "peak_source": f"{pk['source']} burst bf16 (MEASURED_PEAKS.json)",
+                     "kernel": "attn_fwd_impl::fwd_kernel<128>"},
+        "e2e": {"value": world * flops / (t_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": t_e2e},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if "decode" in legs:
+        t_d = max_over_ranks(float(np.mean(dms)), world)
+        gbs = kv_bytes / (float(np.mean(dms)) * 1e-3) / 1e9
+        line["decode"] = {
+            "workload": "split-KV decode B64 Hq32 Hkv8 d128, cache 32768, k_len~U[1024,32768]",
+            "value": world * kv_bytes / (t_d * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": t_d,
+            "kv_bytes_per_step": kv_bytes,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "frac_of_8TBs": gbs / 8000.0,
+                         "traffic": None,
+                         "kernel": "attn_decode_impl::decode_split_kernel<128,4> + combine"},
+            "gpu_launches": 2 * args.steps,
+        }
+        line["gpu_launches"] += 2 * args.steps
+    if bms is not None:
+        bfl = bwd_flops(BWD)
+        t_b = max_over_ranks(float(np.mean(bms)), world)
+        ach = bfl / (float(np.mean(bms)) * 1e-3) / 1e12
+        line["bwd"] = {
+            "workload": "causal backward B2 H16 L8192 d128", "value": world * bfl / (t_b * 1e-3) / 1e12,
+            "unit": "TFLOP/s", "ms_per_step": t_b, "flops_per_step": bfl,
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"], "traffic": None},
+        }
+        line["gpu_launches"] += 3 * max(3, args.steps // 2)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -78,6 +78,11 @@ cudaError_t set_smem(K kernel, int bytes) {
 
 }  // namespace
 
+bool attn_bwd_impl::make_tmap_rows(CUtensorMap* m, const void* base, int L, long long heads,
+                                   int box_rows) {
+  return make_tmap(m, base, attn_bwd_impl::D, L, heads, box_rows);
+}
+
 extern "C" {
 
 const char* attn_status_string(attn_status_t s) {
@@ -123,6 +128,7 @@ attn_status_t attn_fwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf
   p.lse = lse;
   p.k_lens = k_lens;
   p.status = reinterpret_cast<int*>(workspace);
+  p.sched = reinterpret_cast<int*>(workspace) + 1;
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;

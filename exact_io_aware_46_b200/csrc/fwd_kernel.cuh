@@ -44,7 +44,7 @@ struct Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NS * TILE_BYTES;
-  static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;  // barriers + alignment slack
+  static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;  // barriers, item ring + alignment slack
   // TMEM columns: S_0, S_1 (128 fp32 columns each; P_t overwrites the first
   // 64 columns of S_t as packed bf16 pairs), then O_0, O_1 (D columns each)
   __device__ static constexpr uint32_t s_col(int t) { return t * 128u; }
@@ -57,7 +57,8 @@ struct Params {
   __nv_bfloat16* O;
   float* lse;
   const int* k_lens;
-  int* status;
+  int* status;  // device status word (workspace + 0)
+  int* sched;   // [0] next dynamic item, [1] finished CTAs (workspace + 4)
   int B, Hq, Hkv, Lq, Lk;
   float scale_log2;  // scale * log2(e)
   int causal;
@@ -68,9 +69,12 @@ struct Params {
 struct Item {
   int b, h, row0;  // row0: first query row of tile 0; tile 1 starts at row0 + BM
   int kv_len;
-  int n[2];  // key/value tiles each query tile visits
+  int n0, n1;  // key/value tiles each query tile visits
   int nmax;
 };
+
+constexpr int HEAD_GROUP = 8;  // heads whose items are interleaved (L2 reuse of their K/V)
+constexpr int NI = 4;          // depth of the shared-memory item ring
 
 __device__ __forceinline__ int tiles_for(const Params& p, int row0, int kv_len) {
   if (row0 >= p.Lq) return 0;
@@ -80,11 +84,19 @@ __device__ __forceinline__ int tiles_for(const Params& p, int row0, int kv_len) 
   return hi <= 0 ? 0 : (hi + BN - 1) / BN;
 }
 
+// Item order: groups of HEAD_GROUP (batch, head) pairs; inside a group the
+// latest query rows (heaviest under a causal mask) first, heads interleaved.
+// Grouping keeps the concurrently streamed K/V within a few heads (L2-resident)
+// while dynamic fetching keeps the heaviest-first property for load balance.
 __device__ __forceinline__ Item get_item(const Params& p, int w, bool* bad) {
   Item it;
   const int BH = p.B * p.Hq;
-  const int pair = p.n_pairs - 1 - w / BH;  // latest rows first: heaviest under a causal mask
-  const int bh = w % BH;
+  const int per_group = HEAD_GROUP * p.n_pairs;
+  const int g = w / per_group;
+  const int r = w % per_group;
+  const int gsize = min(HEAD_GROUP, BH - g * HEAD_GROUP);
+  const int pair = p.n_pairs - 1 - r / gsize;
+  const int bh = g * HEAD_GROUP + r % gsize;
   it.b = bh / p.Hq;
   it.h = bh % p.Hq;
   it.row0 = pair * 2 * BM;
@@ -97,14 +109,18 @@ __device__ __forceinline__ Item get_item(const Params& p, int w, bool* bad) {
     }
   }
   it.kv_len = kl;
-  it.n[0] = tiles_for(p, it.row0, kl);
-  it.n[1] = tiles_for(p, it.row0 + BM, kl);
-  it.nmax = max(it.n[0], it.n[1]);
+  it.n0 = tiles_for(p, it.row0, kl);
+  it.n1 = tiles_for(p, it.row0 + BM, kl);
+  it.nmax = max(it.n0, it.n1);
   return it;
 }
 
+// Polynomial (FMA-pipe) instead of MUFU exp2 for column pairs whose index
+// c / 2 satisfies (c / 2) % 4 == 3: a quarter of the exponentials.
+__device__ __forceinline__ constexpr bool poly_pair(int cp) { return (cp & 3) == 3; }
+
 template <int D>
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __maxnreg__(200)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const Params p) {
   using C = Cfg<D>;
@@ -124,7 +140,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* o_full = q_full + 6;   // [2]
   uint64_t* o_empty = q_full + 8;  // [2]
   uint64_t* drain = q_full + 10;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 11);
+  uint64_t* item_full = q_full + 11;   // [NI]
+  uint64_t* item_empty = q_full + 11 + NI;  // [NI]
+  int* item_ring = reinterpret_cast<int*>(q_full + 11 + 2 * NI);  // [NI]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_ring + NI);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -143,6 +162,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       sm100::mbar_init(&o_empty[t], 128);
     }
     sm100::mbar_init(drain, 1);
+    for (int i = 0; i < NI; ++i) {
+      sm100::mbar_init(&item_full[i], 1);
+      sm100::mbar_init(&item_empty[i], 1 + 256);  // the MMA thread + both softmax warpgroups
+    }
     *abort_flag = 0;
     sm100::fence_barrier_init();
   }
@@ -160,13 +183,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   sm100::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // consumers' view of the item ring: the k-th item index, or -1 at the end
+  auto next_item = [&](uint32_t k, int& w) -> bool {
+    if (!sm100::mbar_wait(&item_full[k % NI], (k / NI) & 1, abort_flag, p.status)) return false;
+    w = *reinterpret_cast<volatile int*>(&item_ring[k % NI]);
+    sm100::mbar_arrive(&item_empty[k % NI]);
+    return true;
+  };
+
   if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ scheduler + TMA producer
     if (sm100::lane_id() == 0) {
-      uint32_t use = 0, qk = 0;
-      for (int w = blockIdx.x; w < p.n_items; w += gridDim.x, ++qk) {
+      uint32_t use = 0;
+      for (uint32_t k = 0;; ++k) {
+        if (!sm100::mbar_wait(&item_empty[k % NI], ((k / NI) & 1) ^ 1, abort_flag, p.status))
+          break;
+        int w = (k == 0) ? static_cast<int>(blockIdx.x)
+                         : atomicAdd(p.sched, 1) + static_cast<int>(gridDim.x);
+        if (w >= p.n_items) w = -1;
+        *reinterpret_cast<volatile int*>(&item_ring[k % NI]) = w;
+        sm100::mbar_arrive(&item_full[k % NI]);
+        if (w < 0) break;
         const Item it = get_item(p, w, nullptr);
-        if (!sm100::mbar_wait(q_empty, (qk & 1) ^ 1, abort_flag, p.status)) break;
+        if (!sm100::mbar_wait(q_empty, (k & 1) ^ 1, abort_flag, p.status)) break;
         sm100::mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
         const int qh = it.b * p.Hq + it.h;
         for (int t = 0; t < 2; ++t)
@@ -197,8 +236,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (sm100::lane_id() == 0) {
-      uint32_t use = 0, qk = 0;
-      uint32_t sp_cnt[2] = {0, 0};  // P tiles consumed per query tile
+      uint32_t use = 0;
+      uint32_t pc0 = 0, pc1 = 0;  // P tiles consumed per query tile
       bool ok = true;
       const uint32_t q_addr = sbase + C::OFF_Q;
       const uint32_t kv_addr = sbase + C::OFF_KV;
@@ -223,21 +262,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       };
 
-      for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x, ++qk) {
+      for (uint32_t k = 0; ok; ++k) {
+        int w;
+        if (!(ok = next_item(k, w)) || w < 0) break;
         const Item it = get_item(p, w, nullptr);
-        if (!(ok = sm100::mbar_wait(q_full, qk & 1, abort_flag, p.status))) break;
+        if (!(ok = sm100::mbar_wait(q_full, k & 1, abort_flag, p.status))) break;
         sm100::tc_fence_after();
-        const uint32_t oe_par = (qk & 1) ^ 1;
+        const uint32_t oe_par = (k & 1) ^ 1;
         if (it.nmax > 0) {
           const int ks = use % C::NS;
           if (!(ok = sm100::mbar_wait(&kv_full[ks], (use / C::NS) & 1, abort_flag, p.status)))
             break;
           sm100::tc_fence_after();
-          for (int t = 0; t < 2; ++t)
-            if (it.n[t] > 0) {
-              issue_s(t, ks);
-              sm100::tc_commit(&s_full[t]);
-            }
+          if (it.n0 > 0) {
+            issue_s(0, ks);
+            sm100::tc_commit(&s_full[0]);
+          }
+          if (it.n1 > 0) {
+            issue_s(1, ks);
+            sm100::tc_commit(&s_full[1]);
+          }
           sm100::tc_commit(&kv_empty[ks]);
         }
         for (int j = 0; j < it.nmax && ok; ++j) {
@@ -249,45 +293,49 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!(ok = sm100::mbar_wait(&kv_full[vs], (vuse / C::NS) & 1, abort_flag, p.status)))
             break;
           sm100::tc_fence_after();
-          for (int t = 0; t < 2 && ok; ++t) {
-            if (j < it.n[t]) {
-              if (j == 0 && !(ok = sm100::mbar_wait(&o_empty[t], oe_par, abort_flag, p.status)))
-                break;
-              if (!(ok = sm100::mbar_wait(&p_full[t], sp_cnt[t] & 1, abort_flag, p.status)))
-                break;
-              ++sp_cnt[t];
+          // one query tile's step: O_t += P_t V_j, then S_t = Q_t K_{j+1}^T
+          auto step = [&](int t, int n_t, uint32_t& pc) -> bool {
+            if (j < n_t) {
+              if (j == 0 && !sm100::mbar_wait(&o_empty[t], oe_par, abort_flag, p.status))
+                return false;
+              if (!sm100::mbar_wait(&p_full[t], pc & 1, abort_flag, p.status)) return false;
+              ++pc;
               sm100::tc_fence_after();
               issue_pv(t, vs, j > 0);
-              if (j == it.n[t] - 1) sm100::tc_commit(&o_full[t]);
+              if (j == n_t - 1) sm100::tc_commit(&o_full[t]);
             }
-            if (j + 1 < it.n[t]) {
+            if (j + 1 < n_t) {
               if (!k_ready) {
-                if (!(ok = sm100::mbar_wait(&kv_full[ks], (kuse / C::NS) & 1, abort_flag,
-                                            p.status)))
-                  break;
+                if (!sm100::mbar_wait(&kv_full[ks], (kuse / C::NS) & 1, abort_flag, p.status))
+                  return false;
                 sm100::tc_fence_after();
                 k_ready = true;
               }
               issue_s(t, ks);
               sm100::tc_commit(&s_full[t]);
             }
-          }
-          if (!ok) break;
+            return true;
+          };
+          if (!(ok = step(0, it.n0, pc0))) break;
+          if (!(ok = step(1, it.n1, pc1))) break;
           if (k_ready) sm100::tc_commit(&kv_empty[ks]);
           sm100::tc_commit(&kv_empty[vs]);
         }
         if (!ok) break;
-        for (int t = 0; t < 2; ++t)
-          if (it.n[t] == 0) {
-            if (!(ok = sm100::mbar_wait(&o_empty[t], oe_par, abort_flag, p.status))) break;
-            sm100::tc_commit(&o_full[t]);
-          }
+        if (it.n0 == 0) {
+          if (!(ok = sm100::mbar_wait(&o_empty[0], oe_par, abort_flag, p.status))) break;
+          sm100::tc_commit(&o_full[0]);
+        }
+        if (it.n1 == 0) {
+          if (!(ok = sm100::mbar_wait(&o_empty[1], oe_par, abort_flag, p.status))) break;
+          sm100::tc_commit(&o_full[1]);
+        }
         sm100::tc_commit(q_empty);
         use += 2 * it.nmax;
       }
       // all issued tensor-core work (and its commits) must land before TMEM is freed
       sm100::tc_commit(drain);
-      sm100::mbar_wait(drain, 0, abort_flag, p.status);
+      sm100::mbar_wait_drain(drain, 0);
     }
   } else {
     // ------------------------------------------------------------ softmax warpgroups
@@ -297,18 +345,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t s_addr = tmem + lane_base + C::s_col(t);
     const uint32_t o_addr = tmem + lane_base + C::o_col(t);
     const float sl2 = p.scale_log2;
-    uint32_t s_cnt = 0, qk = 0;
+    const float2 sl2x2 = make_float2(sl2, sl2);
+    uint32_t s_cnt = 0;
     bool ok = true;
 
-    for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x, ++qk) {
+    for (uint32_t k = 0; ok; ++k) {
+      int w;
+      if (!(ok = next_item(k, w)) || w < 0) break;
       bool bad = false;
       const Item it = get_item(p, w, &bad);
       if (bad && threadIdx.x == 0) atomicOr(p.status, 1);
+      const int n_t = t ? it.n1 : it.n0;
       const int row0 = it.row0 + t * BM;
       const int row = row0 + r;
       const int diag = row + (p.Lk - p.Lq);  // last visible key under the causal mask
       float m_use = -INFINITY, l = 0.f;
-      for (int j = 0; j < it.n[t]; ++j) {
+      for (int j = 0; j < n_t; ++j) {
         if (!(ok = sm100::mbar_wait(&s_full[t], s_cnt & 1, abort_flag, p.status))) break;
         ++s_cnt;
         sm100::tc_fence_after();
@@ -329,9 +381,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          mx0 = fmaxf(mx0, __uint_as_float(s[c]));
-          mx1 = fmaxf(mx1, __uint_as_float(s[c + 1]));
+        for (int c = 0; c < 128; c += 4) {
+          mx0 = sm100::max3(mx0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+          mx1 = sm100::max3(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
         }
         const float m_new = fmaxf(mx0, mx1) * sl2;
         const bool need = m_new > m_use + RESCALE_THRESHOLD;
@@ -355,31 +407,43 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           m_use = m_upd;
         }
         const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
-        float l0 = 0.f, l1 = 0.f;
+        const float2 negm = make_float2(-m_sub, -m_sub);
+        float2 lsum = make_float2(0.f, 0.f);
+        // exponentials in four 32-column chunks; each chunk's P (packed bf16)
+        // is stored to TMEM while the next chunk is computed
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float p0 = sm100::ex2(fmaf(__uint_as_float(s[2 * c]), sl2, -m_sub));
-          const float p1 = sm100::ex2(fmaf(__uint_as_float(s[2 * c + 1]), sl2, -m_sub));
-          l0 += p0;
-          l1 += p1;
-          s[c] = sm100::pack_bf16x2(p0, p1);
+        for (int q = 0; q < 4; ++q) {
+#pragma unroll
+          for (int cp = 16 * q; cp < 16 * q + 16; ++cp) {
+            const float2 x = __ffma2_rn(
+                make_float2(__uint_as_float(s[2 * cp]), __uint_as_float(s[2 * cp + 1])), sl2x2,
+                negm);
+            float2 e;
+            if (poly_pair(cp)) {
+              e = sm100::ex2_poly2(x);
+            } else {
+              e.x = sm100::ex2(x.x);
+              e.y = sm100::ex2(x.y);
+            }
+            lsum = __fadd2_rn(lsum, e);
+            s[cp] = sm100::pack_bf16x2(e.x, e.y);
+          }
+          sm100::tmem_st16(s_addr + 16 * q, &s[16 * q]);
         }
-        l += l0 + l1;
-        sm100::tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-        sm100::tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+        l += lsum.x + lsum.y;
         sm100::tmem_st_wait();
         sm100::tc_fence_before();
         sm100::mbar_arrive(&p_full[t]);
       }
       if (!ok) break;
       // ---------------- epilogue: O = o / l (bf16), LSE = ln(2) * (m + log2 l)
-      if (!(ok = sm100::mbar_wait(&o_full[t], qk & 1, abort_flag, p.status))) break;
+      if (!(ok = sm100::mbar_wait(&o_full[t], k & 1, abort_flag, p.status))) break;
       sm100::tc_fence_after();
       const bool live = row < p.Lq;
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       __nv_bfloat16* orow =
           p.O + ((static_cast<size_t>(it.b) * p.Hq + it.h) * p.Lq + (live ? row : 0)) * D;
-      if (it.n[t] > 0) {
+      if (n_t > 0) {
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -414,6 +478,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == 9) {
     sm100::tc_fence_after();
     sm100::tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0) {
+    // the last CTA to finish re-arms the dynamic scheduler for the next launch
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+      p.sched[0] = 0;
+      p.sched[1] = 0;
+      __threadfence();
+    }
   }
 }
 

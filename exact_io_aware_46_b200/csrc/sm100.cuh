@@ -93,6 +93,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   return false;
 }
 
+// Bounded wait that ignores the abort flag: used to drain in-flight tensor-core
+// work before tensor memory is released, also on the abort path.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const long long t0 = clock64();
+  for (uint32_t it = 0; it < 0x40000000u; ++it) {
+    if (mbar_try_wait(a, parity)) return true;
+    if (clock64() - t0 > ATTN_WAIT_CYCLES) break;
+  }
+  return false;
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
@@ -217,6 +229,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -231,6 +253,36 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// max(a, b, c) in one instruction (sm_100 three-input max).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair of floats on the FMA pipe instead of the special-function
+// unit: Cody-Waite reduction x = n + f with n = round(x) (the 1.5 * 2^23
+// addition rounds to an integer in the low mantissa bits), f in [-1/2, 1/2];
+// 2^f by a degree-3 polynomial whose coefficients minimise the maximum relative
+// error on that interval (fitted by exp2_poly_fit.py: 1.01e-4); 2^n enters by
+// adding n to the exponent field.  Inputs are clamped at -126, so masked (-inf)
+// entries give ~1e-38 instead of 0.  Valid for x <= 127.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 magic = make_float2(12582912.f, 12582912.f);
+  const float2 t = __fadd2_rn(x, magic);
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
+  float2 q = __ffma2_rn(make_float2(0.055008937f, 0.055008937f), f,
+                        make_float2(0.24221095f, 0.24221095f));
+  q = __ffma2_rn(q, f, make_float2(0.6932829f, 0.6932829f));
+  q = __ffma2_rn(q, f, make_float2(1.f, 1.f));
+  // (t_bits - bits(1.5 * 2^23)) << 23 == t_bits << 23 modulo 2^32
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` lands in bits 0-15.

@@ -44,8 +44,10 @@ def test_workspace_sizes_are_closed_forms(lib):
     n = 64 * 32 * 32
     assert attn.attn_decode_workspace_size(64, 32, 8, 32768, 128) == 256 + ((n * 128 * 4 + n * 4 + 255) // 256) * 256
     # backward: fp32 dQ accumulator and D per query row; nothing of size Lq x Lk
-    rows = 2 * 16 * 8192
-    assert attn.attn_bwd_workspace_size(2, 16, 16, 8192, 8192, 128) == 256 + ((rows * 128 * 4 + rows * 4 + 255) // 256) * 256
+    rows = 2 * 16 * 8192  # query rows, padded per head to a multiple of 64
+    assert attn.attn_bwd_workspace_size(2, 16, 16, 8192, 8192, 128) == 256 + ((rows * 128 * 4 + rows * 8 + 255) // 256) * 256
+    rows = 1 * 2 * 128  # Lq = 100 pads to 128
+    assert attn.attn_bwd_workspace_size(1, 2, 1, 100, 300, 128) == 256 + ((rows * 128 * 4 + rows * 8 + 255) // 256) * 256
 
 
 def test_status_strings(lib):

@@ -1,0 +1,96 @@
+"""Backward parity: the CUDA backward (fed with the CUDA forward's O and LSE)
+against the fp64 oracle's gradients computed from Q, K, V and dO alone."""
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests._util import GRAD_REL_L2, bits, dev_bf16, rel_l2, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _lib():
+    import exact_io_aware_46_b200 as attn
+
+    return attn
+
+
+def _check(got, ref, what):
+    rl = rel_l2(got, ref)
+    assert rl <= GRAD_REL_L2, f"{what}: rel-L2 {rl:.3e}"
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+
+
+CASES = [
+    # B, Hq, Hkv, Lq, Lk, causal, k_lens
+    (1, 2, 2, 200, 200, True, None),
+    (1, 2, 2, 200, 200, False, None),
+    (1, 4, 2, 150, 150, True, None),           # grouped-query heads: dK/dV sum over 2 heads
+    (2, 2, 2, 190, 190, False, [120, 50]),     # key padding
+    (2, 1, 1, 257, 257, True, [257, 130]),     # causal + padding, ragged tiles
+    (1, 2, 2, 100, 260, True, None),           # Lq < Lk
+    (1, 2, 2, 260, 100, True, None),           # Lq > Lk: leading rows see no key
+    (1, 1, 1, 64, 128, False, None),           # exactly one query tile and one key tile
+    (1, 2, 1, 300, 300, True, [0]),            # k_len = 0: all gradients zero
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,causal,k_lens", CASES)
+def test_bwd_matches_oracle(B, Hq, Hkv, Lq, Lk, causal, k_lens):
+    import torch
+
+    attn = _lib()
+    d = 128
+    seed = 500 + Lq + 3 * Lk + Hq
+    Q = synth.normal_bf16(seed * 16 + 1, (B, Hq, Lq, d))
+    K = synth.normal_bf16(seed * 16 + 2, (B, Hkv, Lk, d))
+    V = synth.normal_bf16(seed * 16 + 3, (B, Hkv, Lk, d))
+    dO = synth.normal_bf16(seed * 16 + 4, (B, Hq, Lq, d))
+    scale = 1.0 / math.sqrt(d)
+    q, k, v, do = (dev_bf16(x) for x in (Q, K, V, dO))
+    kl = None if k_lens is None else torch.tensor(k_lens, dtype=torch.int32, device="cuda")
+    O, L = attn.attn_fwd(q, k, v, causal=causal, k_lens=kl)
+    dq, dk, dv = attn.attn_bwd(q, k, v, O, do, L, causal=causal, k_lens=kl)
+    torch.cuda.synchronize()
+    rQ, rK, rV = oracle.bwd(Q, K, V, dO, scale, causal=causal, k_lens=k_lens)
+    if k_lens == [0]:
+        for t in (dq, dk, dv):
+            assert torch.all(t == 0)
+        return
+    _check(to_f64(dq), rQ, "dQ")
+    _check(to_f64(dk), rK, "dK")
+    _check(to_f64(dv), rV, "dV")
+
+
+def test_bwd_full_size_sampled():
+    """B=2, H=16, L=8192, d=128, causal: sampled rows of dQ and keys of dK, dV."""
+    import torch
+
+    attn = _lib()
+    B, H, L, d = 2, 16, 8192, 128
+    seed = 4605
+    shp = (B, H, L, d)
+    q = synth.normal_bf16_device(seed * 16 + 1, shp, "cuda")
+    k = synth.normal_bf16_device(seed * 16 + 2, shp, "cuda")
+    v = synth.normal_bf16_device(seed * 16 + 3, shp, "cuda")
+    do = synth.normal_bf16_device(seed * 16 + 4, shp, "cuda")
+    O, Lse = attn.attn_fwd(q, k, v, causal=True)
+    dq, dk, dv = attn.attn_bwd(q, k, v, O, do, Lse, causal=True)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([[0, 1, 63, 64, 127, L - 1],
+                                     rng.choice(L, 40, replace=False)])).astype(np.int32)
+    cols = np.unique(np.concatenate([[0, 127, 128, L - 128, L - 1],
+                                     rng.choice(L, 40, replace=False)])).astype(np.int32)
+    for b, h in ((0, 0), (1, 11)):
+        sl = lambda t: bits(t[b:b + 1, h:h + 1])
+        Qh, Kh, Vh, dOh = sl(q), sl(k), sl(v), sl(do)
+        rQ, rK, rV = oracle.bwd_sampled(Qh, Kh, Vh, dOh, 1 / math.sqrt(d), True, None, 0, 0,
+                                        rows, cols)
+        _check(to_f64(dq[b, h, rows]), rQ[0], f"dQ[{b},{h}]")
+        _check(to_f64(dk[b, h, cols]), rK, f"dK[{b},{h}]")
+        _check(to_f64(dv[b, h, cols]), rV, f"dV[{b},{h}]")
