@@ -316,7 +316,7 @@ def cpu_baseline(budget_s=12.0):
     V = synth.normal_bf16(synth.workload_seed(2, "v") ^ 0x55, (1, 1, L, d))
     stride = 16
     done_flops, t_used, reps = 0.0, 0.0, 0
-    while t_used < budget_s and reps < 64:
+    while t_used < budget_s and reps < 4096:
         rows = np.arange(reps % stride, L, stride, dtype=np.int32)
         t0 = time.perf_counter()
         oracle.fwd(Q, K, V, 1 / math.sqrt(d), causal=True, rows=rows)
@@ -378,7 +378,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--legs", default="fwd,decode,bwd")
+    ap.add_argument("--legs", default="fwd,decode,bwd",
+                    help="comma list of fwd, decode, bwd (subsets are for profiling runs)")
+    ap.add_argument("--decode-lmax", type=int, default=DEC["Lmax"],
+                    help="smaller KV cache for profiling captures (k_len ~ U[1024, Lmax])")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -401,8 +404,10 @@ def main():
 
     gpu_idx = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]
                   if os.environ.get("CUDA_VISIBLE_DEVICES") else local)
+    DEC["Lmax"] = args.decode_lmax
     with Clocks(gpu_idx) as clk:
-        ms, ms_e2e, h2d, d2h = fwd_leg(args.steps, args.warmup, world, flush)
+        if "fwd" in legs:
+            ms, ms_e2e, h2d, d2h = fwd_leg(args.steps, args.warmup, world, flush)
         if "decode" in legs:
             dms, kv_bytes, _ = decode_leg(args.steps, args.warmup, world, flush)
         if "bwd" in legs:
@@ -410,6 +415,17 @@ def main():
         else:
             bms = None
     clocks = clk.summary()
+    if "fwd" not in legs:  # profiling runs of single legs: report what ran
+        rep = {"legs": legs, "clocks": clocks}
+        if "decode" in legs:
+            rep["decode_ms"] = float(np.mean(dms))
+            rep["decode_GBs"] = kv_bytes / (float(np.mean(dms)) * 1e-3) / 1e9
+        if bms is not None:
+            rep["bwd_ms"] = float(np.mean(bms))
+            rep["bwd_TFLOPs"] = bwd_flops(BWD) / (float(np.mean(bms)) * 1e-3) / 1e12
+        if rank == 0:
+            print(json.dumps(rep), flush=True)
+        return
 
     flops = fwd_flops(FWD)
     t_step = max_over_ranks(float(np.mean(ms)), world)
@@ -443,7 +459,8 @@ def main():
         t_d = max_over_ranks(float(np.mean(dms)), world)
         gbs = kv_bytes / (float(np.mean(dms)) * 1e-3) / 1e9
         line["decode"] = {
-            "workload": "split-KV decode B64 Hq32 Hkv8 d128, cache 32768, k_len~U[1024,32768]",
+            "workload": f"split-KV decode B64 Hq32 Hkv8 d128, cache {DEC['Lmax']}, "
+                        f"k_len~U[1024,{DEC['Lmax']}]",
             "value": world * kv_bytes / (t_d * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": t_d,
             "kv_bytes_per_step": kv_bytes,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",

@@ -37,7 +37,7 @@ constexpr int BN = 128;  // keys per work item (TMEM lanes)
 constexpr int BMQ = 64;  // query rows per query tile
 constexpr int D = 128;   // head dimension handled by the main kernel
 constexpr int NQS = 3;   // query/dO ring stages
-constexpr int NTHREADS = 320;
+constexpr int NTHREADS = 320;  // P/dS warpgroup, dQ warpgroup, load warp, MMA warp
 
 // shared memory map (bytes); the swizzled panels are 1024-byte aligned
 constexpr int OFF_K = 0;                              // [128 keys][d]: 2 panels of 16 KB
@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const float* dq_acc
 
 // ------------------------------------------------------------------ main
 
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(NTHREADS, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmdO,
                     const __grid_constant__ CUtensorMap tmK,
@@ -263,7 +263,6 @@ __global__ void __maxnreg__(200)
   sm100::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int off = p.Lk - p.Lq;  // bottom-right causal alignment
-
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (sm100::lane_id() == 0) {

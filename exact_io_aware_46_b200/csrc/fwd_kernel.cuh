@@ -119,8 +119,34 @@ __device__ __forceinline__ Item get_item(const Params& p, int w, bool* bad) {
 // c / 2 satisfies (c / 2) % 4 == 3: a quarter of the exponentials.
 __device__ __forceinline__ constexpr bool poly_pair(int cp) { return (cp & 3) == 3; }
 
+// S_t = Q_t K_j^T: 128 x 128 (keys) x D, both operands K-major SW128 panels.
+// One base descriptor per operand; the K-steps add constant offsets (>> 4) to
+// the start-address field.
 template <int D>
-__global__ void __maxnreg__(200)
+__device__ __noinline__ void issue_s_tile(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+  const uint64_t qd = sm100::sdesc_sw128(q_smem, 16, 1024);
+  const uint64_t kd = sm100::sdesc_sw128(k_smem, 16, 1024);
+#pragma unroll
+  for (int k = 0; k < D / 16; ++k) {
+    const uint64_t off = static_cast<uint64_t>(((k >> 2) * CHUNK_BYTES + (k & 3) * 32) >> 4);
+    sm100::mma_ss(d_tmem, qd + off, kd + off, Cfg<D>::IDESC_S, k > 0 ? 1u : 0u);
+  }
+}
+
+// O_t (+)= P_t V_j: A = P_t from TMEM (packed bf16, 8 columns per 16 keys),
+// B = V_j MN-major (LBO = next 64-column panel, SBO = next 8 keys).
+template <int D>
+__device__ __noinline__ void issue_pv_tile(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem,
+                                           bool acc) {
+  const uint64_t vd = sm100::sdesc_sw128(v_smem, CHUNK_BYTES, 1024);
+#pragma unroll
+  for (int k = 0; k < BN / 16; ++k)
+    sm100::mma_ts(o_tmem, p_tmem + k * 8, vd + static_cast<uint64_t>((k * 2048) >> 4),
+                  Cfg<D>::IDESC_PV, (acc || k > 0) ? 1u : 0u);
+}
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const Params p) {
   using C = Cfg<D>;
@@ -243,23 +269,12 @@ __global__ void __maxnreg__(200)
       const uint32_t kv_addr = sbase + C::OFF_KV;
 
       auto issue_s = [&](int t, int slot) {
-        const uint32_t qa = q_addr + t * C::TILE_BYTES;
-        const uint32_t ka = kv_addr + slot * C::TILE_BYTES;
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * CHUNK_BYTES + (k & 3) * 32;
-          sm100::mma_ss(tmem + C::s_col(t), sm100::sdesc_sw128(qa + off, 16, 1024),
-                        sm100::sdesc_sw128(ka + off, 16, 1024), C::IDESC_S, k > 0);
-        }
+        issue_s_tile<D>(tmem + C::s_col(t), q_addr + t * C::TILE_BYTES,
+                        kv_addr + slot * C::TILE_BYTES);
       };
       auto issue_pv = [&](int t, int slot, bool acc) {
-        const uint32_t va = kv_addr + slot * C::TILE_BYTES;
-#pragma unroll
-        for (int k = 0; k < BN / 16; ++k) {
-          sm100::mma_ts(tmem + C::o_col(t), tmem + C::s_col(t) + k * 8,
-                        sm100::sdesc_sw128(va + k * 2048, CHUNK_BYTES, 1024), C::IDESC_PV,
-                        (acc || k > 0) ? 1u : 0u);
-        }
+        issue_pv_tile<D>(tmem + C::o_col(t), tmem + C::s_col(t), kv_addr + slot * C::TILE_BYTES,
+                         acc);
       };
 
       for (uint32_t k = 0; ok; ++k) {

@@ -267,11 +267,14 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // addition rounds to an integer in the low mantissa bits), f in [-1/2, 1/2];
 // 2^f by a degree-3 polynomial whose coefficients minimise the maximum relative
 // error on that interval (fitted by exp2_poly_fit.py: 1.01e-4); 2^n enters by
-// adding n to the exponent field.  Inputs are clamped at -126, so masked (-inf)
-// entries give ~1e-38 instead of 0.  Valid for x <= 127.
-__device__ __forceinline__ float2 ex2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
+// adding n to the exponent field.  Inputs below -125 (masked entries are
+// -inf) return exactly 0, as the special-function unit does for -inf; the
+// reduction itself is applied to inputs clamped at -126 so the exponent field
+// never underflows into the sign bit.  Valid for x <= 127.
+__device__ __forceinline__ float2 ex2_poly2(float2 x_in) {
+  float2 x;
+  x.x = fmaxf(x_in.x, -126.f);
+  x.y = fmaxf(x_in.y, -126.f);
   const float2 magic = make_float2(12582912.f, 12582912.f);
   const float2 t = __fadd2_rn(x, magic);
   const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
@@ -281,8 +284,9 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
   q = __ffma2_rn(q, f, make_float2(0.6932829f, 0.6932829f));
   q = __ffma2_rn(q, f, make_float2(1.f, 1.f));
   // (t_bits - bits(1.5 * 2^23)) << 23 == t_bits << 23 modulo 2^32
-  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+  const float rx = __int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23));
+  const float ry = __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23));
+  return make_float2(x_in.x < -125.f ? 0.f : rx, x_in.y < -125.f ? 0.f : ry);
 }
 
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` lands in bits 0-15.
