@@ -25,7 +25,10 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libattn.so")
 
-ATTN_OK, ATTN_ERR_INVALID, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT = range(5)
+(ATTN_OK, ATTN_ERR_INVALID, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT,
+ ATTN_ERR_CAPACITY) = range(6)
+#: size of the fixed device scratch used by attn_fwd_splitkv_decode_noalloc
+ATTN_NOALLOC_SCRATCH_BYTES = 16 << 20
 ATTN_MASK_NONE, ATTN_MASK_CAUSAL = 0, 1
 ATTN_DEV_BAD_KLEN, ATTN_DEV_TIMEOUT = 1, 2
 
@@ -50,6 +53,8 @@ SIGNATURES = {
     "attn_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "attn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f,
                       _i, _vp, _vp, _sz, _vp]),
+    "attn_fwd_splitkv_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f,
+                                             _vp, _vp]),
     "attn_read_device_status": (_i, [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]),
     "attn_clear_device_status": (_i, [_vp, _vp]),
 }
@@ -183,6 +188,29 @@ def attn_fwd_splitkv_decode(Q, Kc, Vc, k_lens, scale=None, O=None, lse=None, wor
                                          Hkv, Lmax, d, float(scale), _ptr(k_lens),
                                          _ptr(workspace), workspace.numel(), _stream(stream))
     _check(code, "attn_fwd_splitkv_decode")
+    return O, lse
+
+
+def attn_fwd_splitkv_decode_noalloc(Q, Kc, Vc, k_lens, scale=None, O=None, lse=None,
+                                    stream=None, want_lse=True):
+    """Split-KV decode without a workspace, for callers that cannot allocate
+    device memory (the library call itself allocates nothing; this wrapper only
+    creates O / LSE when they are not passed in).  Calls that overlap on the
+    GPU share one fixed scratch array and race: serialise them."""
+    for t, n in ((Q, "Q"), (Kc, "Kcache"), (Vc, "Vcache")):
+        _bf16(t, n)
+    B, Hq, _, d = Q.shape
+    Hkv, Lmax = Kc.shape[1], Kc.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if O is None:
+        O = torch.empty_like(Q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=Q.device)
+    code = lib().attn_fwd_splitkv_decode_noalloc(_ptr(Q), _ptr(Kc), _ptr(Vc), _ptr(O), _ptr(lse),
+                                                 B, Hq, Hkv, Lmax, d, float(scale),
+                                                 _ptr(k_lens), _stream(stream))
+    _check(code, "attn_fwd_splitkv_decode_noalloc")
     return O, lse
 
 

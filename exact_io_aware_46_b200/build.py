@@ -11,6 +11,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SO = os.path.join(HERE, "libattn.so")
 SRC = os.path.join(HERE, "csrc", "attn_api.cu")
+SRC_NOALLOC = os.path.join(HERE, "csrc", "decode_noalloc.cu")
 
 
 def nvcc() -> str:
@@ -21,7 +22,7 @@ def nvcc() -> str:
 
 
 def sources():
-    return [SRC] + sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh"))) + [
+    return [SRC, SRC_NOALLOC] + sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh"))) + [
         os.path.join(ROOT, "include", "attn.h")]
 
 
@@ -38,7 +39,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     tmp = SO + f".tmp{os.getpid()}"
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3",
            "-std=c++17", "-Xcompiler", "-fPIC", "-shared", "-I", os.path.join(ROOT, "include"),
-           "-Xptxas", "-v" if verbose else "-O3", SRC, "-o", tmp]
+           "-Xptxas", "-v" if verbose else "-O3", SRC, SRC_NOALLOC, "-o", tmp]
     subprocess.check_call(cmd)
     os.replace(tmp, SO)
     return SO

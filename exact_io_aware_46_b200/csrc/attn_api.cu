@@ -92,6 +92,7 @@ const char* attn_status_string(attn_status_t s) {
     case ATTN_ERR_UNSUPPORTED: return "unsupported";
     case ATTN_ERR_CUDA: return "cuda error";
     case ATTN_ERR_TIMEOUT: return "device wait timed out";
+    case ATTN_ERR_CAPACITY: return "request exceeds the fixed scratch of the no-alloc call";
   }
   return "unknown status";
 }

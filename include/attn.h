@@ -65,7 +65,8 @@ typedef enum {
   ATTN_ERR_INVALID = 1,     /* bad pointer, size, alignment, or workspace too small */
   ATTN_ERR_UNSUPPORTED = 2, /* valid request outside what the kernels implement */
   ATTN_ERR_CUDA = 3,        /* a CUDA runtime/driver call or launch failed */
-  ATTN_ERR_TIMEOUT = 4      /* (device status) a bounded internal wait expired */
+  ATTN_ERR_TIMEOUT = 4,     /* (device status) a bounded internal wait expired */
+  ATTN_ERR_CAPACITY = 5     /* request needs more than the fixed scratch of a no-alloc call */
 } attn_status_t;
 
 enum { ATTN_MASK_NONE = 0, ATTN_MASK_CAUSAL = 1 };
@@ -134,6 +135,39 @@ attn_status_t attn_bwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf
                        attn_bf16_t* dQ, attn_bf16_t* dK, attn_bf16_t* dV, int B, int Hq, int Hkv,
                        int Lq, int Lk, int d, float scale, int mask_flags, const int32_t* k_lens,
                        void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ decode without allocation
+ * No counterpart in the pages: an interface addition for callers that cannot
+ * allocate device memory.  attn_fwd_splitkv_decode needs a workspace for its
+ * fp32 per-chunk partials; callers that cannot hand one over (code running
+ * while a stream is being captured into a CUDA graph, where an allocation would
+ * break the capture; runtimes with a fixed memory plan that only pass the
+ * tensors they own; latency-critical loops that must not pay an allocation's
+ * implicit synchronisation) use this variant instead.  It computes exactly what
+ * attn_fwd_splitkv_decode computes, with the same kernels and arguments minus
+ * the workspace.
+ *
+ * Scratch: a file-scope device array of ATTN_NOALLOC_SCRATCH_BYTES that every
+ * GPU loading the library holds until the process exits.  A request whose
+ * partials need more (256 + B*Hq*ceil(Lmax/1024)*(4*d + 4) bytes, rounded up to
+ * 256) returns ATTN_ERR_CAPACITY before anything is launched.  The first call
+ * on a device looks up the array's device address (cudaGetSymbolAddress, with
+ * that device current); make that first call before any stream capture.  The
+ * call allocates and frees nothing.
+ *
+ * All calls share the one array: calls that may overlap on the GPU (different
+ * streams, or different host threads on one device) race and corrupt each
+ * other's results; serialise them.  Each call clears the status word it keeps
+ * at the head of the array; the partials need no clearing.  Device-side errors
+ * (a k_lens entry outside [0, Lmax]) zero the affected outputs but are not
+ * reported (there is no workspace to read them from).
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (16u << 20)
+attn_status_t attn_fwd_splitkv_decode_noalloc(const attn_bf16_t* Q, const attn_bf16_t* Kcache,
+                                              const attn_bf16_t* Vcache, attn_bf16_t* O,
+                                              float* lse, int B, int Hq, int Hkv, int Lmax,
+                                              int d, float scale, const int32_t* k_lens,
+                                              void* stream);
 
 /* ------------------------------------------------------------------ status
  * Reads (after synchronising `stream`) the device status word of `workspace`:
