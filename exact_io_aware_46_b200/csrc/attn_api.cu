@@ -118,42 +118,45 @@ attn_status_t attn_fwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (Lq == 0) return ATTN_OK;
 
-  CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, Q, d, Lq, static_cast<long long>(B) * Hq, 128) ||
-      !make_tmap(&tk, K, d, Lk, static_cast<long long>(B) * Hkv, 128) ||
-      !make_tmap(&tv, V, d, Lk, static_cast<long long>(B) * Hkv, 128))
-    return ATTN_ERR_CUDA;
-
-  attn_fwd_impl::Params p;
-  p.O = reinterpret_cast<__nv_bfloat16*>(O);
-  p.lse = lse;
-  p.k_lens = k_lens;
-  p.status = reinterpret_cast<int*>(workspace);
-  p.sched = reinterpret_cast<int*>(workspace) + 1;
-  p.B = B;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.Lq = Lq;
-  p.Lk = Lk;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.causal = (mask_flags & ATTN_MASK_CAUSAL) ? 1 : 0;
-  p.n_pairs = (Lq + 2 * attn_fwd_impl::BM - 1) / (2 * attn_fwd_impl::BM);
-  p.n_items = B * Hq * p.n_pairs;
   const int sms = device_sms();
   if (sms <= 0) return ATTN_ERR_CUDA;
-  const int grid = p.n_items < sms ? p.n_items : sms;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int n_pairs = (Lq + 2 * attn_fwd_impl::BM - 1) / (2 * attn_fwd_impl::BM);
+  const int n_items = B * Hq * n_pairs;
   cudaError_t e;
-  if (d == 128) {
-    constexpr int smem = attn_fwd_impl::Cfg<128>::SMEM_BYTES;
-    e = set_smem(attn_fwd_impl::fwd_kernel<128>, smem);
-    if (e == cudaSuccess)
-      attn_fwd_impl::fwd_kernel<128><<<grid, attn_fwd_impl::NTHREADS, smem, s>>>(tq, tk, tv, p);
-  } else {
-    constexpr int smem = attn_fwd_impl::Cfg<64>::SMEM_BYTES;
-    e = set_smem(attn_fwd_impl::fwd_kernel<64>, smem);
-    if (e == cudaSuccess)
-      attn_fwd_impl::fwd_kernel<64><<<grid, attn_fwd_impl::NTHREADS, smem, s>>>(tq, tk, tv, p);
+  {
+    CUtensorMap tq, tk, tv;
+    if (!make_tmap(&tq, Q, d, Lq, static_cast<long long>(B) * Hq, 128) ||
+        !make_tmap(&tk, K, d, Lk, static_cast<long long>(B) * Hkv, 128) ||
+        !make_tmap(&tv, V, d, Lk, static_cast<long long>(B) * Hkv, 128))
+      return ATTN_ERR_CUDA;
+    attn_fwd_impl::Params p;
+    p.O = reinterpret_cast<__nv_bfloat16*>(O);
+    p.lse = lse;
+    p.k_lens = k_lens;
+    p.status = reinterpret_cast<int*>(workspace);
+    p.sched = reinterpret_cast<int*>(workspace) + 1;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Lq = Lq;
+    p.Lk = Lk;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = (mask_flags & ATTN_MASK_CAUSAL) ? 1 : 0;
+    p.n_pairs = n_pairs;
+    p.n_items = n_items;
+    const int grid = n_items < sms ? n_items : sms;
+    if (d == 128) {
+      constexpr int smem = attn_fwd_impl::Cfg<128>::SMEM_BYTES;
+      e = set_smem(attn_fwd_impl::fwd_kernel<128>, smem);
+      if (e == cudaSuccess)
+        attn_fwd_impl::fwd_kernel<128><<<grid, attn_fwd_impl::NTHREADS, smem, s>>>(tq, tk, tv, p);
+    } else {
+      constexpr int smem = attn_fwd_impl::Cfg<64>::SMEM_BYTES;
+      e = set_smem(attn_fwd_impl::fwd_kernel<64>, smem);
+      if (e == cudaSuccess)
+        attn_fwd_impl::fwd_kernel<64><<<grid, attn_fwd_impl::NTHREADS, smem, s>>>(tq, tk, tv, p);
+    }
   }
   if (e != cudaSuccess) return ATTN_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;

@@ -75,11 +75,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 #define ATTN_WAIT_CYCLES (4000000000LL)
 #endif
 
+// Records an expired wait: ATTN_DEV_TIMEOUT (= 2) in status[0] and, for the
+// first expiry only, the wait's site id in status[3] (diagnostics).
+__device__ __forceinline__ void record_timeout(int* status, int site) {
+  atomicOr(status, 2);
+  atomicCAS(status + 3, 0, site);
+}
+
 // Bounded wait on phase `parity` of `bar`.  `abort` is a CTA-shared flag: once
 // any role of the CTA has timed out, every other wait returns false at once.
-// On expiry sets the flag and ATTN_DEV_TIMEOUT (= 2) in *status.
+// On expiry sets the flag and records the timeout (site id `site`).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int* status) {
+                                          int* status, int site = 1) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const long long t0 = clock64();
@@ -89,7 +96,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (clock64() - t0 > ATTN_WAIT_CYCLES) break;
   }
   *abort = 1;
-  atomicOr(status, 2);
+  record_timeout(status, site);
   return false;
 }
 
