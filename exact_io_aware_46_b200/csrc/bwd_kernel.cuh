@@ -46,8 +46,10 @@ constexpr int OFF_QS = 65536;                         // stage s: Q (2 x 8 KB) t
 constexpr int QS_BYTES = 32768;
 constexpr int OFF_DS = OFF_QS + NQS * QS_BYTES;       // dS^T buffers [128 keys][64 rows], 16 KB each
 constexpr int OFF_LD = OFF_DS + 2 * 16384;            // stage s: lse2 [64] then D [64]
-constexpr int OFF_BAR = OFF_LD + NQS * 512;
+constexpr int OFF_DQ = OFF_LD + NQS * 512;            // dQ tile staging [64 rows][128] fp32, 32 KB
+constexpr int OFF_BAR = OFF_DQ + 32768;
 constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;
+static_assert(SMEM_BYTES <= 232448, "dynamic shared memory limit");
 
 // TMEM columns
 constexpr uint32_t S_COL0 = 0;      // S^T / P^T, 2 buffers x 64
@@ -127,6 +129,25 @@ __device__ __forceinline__ Item get_item(const Params& p, int w, bool* bad) {
   const int nq = (p.Lq + BMQ - 1) / BMQ;
   it.T = p.G * (nq - it.i_lo);
   return it;
+}
+
+// Bulk reduce-add of `bytes` fp32 values from shared to global memory (the
+// TMA unit performs the additions at L2), tracked by a bulk async-group.
+__device__ __forceinline__ void bulk_reduce_add_f32(float* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile(
+      "cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
+          reinterpret_cast<uint64_t>(gdst)),
+      "r"(sm100::smem_u32(ssrc)), "r"(bytes)
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until the shared-memory sources of all committed bulk groups were read.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Waits until all committed bulk groups completed (writes visible).
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -500,8 +521,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ dQ drain (one d column per thread)
+    // dQ^T of a query tile (lanes = head-dimension index, columns = 64 rows)
+    // is staged row-major in shared memory and added into the fp32
+    // accumulator with one 32 KB bulk reduce (the tile's rows are contiguous
+    // there); the staging buffer is reused once the previous reduce has read it.
     const int dl = threadIdx.x - 128;  // TMEM lane = head-dimension index
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    float* stage = reinterpret_cast<float*>(smem + OFF_DQ);
     uint32_t tq = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
@@ -521,15 +547,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         sm100::tmem_ld_wait();
         sm100::tc_fence_before();
         sm100::mbar_arrive(&dq_empty[b]);
-        const int qh = it.b * p.Hq + it.hkv * p.G + g;
-        float* dst = p.dq_acc + (static_cast<size_t>(qh) * p.Lqp + i * BMQ) * D + dl;
-        const int rows = min(BMQ, p.Lq - i * BMQ);
+        // the previous tile's reduce must have finished reading the staging buffer
+        if (threadIdx.x == 128) bulk_wait_read_all();
+        sm100::named_bar_sync(1, 128);
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c < rows) atomicAdd(dst + static_cast<size_t>(c) * D, __uint_as_float(v[c]));
+        for (int c = 0; c < 64; ++c) stage[c * D + dl] = __uint_as_float(v[c]);
+        fence_proxy_async_smem();
+        sm100::named_bar_sync(1, 128);
+        if (threadIdx.x == 128) {
+          const int qh = it.b * p.Hq + it.hkv * p.G + g;
+          bulk_reduce_add_f32(p.dq_acc + (static_cast<size_t>(qh) * p.Lqp + i * BMQ) * D, stage,
+                              BMQ * D * 4);
+        }
       }
       tq += it.T;
     }
+    // the convert pass reads the accumulator after this kernel; the reduces
+    // must be complete before the CTA exits
+    if (threadIdx.x == 128) bulk_wait_all();
   }
 
   sm100::tc_fence_before();
