@@ -348,7 +348,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           sm100::tc_commit(kv_empty);
           continue;
         }
-        // prologue: S and dP of the first query tile
+        // Issue order per query tile t (buffers b = t & 1, nb = (t + 1) & 1):
+        //   S(t+1) | dV(t) [P(t)] | dP(t+1) [dQ^T(t-1) drained] | dK(t), dQ^T(t) [dS(t)]
+        // so each wait on another warp's signal has half an iteration of queued
+        // tensor work in front of it.
         {
           const int slot = tq % NQS, b = tq & 1;
           if (!(ok = sm100::mbar_wait(&qdo_full[slot], (tq / NQS) & 1, abort_flag, p.status)))
@@ -366,20 +369,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const uint32_t cur = tq + t;
           const int slot = cur % NQS, b = cur & 1;
           const uint32_t u = cur >> 1;
-          if (t + 1 < it.T) {
-            const uint32_t nx = cur + 1;
-            const int ns = nx % NQS, nb = nx & 1;
+          const uint32_t nx = cur + 1;
+          const int ns = nx % NQS, nb = nx & 1;
+          const bool more = t + 1 < it.T;
+          if (more) {
             if (!(ok = sm100::mbar_wait(&qdo_full[ns], (nx / NQS) & 1, abort_flag, p.status)))
               break;
             sm100::tc_fence_after();
             issue_kmajor(S_COL0 + nb * 64, kA, qA(ns));
             sm100::tc_commit(&s_full[nb]);
-            if (!(ok = sm100::mbar_wait(&dq_empty[nb], ((nx >> 1) & 1) ^ 1, abort_flag,
-                                        p.status)))
-              break;
-            sm100::tc_fence_after();
-            issue_kmajor(DP_COL0 + nb * 64, vA, doA(ns));
-            sm100::tc_commit(&dp_full[nb]);
           }
           if (!(ok = sm100::mbar_wait(&p_full[b], u & 1, abort_flag, p.status))) break;
           sm100::tc_fence_after();
@@ -393,6 +391,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             sm100::mma_ts(tmem + DV_COL, tmem + S_COL0 + b * 64 + k * 8,
                           sm100::sdesc_sw128(doA(slot) + k * 2048, 8192, 1024), IDESC_DV,
                           (t > 0 || k > 0) ? 1u : 0u);
+          if (more) {
+            if (!(ok = sm100::mbar_wait(&dq_empty[nb], ((nx >> 1) & 1) ^ 1, abort_flag,
+                                        p.status)))
+              break;
+            sm100::tc_fence_after();
+            issue_kmajor(DP_COL0 + nb * 64, vA, doA(ns));
+            sm100::tc_commit(&dp_full[nb]);
+          }
           if (!(ok = sm100::mbar_wait(&ds_full[b], u & 1, abort_flag, p.status))) break;
           sm100::tc_fence_after();
           // dK += dS^T Q : A = dS^T (K-major over rows), B = Q (MN-major)
@@ -449,13 +455,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         sm100::tmem_ld32(tmem + lane_base + S_COL0 + b * 64 + 32,
                          *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
         sm100::tmem_ld_wait();
-        float pr[64];
-        const bool key_ok = key <= lim;
+        // key visible to query row r0 + c iff key <= lim_key and c >= cmin
         const int r0 = i * BMQ;
+        const bool key_ok = key <= lim;
+        const int cmin = p.causal ? key - r0 - off : -1;
+        // whole tile visible: no per-element test (warp-uniform; usual case)
+        const bool all_vis = __all_sync(0xffffffffu, key_ok && cmin <= 0);
+        const float4* l2v = reinterpret_cast<const float4*>(l2s);
+        const float2 sl2x2 = make_float2(p.scale_log2, p.scale_log2);
+        float pr[64];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const bool vis = key_ok && (!p.causal || key <= r0 + c + off);
-          pr[c] = vis ? sm100::ex2(fmaf(__uint_as_float(s[c]), p.scale_log2, -l2s[c])) : 0.f;
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 lq = l2v[c4];
+          const float2 x0 = __ffma2_rn(
+              make_float2(__uint_as_float(s[4 * c4]), __uint_as_float(s[4 * c4 + 1])), sl2x2,
+              make_float2(-lq.x, -lq.y));
+          const float2 x1 = __ffma2_rn(
+              make_float2(__uint_as_float(s[4 * c4 + 2]), __uint_as_float(s[4 * c4 + 3])), sl2x2,
+              make_float2(-lq.z, -lq.w));
+          pr[4 * c4] = sm100::ex2(x0.x);
+          pr[4 * c4 + 1] = sm100::ex2(x0.y);
+          pr[4 * c4 + 2] = sm100::ex2(x1.x);
+          pr[4 * c4 + 3] = sm100::ex2(x1.y);
+        }
+        if (!all_vis) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (!key_ok || c < cmin) pr[c] = 0.f;
         }
         uint32_t pk[32];
 #pragma unroll
@@ -472,10 +498,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         sm100::tmem_ld32(tmem + lane_base + DP_COL0 + b * 64 + 32,
                          *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
         sm100::tmem_ld_wait();
+        const float4* dvv = reinterpret_cast<const float4*>(dsv);
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
-          pk[c] = sm100::pack_bf16x2(pr[2 * c] * (__uint_as_float(s[2 * c]) - dsv[2 * c]),
-                                     pr[2 * c + 1] * (__uint_as_float(s[2 * c + 1]) - dsv[2 * c + 1]));
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 dq = dvv[c4];
+          const float2 d0 = __fmul2_rn(
+              make_float2(pr[4 * c4], pr[4 * c4 + 1]),
+              __fadd2_rn(make_float2(__uint_as_float(s[4 * c4]), __uint_as_float(s[4 * c4 + 1])),
+                         make_float2(-dq.x, -dq.y)));
+          const float2 d1 = __fmul2_rn(
+              make_float2(pr[4 * c4 + 2], pr[4 * c4 + 3]),
+              __fadd2_rn(make_float2(__uint_as_float(s[4 * c4 + 2]), __uint_as_float(s[4 * c4 + 3])),
+                         make_float2(-dq.z, -dq.w)));
+          pk[2 * c4] = sm100::pack_bf16x2(d0.x, d0.y);
+          pk[2 * c4 + 1] = sm100::pack_bf16x2(d1.x, d1.y);
+        }
         if (!(ok = sm100::mbar_wait(&ds_empty[b], (u & 1) ^ 1, abort_flag, p.status))) break;
         uint8_t* line = smem + OFF_DS + b * 16384 + kl_ * 128;
 #pragma unroll
