@@ -154,7 +154,8 @@ def dist_setup(n_gpus):
 def barrier(world):
     import torch
 
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
     if world > 1:
         import torch.distributed as dist
 
@@ -162,14 +163,50 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Max of a host float over the ranks (NCCL on the GPU, gloo on the CPU)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+# ------------------------------------------------------------------ DRAM traffic of the kernels
+
+TRAFFIC_TABLE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def kernel_sources_sha(files):
+    """sha256 over the listed source files (relative to the repo root)."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def traffic_per_launch(kernel, algorithmic=None):
+    """DRAM bytes (read + write) per launch from the committed ncu table, or
+    None when there is no entry or the kernel's sources changed since.  When
+    the capture ran a smaller case of the same kernel, its traffic is scaled by
+    the ratio of algorithmic bytes (``algorithmic`` = this launch's)."""
+    try:
+        with open(TRAFFIC_TABLE) as f:
+            t = json.load(f)[kernel]
+        if kernel_sources_sha(t["sources"]) != t["sources_sha256"]:
+            return None
+        dram = float(t["dram_bytes_per_launch"])
+        if algorithmic is not None and t.get("algorithmic_bytes_per_launch"):
+            dram *= algorithmic / float(t["algorithmic_bytes_per_launch"])
+        return dram
+    except Exception:
+        return None
 
 
 # ------------------------------------------------------------------ legs
@@ -446,7 +483,8 @@ def main():
                    "l2": "flushed (256 MB write) before every timed call",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                     "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+                     "traffic": traffic_per_launch("attn_fwd_impl::fwd_kernel<128>"),
                      "peak_source": f"{pk['source']} burst bf16 (MEASURED_PEAKS.json)",
                      "kernel": "attn_fwd_impl::fwd_kernel<128>"},
         "e2e": {"value": world * flops / (t_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
@@ -465,7 +503,8 @@ def main():
             "kv_bytes_per_step": kv_bytes,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "frac_of_8TBs": gbs / 8000.0,
-                         "traffic": None,
+                         "traffic": traffic_per_launch(
+                             "attn_decode_impl::decode_split_kernel<128,4>", kv_bytes),
                          "kernel": "attn_decode_impl::decode_split_kernel<128,4> + combine"},
             "gpu_launches": 2 * args.steps,
         }
@@ -478,7 +517,8 @@ def main():
             "workload": "causal backward B2 H16 L8192 d128", "value": world * bfl / (t_b * 1e-3) / 1e12,
             "unit": "TFLOP/s", "ms_per_step": t_b, "flops_per_step": bfl,
             "roofline": {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
-                         "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"], "traffic": None},
+                         "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"],
+                         "traffic": traffic_per_launch("attn_bwd_impl::bwd_main_kernel")},
         }
         line["gpu_launches"] += 3 * max(3, args.steps // 2)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
