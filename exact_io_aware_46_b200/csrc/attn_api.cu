@@ -266,3 +266,32 @@ attn_status_t attn_clear_device_status(void* workspace, void* stream) {
 }
 
 }  // extern "C"
+
+#ifdef ATTN_SELFTEST
+// Self-test of the bounded-wait machinery, compiled only into test builds of
+// the library (-DATTN_SELFTEST): one CTA waits on an mbarrier that nothing
+// arrives on.  The wait must give up after its cycle budget, record
+// ATTN_DEV_TIMEOUT and the site id in the status words and let the kernel end
+// normally, leaving the CUDA context usable.
+namespace {
+__global__ void selftest_expired_wait_kernel(int* status, int site) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    abort_flag = 0;
+    sm100::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    sm100::mbar_wait(&bar, 0, reinterpret_cast<volatile int*>(&abort_flag), status, site);
+}
+}  // namespace
+
+extern "C" attn_status_t attn_selftest_expired_wait(void* workspace, int site, void* stream) {
+  if (!workspace) return ATTN_ERR_INVALID;
+  selftest_expired_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<int*>(workspace), site);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+#endif
