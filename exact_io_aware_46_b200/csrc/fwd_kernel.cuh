@@ -12,14 +12,17 @@
 // B200 design (not the A100/Hopper designs the pages describe):
 //  * persistent CTAs, one per SM, walking a heaviest-first list of work items;
 //    an item is a pair of 128-row query tiles of one (batch, head);
-//  * warp 8 streams K and V tiles with TMA (128-byte swizzle) into a ring of
+//  * warp 16 streams K and V tiles with TMA (128-byte swizzle) into a ring of
 //    shared-memory slots; the two query tiles are loaded once per item;
-//  * warp 9 owns tensor memory and one elected thread issues every tcgen05.mma:
+//  * warp 17 owns tensor memory and one elected lane issues every tcgen05.mma:
 //    S_t = Q_t K_j^T (both operands in shared memory) into TMEM, and
 //    O_t += P_t V_j with P_t read from TMEM where the softmax wrote it over S_t;
-//  * warps 0-3 and 4-7 are two softmax warpgroups, one per query tile, so the
+//  * warps 0-7 and 8-15 are the softmax warps of query tile 0 and 1, so the
 //    tensor core computes one tile's scores while the other tile's softmax
-//    runs (ping-pong).  Each thread owns one query row (= one TMEM lane).
+//    runs (ping-pong).  Two warps share each row (= TMEM lane) of a tile, one
+//    per half of the key columns, and agree on the row max through shared
+//    memory; two warps per scheduler and tile hide the latency of the
+//    exponential chains that a single warp left exposed.
 //  * an eighth of the exponentials run on the FMA pipe (polynomial exp2), the
 //    rest on the special-function unit;
 //  * the running max is kept in the log2 domain and is only moved when a row's
@@ -34,7 +37,10 @@ namespace attn_fwd_impl {
 
 constexpr int BM = 128;        // query rows per tile (= TMEM lanes)
 constexpr int BN = 128;        // keys per key/value tile
-constexpr int NTHREADS = 320;  // 8 softmax warps + load warp + MMA warp
+constexpr int NSMX = 16;       // softmax warps: 2 tiles x 2 column halves x 4 lane quarters
+constexpr int NTHREADS = 32 * NSMX + 64;  // + load warp + MMA warp
+constexpr int W_LOAD = NSMX;
+constexpr int W_MMA = NSMX + 1;
 constexpr int CHUNK_BYTES = 128 * 128;  // one 128-row x 64-column bf16 swizzle panel
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 
@@ -45,10 +51,14 @@ struct Cfg {
   static constexpr int NS = (D == 128) ? 4 : 8;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_KV + NS * TILE_BYTES;
+  // row-max exchange [parity][tile][half][row] and row-sum exchange (same shape)
+  static constexpr int OFF_RED = OFF_KV + NS * TILE_BYTES;
+  static constexpr int OFF_LSUM = OFF_RED + 2 * 2 * 2 * BM * 4;
+  static constexpr int OFF_BAR = OFF_LSUM + 2 * 2 * 2 * BM * 4;
   static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;  // barriers, item ring + alignment slack
-  // TMEM columns: S_0, S_1 (128 fp32 columns each; P_t overwrites the first
-  // 64 columns of S_t as packed bf16 pairs), then O_0, O_1 (D columns each)
+  // TMEM columns: S_0, S_1 (128 fp32 columns each), then O_0, O_1 (D columns
+  // each).  The P of key half h (64 keys, packed bf16 pairs) overwrites the
+  // first 32 of the 64 S columns that half h was read from.
   __device__ static constexpr uint32_t s_col(int t) { return t * 128u; }
   __device__ static constexpr uint32_t o_col(int t) { return 256u + t * D; }
   static constexpr uint32_t IDESC_S = sm100::idesc_bf16_f32(128, BN, false, false);
@@ -119,15 +129,17 @@ __device__ __forceinline__ Item get_item(const Params& p, int w, bool* bad) {
 
 // Polynomial (FMA-pipe) instead of MUFU exp2 for column pairs whose index
 // c / 2 satisfies (c / 2) % 8 == 7: an eighth of the exponentials.  The softmax
-// warp is issue-bound as much as MUFU-bound; measured on B200 (causal
-// B4 H16 L4096 d128): 0 % 0.313 ms, 12.5 % 0.310 ms, 25 % 0.325 ms, 50 % 0.349 ms.
+// warp is issue-bound as much as MUFU-bound; measured on B200 with one softmax
+// warp per row (causal B4 H16 L4096 d128): 0 % 0.313 ms, 12.5 % 0.310 ms,
+// 25 % 0.325 ms, 50 % 0.349 ms.
 __device__ __forceinline__ constexpr bool poly_pair(int cp) { return (cp & 7) == 7; }
 
 // S_t = Q_t K_j^T: 128 x 128 (keys) x D, both operands K-major SW128 panels.
 // One base descriptor per operand; the K-steps add constant offsets (>> 4) to
-// the start-address field.
+// the start-address field.  Inlined: an out-of-line call put its argument and
+// descriptor set-up between consecutive MMAs.
 template <int D>
-__device__ __noinline__ void issue_s_tile(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+__device__ __forceinline__ void issue_s_tile(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
   const uint64_t qd = sm100::sdesc_sw128(q_smem, 16, 1024);
   const uint64_t kd = sm100::sdesc_sw128(k_smem, 16, 1024);
 #pragma unroll
@@ -137,16 +149,18 @@ __device__ __noinline__ void issue_s_tile(uint32_t d_tmem, uint32_t q_smem, uint
   }
 }
 
-// O_t (+)= P_t V_j: A = P_t from TMEM (packed bf16, 8 columns per 16 keys),
-// B = V_j MN-major (LBO = next 64-column panel, SBO = next 8 keys).
+// O_t (+)= P_t V_j: A = P_t from TMEM (packed bf16, 8 columns per 16 keys;
+// keys 64..127 start 64 columns further on), B = V_j MN-major (LBO = next
+// 64-column panel, SBO = next 8 keys).
 template <int D>
-__device__ __noinline__ void issue_pv_tile(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem,
-                                           bool acc) {
+__device__ __forceinline__ void issue_pv_tile(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem,
+                                              bool acc) {
   const uint64_t vd = sm100::sdesc_sw128(v_smem, CHUNK_BYTES, 1024);
 #pragma unroll
   for (int k = 0; k < BN / 16; ++k)
-    sm100::mma_ts(o_tmem, p_tmem + k * 8, vd + static_cast<uint64_t>((k * 2048) >> 4),
-                  Cfg<D>::IDESC_PV, (acc || k > 0) ? 1u : 0u);
+    sm100::mma_ts(o_tmem, p_tmem + (k >> 2) * 64 + (k & 3) * 8,
+                  vd + static_cast<uint64_t>((k * 2048) >> 4), Cfg<D>::IDESC_PV,
+                  (acc || k > 0) ? 1u : 0u);
 }
 
 template <int D>
@@ -187,24 +201,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     sm100::mbar_init(q_empty, 1);
     for (int t = 0; t < 2; ++t) {
       sm100::mbar_init(&s_full[t], 1);
-      sm100::mbar_init(&p_full[t], 128);
+      sm100::mbar_init(&p_full[t], NSMX / 2);  // one arrival per softmax warp of the tile
       sm100::mbar_init(&o_full[t], 1);
-      sm100::mbar_init(&o_empty[t], 128);
+      sm100::mbar_init(&o_empty[t], NSMX / 2);
     }
     sm100::mbar_init(drain, 1);
     for (int i = 0; i < NI; ++i) {
       sm100::mbar_init(&item_full[i], 1);
-      sm100::mbar_init(&item_empty[i], 1 + 256);  // the MMA thread + both softmax warpgroups
+      sm100::mbar_init(&item_empty[i], 1 + 32 * NSMX);  // the MMA thread + all softmax threads
     }
     *abort_flag = 0;
     sm100::fence_barrier_init();
   }
-  if (warp == 8 && sm100::lane_id() == 0) {
+  if (warp == W_LOAD && sm100::lane_id() == 0) {
     sm100::prefetch_tmap(&tmQ);
     sm100::prefetch_tmap(&tmK);
     sm100::prefetch_tmap(&tmV);
   }
-  if (warp == 9) {
+  if (warp == W_MMA) {
     sm100::tmem_alloc(tmem_slot, 512);
     sm100::tmem_relinquish();
   }
@@ -221,7 +235,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     return true;
   };
 
-  if (warp == 8) {
+  if (warp == W_LOAD) {
     // ------------------------------------------------------------ scheduler + TMA producer
     if (sm100::lane_id() == 0) {
       uint32_t use = 0;
@@ -263,27 +277,46 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!ok) break;
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == W_MMA) {
     // ------------------------------------------------------------ MMA issuer
-    if (sm100::lane_id() == 0) {
+    // The whole warp runs the loop so that its warp-uniform values (slots,
+    // parities, descriptors) live in uniform registers; one elected lane
+    // issues the tensor-core instructions.  Issue is close to synchronous (an
+    // MMA is accepted about when the previous one starts), so any per-MMA
+    // scalar work between them idles the tensor pipe: measured on B200,
+    // lane-0-only code with out-of-line issue functions ran this kernel at
+    // 0.306 ms (causal B4 H16 L4096 d128), inlined issue at 0.270 ms, and
+    // this warp-wide form at 0.254 ms.
+    const bool leader = sm100::elect_one();
+    {
       uint32_t use = 0;
       uint32_t pc0 = 0, pc1 = 0;  // P tiles consumed per query tile
       bool ok = true;
       const uint32_t q_addr = sbase + C::OFF_Q;
       const uint32_t kv_addr = sbase + C::OFF_KV;
 
+      auto commit = [&](uint64_t* b) {
+        if (leader) sm100::tc_commit(b);
+        __syncwarp();
+      };
       auto issue_s = [&](int t, int slot) {
-        issue_s_tile<D>(tmem + C::s_col(t), q_addr + t * C::TILE_BYTES,
-                        kv_addr + slot * C::TILE_BYTES);
+        if (leader)
+          issue_s_tile<D>(tmem + C::s_col(t), q_addr + t * C::TILE_BYTES,
+                          kv_addr + slot * C::TILE_BYTES);
       };
       auto issue_pv = [&](int t, int slot, bool acc) {
-        issue_pv_tile<D>(tmem + C::o_col(t), tmem + C::s_col(t), kv_addr + slot * C::TILE_BYTES,
-                         acc);
+        if (leader)
+          issue_pv_tile<D>(tmem + C::o_col(t), tmem + C::s_col(t),
+                           kv_addr + slot * C::TILE_BYTES, acc);
       };
 
       for (uint32_t k = 0; ok; ++k) {
         int w;
-        if (!(ok = next_item(k, w)) || w < 0) break;
+        if (!(ok = sm100::mbar_wait(&item_full[k % NI], (k / NI) & 1, abort_flag, p.status))) break;
+        w = *reinterpret_cast<volatile int*>(&item_ring[k % NI]);
+        __syncwarp();
+        if (leader) sm100::mbar_arrive(&item_empty[k % NI]);
+        if (w < 0) break;
         const Item it = get_item(p, w, nullptr);
         if (!(ok = sm100::mbar_wait(q_full, k & 1, abort_flag, p.status))) break;
         sm100::tc_fence_after();
@@ -295,13 +328,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           sm100::tc_fence_after();
           if (it.n0 > 0) {
             issue_s(0, ks);
-            sm100::tc_commit(&s_full[0]);
+            commit(&s_full[0]);
           }
           if (it.n1 > 0) {
             issue_s(1, ks);
-            sm100::tc_commit(&s_full[1]);
+            commit(&s_full[1]);
           }
-          sm100::tc_commit(&kv_empty[ks]);
+          commit(&kv_empty[ks]);
         }
         for (int j = 0; j < it.nmax && ok; ++j) {
           const uint32_t vuse = use + 2 * j + 1;
@@ -321,7 +354,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               ++pc;
               sm100::tc_fence_after();
               issue_pv(t, vs, j > 0);
-              if (j == n_t - 1) sm100::tc_commit(&o_full[t]);
+              if (j == n_t - 1) commit(&o_full[t]);
             }
             if (j + 1 < n_t) {
               if (!k_ready) {
@@ -331,41 +364,47 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 k_ready = true;
               }
               issue_s(t, ks);
-              sm100::tc_commit(&s_full[t]);
+              commit(&s_full[t]);
             }
             return true;
           };
           if (!(ok = step(0, it.n0, pc0))) break;
           if (!(ok = step(1, it.n1, pc1))) break;
-          if (k_ready) sm100::tc_commit(&kv_empty[ks]);
-          sm100::tc_commit(&kv_empty[vs]);
+          if (k_ready) commit(&kv_empty[ks]);
+          commit(&kv_empty[vs]);
         }
         if (!ok) break;
         if (it.n0 == 0) {
           if (!(ok = sm100::mbar_wait(&o_empty[0], oe_par, abort_flag, p.status))) break;
-          sm100::tc_commit(&o_full[0]);
+          commit(&o_full[0]);
         }
         if (it.n1 == 0) {
           if (!(ok = sm100::mbar_wait(&o_empty[1], oe_par, abort_flag, p.status))) break;
-          sm100::tc_commit(&o_full[1]);
+          commit(&o_full[1]);
         }
-        sm100::tc_commit(q_empty);
+        commit(q_empty);
         use += 2 * it.nmax;
       }
       // all issued tensor-core work (and its commits) must land before TMEM is freed
-      sm100::tc_commit(drain);
+      commit(drain);
       sm100::mbar_wait_drain(drain, 0);
     }
   } else {
-    // ------------------------------------------------------------ softmax warpgroups
-    const int t = warp >> 2;            // query tile of this warpgroup
-    const int r = threadIdx.x & 127;    // row within the tile = TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t s_addr = tmem + lane_base + C::s_col(t);
-    const uint32_t o_addr = tmem + lane_base + C::o_col(t);
+    // ------------------------------------------------------------ softmax warps
+    const int t = warp >> 3;          // query tile
+    const int hf = (warp >> 2) & 1;   // key-column half: columns [64 hf, 64 hf + 64)
+    const int qd = warp & 3;          // lane quarter
+    const int r = qd * 32 + sm100::lane_id();  // row within the tile = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
+    const uint32_t s_addr = tmem + lane_base + C::s_col(t) + 64 * hf;
+    constexpr int DH = D / 2;  // output columns this thread rescales and writes
+    const uint32_t o_addr = tmem + lane_base + C::o_col(t) + DH * hf;
+    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);    // [2][2][2][BM]
+    float* lsum_x = reinterpret_cast<float*>(smem + C::OFF_LSUM);  // [2][2][2][BM]
+    const int bar_id = 1 + t * 4 + qd;  // named barrier of the two warps sharing these rows
     const float sl2 = p.scale_log2;
     const float2 sl2x2 = make_float2(sl2, sl2);
-    uint32_t s_cnt = 0;
+    uint32_t s_cnt = 0, e_cnt = 0;
     bool ok = true;
 
     for (uint32_t k = 0; ok; ++k) {
@@ -381,30 +420,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       float m_use = -INFINITY, l = 0.f;
       for (int j = 0; j < n_t; ++j) {
         if (!(ok = sm100::mbar_wait(&s_full[t], s_cnt & 1, abort_flag, p.status))) break;
+        float* red_w = red + ((s_cnt & 1) * 4 + t * 2) * BM;
         ++s_cnt;
         sm100::tc_fence_after();
-        uint32_t s[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          sm100::tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
+        uint32_t s[64];
+        sm100::tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        sm100::tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
         sm100::tmem_ld_wait();
 
-        const int k0 = j * BN;
+        const int k0 = j * BN + 64 * hf;
         const bool need_mask =
-            (k0 + BN > it.kv_len) || (p.causal && (k0 + BN - 1 > row0 + (p.Lk - p.Lq)));
+            (k0 + 64 > it.kv_len) || (p.causal && (k0 + 63 > row0 + (p.Lk - p.Lq)));
         if (need_mask) {
           const int lim = p.causal ? min(it.kv_len - 1, diag) : it.kv_len - 1;
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
+          for (int c = 0; c < 64; ++c)
             if (k0 + c > lim) s[c] = __float_as_uint(-INFINITY);
         }
         float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 128; c += 4) {
+        for (int c = 0; c < 64; c += 4) {
           mx0 = sm100::max3(mx0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
           mx1 = sm100::max3(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
         }
-        const float m_new = fmaxf(mx0, mx1) * sl2;
+        // the row max over all 128 keys: exchange with the warp holding the other half
+        red_w[hf * BM + r] = fmaxf(mx0, mx1);
+        sm100::named_bar_sync(bar_id, 64);
+        const float m_new = fmaxf(fmaxf(mx0, mx1), red_w[(hf ^ 1) * BM + r]) * sl2;
         const bool need = m_new > m_use + RESCALE_THRESHOLD;
         if (__any_sync(0xffffffffu, need)) {
           const float m_upd = fmaxf(m_use, m_new);
@@ -412,15 +454,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           l *= alpha;
           if (j > 0) {
             // O holds PV of the previous tiles (complete: S of this tile was
-            // committed after them); rescale it in place
+            // committed after them); rescale this thread's half in place
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t o[32];
-              sm100::tmem_ld32(o_addr + c * 32, o);
+            for (int c = 0; c < DH / 16; ++c) {
+              uint32_t o[16];
+              sm100::tmem_ld16(o_addr + c * 16, o);
               sm100::tmem_ld_wait();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              sm100::tmem_st32(o_addr + c * 32, o);
+              for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              sm100::tmem_st16(o_addr + c * 16, o);
             }
           }
           m_use = m_upd;
@@ -428,10 +470,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
         const float2 negm = make_float2(-m_sub, -m_sub);
         float2 lsum = make_float2(0.f, 0.f);
-        // exponentials in four 32-column chunks; each chunk's P (packed bf16)
+        // exponentials in two 32-column chunks; each chunk's P (packed bf16)
         // is stored to TMEM while the next chunk is computed
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
 #pragma unroll
           for (int cp = 16 * q; cp < 16 * q + 16; ++cp) {
             const float2 x = __ffma2_rn(
@@ -452,19 +494,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         l += lsum.x + lsum.y;
         sm100::tmem_st_wait();
         sm100::tc_fence_before();
-        sm100::mbar_arrive(&p_full[t]);
+        __syncwarp();
+        if (sm100::lane_id() == 0) sm100::mbar_arrive(&p_full[t]);
       }
       if (!ok) break;
       // ---------------- epilogue: O = o / l (bf16), LSE = ln(2) * (m + log2 l)
       if (!(ok = sm100::mbar_wait(&o_full[t], k & 1, abort_flag, p.status))) break;
       sm100::tc_fence_after();
+      if (n_t > 0) {
+        float* lx = lsum_x + ((e_cnt & 1) * 4 + t * 2) * BM;
+        ++e_cnt;
+        lx[hf * BM + r] = l;
+        sm100::named_bar_sync(bar_id, 64);
+        l += lx[(hf ^ 1) * BM + r];
+      }
       const bool live = row < p.Lq;
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       __nv_bfloat16* orow =
-          p.O + ((static_cast<size_t>(it.b) * p.Hq + it.h) * p.Lq + (live ? row : 0)) * D;
+          p.O + ((static_cast<size_t>(it.b) * p.Hq + it.h) * p.Lq + (live ? row : 0)) * D + DH * hf;
       if (n_t > 0) {
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < DH / 32; ++c) {
           uint32_t o[32];
           sm100::tmem_ld32(o_addr + c * 32, o);
           sm100::tmem_ld_wait();
@@ -482,19 +532,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       } else if (live) {
         uint4* dst = reinterpret_cast<uint4*>(orow);
-        for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0, 0, 0, 0);
+        for (int v = 0; v < DH / 8; ++v) dst[v] = make_uint4(0, 0, 0, 0);
       }
-      if (live && p.lse)
+      if (live && p.lse && hf == 0)
         p.lse[(static_cast<size_t>(it.b) * p.Hq + it.h) * p.Lq + row] =
             (l > 0.f) ? (m_use + log2f(l)) * 0.69314718055994531f : -INFINITY;
       sm100::tc_fence_before();
-      sm100::mbar_arrive(&o_empty[t]);
+      __syncwarp();
+      if (sm100::lane_id() == 0) sm100::mbar_arrive(&o_empty[t]);
     }
   }
 
   sm100::tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == W_MMA) {
     sm100::tc_fence_after();
     sm100::tmem_dealloc(tmem, 512);
   }
