@@ -1,6 +1,6 @@
 // bwd_kernel.cuh -- attention backward by recomputation on sm_100a.
 //
-// "FlashAttention and long context: three ledgers" (page 1, online-softmax
+// "FlashAttention and long context: three ledgers" (online-softmax
 // section) states the backward keeps only small per-row statistics and
 // recomputes the score blocks it needs, trading compute for memory traffic.
 // With the saved LSE (and D_i = sum_d dO_id O_id) every score tile is rebuilt

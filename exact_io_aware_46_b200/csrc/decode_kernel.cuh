@@ -6,14 +6,15 @@
 // (4 FLOP/B with 4 query heads per key/value head), so the kernel is bound by
 // HBM bandwidth, not by the tensor core.  It therefore runs on CUDA cores:
 //
-//  * split kernel: one CTA per (sequence, key/value head, chunk of CH keys).
+//  * split kernel: one CTA per (sequence, key/value head, chunk of CH keys),
+//    three CTAs per SM.
 //    A producer thread streams the chunk's K and V rows (contiguous in the
 //    cache) with 1-D bulk copies into a ring of shared-memory stages; four
 //    compute warps each own 16 rows of every stage.  A half-warp covers one
 //    key row (16 lanes x d/16 elements), forms partial dot products with all
 //    query heads of the group (packed fp32x2 FMA), and a transpose-reduction
 //    across the 16 lanes leaves every lane with one complete (row, head)
-//    score.  The online softmax of page 1 runs per warp with a stale-max
+//    score.  The online softmax of the three-ledgers page runs per warp with a stale-max
 //    rescale threshold; warps are merged at the end and the chunk's
 //    normalised output and log2-sum-exp are written as a partial.
 //  * combine kernel: merges a sequence's partials with the normalised rule of
@@ -26,9 +27,16 @@
 
 namespace attn_decode_impl {
 
-constexpr int CH = 1024;  // keys per split
+// Measured on B200 (B64 Hq32 Hkv8 d128, cache 32768, k_len ~ U[1024, 32768]):
+// chunk 1024 / 3 stages / 2 CTAs per SM 5.56 TB/s; 2 stages / 3 CTAs per SM
+// 5.98 TB/s; chunk 2048 with 2 stages / 3 CTAs per SM 6.11 TB/s (shipped);
+// chunk 4096 5.88 TB/s, chunk 512 5.01 TB/s.  More resident warps hide the
+// shared-memory and shuffle latency of the compute warps; longer chunks
+// amortise a CTA's start (query load, first copy) and its final merge.
+constexpr int CH = 2048;  // keys per split
 constexpr int SR = 64;    // key rows per shared-memory stage
-constexpr int NST = 3;    // stages
+constexpr int NST = 2;    // stages
+constexpr int CTAS_PER_SM = 3;
 constexpr int NCW = 4;    // compute warps
 constexpr int NTHREADS = (NCW + 1) * 32;
 
@@ -109,11 +117,12 @@ __device__ __forceinline__ float transpose_reduce16(float (&v)[16], int hl) {
 
 // GP: query heads per key/value head, padded to 4 or 8 (heads >= G are inert).
 template <int D, int GP>
-__global__ void __launch_bounds__(NTHREADS, 2) decode_split_kernel(const SplitParams p) {
+__global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) decode_split_kernel(const SplitParams p) {
   constexpr int EPL = D / 16;    // elements of a row per lane
   constexpr int R = 16 / GP;     // rows per half-warp per step
   constexpr int STEP = 2 * R;    // rows per warp per step
   constexpr int WROWS = SR / NCW;
+  static_assert(SR % NCW == 0 && WROWS % STEP == 0, "a warp's rows of a stage must be whole steps");
   constexpr int ROWB = D * 2;    // bytes per row
   constexpr int STAGE = SR * ROWB;  // bytes of K (or V) per stage
 

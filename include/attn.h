@@ -29,8 +29,9 @@
  *   sequence b is visible iff j < k_lens[b].  Both combine by AND.  A query row
  *   with no visible key gets O = 0, LSE = -inf and zero gradients.
  * - LSE is the natural-log log-sum-exp of the row's scaled, masked scores: the
- *   per-row statistic the backward recomputes from (page 1: the backward keeps
- *   small row statistics and recomputes score blocks).
+ *   per-row statistic the backward recomputes from (the three-ledgers page,
+ *   online-softmax section: the backward keeps small row statistics and
+ *   recomputes score blocks).
  * - Ownership: the caller allocates and owns every buffer, including the
  *   workspace, and the stream.  The library never allocates, frees or
  *   synchronises, except attn_read_device_status (which synchronises `stream`).
@@ -79,7 +80,7 @@ const char* attn_status_string(attn_status_t s);
 
 /* ------------------------------------------------------------------ forward
  * Prefill / training forward.  Defined by the attention formula and the online
- * softmax of page 1 (m' = max(m, max S_j); l' = e^{m-m'} l + sum e^{S_j-m'};
+ * softmax of the three-ledgers page (m' = max(m, max S_j); l' = e^{m-m'} l + sum e^{S_j-m'};
  * o' = e^{m-m'} o + sum e^{S_j-m'} V_j; O = o / l), with the tiling of the
  * FlashAttention-2 tutorial, 2.1.2.
  *
@@ -97,7 +98,8 @@ attn_status_t attn_fwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf
 
 /* ------------------------------------------------------------------ decode
  * Split-KV decode (one query token per sequence over a contiguous KV cache):
- * the "short query scans a long history" case of page 1 (prefill vs decode).
+ * the "short query scans a long history" case of the three-ledgers page
+ * (section on prefill vs decode).
  * The cache rows [0, k_lens[b]) of each sequence are split into chunks; each
  * chunk yields a partial (m, l, O) and the partials are combined with the
  * normalised merge of the FlashAttention-2 tutorial, 2.1.3:
@@ -117,7 +119,7 @@ attn_status_t attn_fwd_splitkv_decode(const attn_bf16_t* Q, const attn_bf16_t* K
                                       void* stream);
 
 /* ------------------------------------------------------------------ backward
- * Backward by recomputation: page 1 says the backward keeps only small row
+ * Backward by recomputation: the three-ledgers page says the backward keeps only small row
  * statistics and recomputes the score blocks it needs.  From the saved LSE
  * (and D_i = sum_d dO_id O_id) each score tile is rebuilt as
  * P = exp(S * scale - LSE), and
@@ -149,7 +151,7 @@ attn_status_t attn_bwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf
  *
  * Scratch: a file-scope device array of ATTN_NOALLOC_SCRATCH_BYTES that every
  * GPU loading the library holds until the process exits.  A request whose
- * partials need more (256 + B*Hq*ceil(Lmax/1024)*(4*d + 4) bytes, rounded up to
+ * partials need more (256 + B*Hq*ceil(Lmax/2048)*(4*d + 4) bytes, rounded up to
  * 256) returns ATTN_ERR_CAPACITY before anything is launched.  The first call
  * on a device looks up the array's device address (cudaGetSymbolAddress, with
  * that device current); make that first call before any stream capture.  The

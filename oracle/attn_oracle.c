@@ -8,7 +8,7 @@
  * What it computes (no tiling, no fusion, no reordering beyond the definition):
  *
  *   Attention definition, "FlashAttention and long context: three ledgers"
- *   (page 1), section "the problem with standard attention is not only FLOPs":
+ *   section "the problem with standard attention is not only FLOPs":
  *       O = softmax((Q K^T + M) / sqrt(d_h)) V
  *   and the three-step naive form of the FlashAttention-2 tutorial, 2.1.1:
  *       S = Q K^T * scale ; P = softmax(S) along keys ; O = P V.
@@ -23,15 +23,15 @@
  *     a row with no visible key has O = 0 and LSE = -inf.
  *
  *   LSE_i = m_i + ln(sum_j exp(S_ij - m_i)) over visible j: the per-row
- *   statistic that page 1 says the backward keeps.
+ *   statistic that the same page says the backward keeps.
  *
- *   Backward (page 1 only says the backward recomputes score blocks from saved
+ *   Backward (that page only says the backward recomputes score blocks from saved
  *   row statistics; the formulas are the calculus of the definition):
  *       dV = P^T dO ; dP = dO V^T ; D_i = sum_j P_ij dP_ij ;
  *       dS = P o (dP - D) ; dQ = scale dS K ; dK = scale dS^T Q.
  *
  *   Online softmax, for the equivalence pins only (never the parity reference):
- *     unnormalised form of page 1 ("the key is online softmax"):
+ *     unnormalised form of the three-ledgers page ("the key is online softmax"):
  *       m' = max(m, max S_j); l' = e^{m-m'} l + sum_t e^{S_jt - m'};
  *       o' = e^{m-m'} o + sum_t e^{S_jt - m'} V_jt; O = o / l.
  *     normalised merge of the FlashAttention-2 tutorial, 2.1.3:

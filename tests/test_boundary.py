@@ -40,8 +40,8 @@ def test_workspace_sizes_are_closed_forms(lib):
     import exact_io_aware_46_b200 as attn
 
     assert attn.attn_fwd_workspace_size(4, 16, 16, 4096, 4096, 128) == 256
-    # decode: fp32 partial output and log-sum-exp per (sequence, head, 1024-key chunk)
-    n = 64 * 32 * 32
+    # decode: fp32 partial output and log-sum-exp per (sequence, head, 2048-key chunk)
+    n = 64 * 32 * 16
     assert attn.attn_decode_workspace_size(64, 32, 8, 32768, 128) == 256 + ((n * 128 * 4 + n * 4 + 255) // 256) * 256
     # backward: fp32 dQ accumulator and D per query row; nothing of size Lq x Lk
     rows = 2 * 16 * 8192  # query rows, padded per head to a multiple of 64

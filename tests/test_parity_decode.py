@@ -30,7 +30,8 @@ def _run(Q, K, V, k_lens, scale):
 
 CASES = [
     # B, Hq, Hkv, Lmax, d, k_lens
-    (3, 8, 2, 3000, 128, [2500, 1, 1024]),        # chunk boundary, single key, exact chunk
+    (3, 8, 2, 3000, 128, [2500, 1, 2048]),        # chunk boundary, single key, exact chunk
+    (1, 4, 1, 5000, 128, [4097]),                 # three chunks, the last holding one key
     (2, 4, 4, 2100, 128, [2049, 2100]),           # G = 1 (padded to 4 lanes' heads)
     (2, 16, 2, 1500, 128, [1500, 777]),           # G = 8
     (2, 4, 2, 1300, 64, [1300, 65]),              # d = 64, G = 2

@@ -52,7 +52,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
     scale = 1.0 / math.sqrt(d)
     Q, K, V = _inputs(71, B, Hq, Hkv, Lmax, d)
     # two calls in a row with different lengths: stale partials of the first
-    # call (three 1024-key chunks of sequence 0) must not reach the second
+    # call (two 2048-key chunks of sequence 0) must not reach the second
     for k_lens in ([2600, 1, 1024], [700, 2048, 0]):
         kl = torch.tensor(k_lens, dtype=torch.int32, device="cuda")
         ref_O, ref_L = attn.attn_fwd_splitkv_decode(Q, K, V, kl, scale=scale)
