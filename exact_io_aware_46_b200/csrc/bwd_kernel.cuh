@@ -150,10 +150,6 @@ __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
                                          uint64_t* bar) {
   asm volatile(
@@ -321,21 +317,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (sm100::lane_id() == 0) {
+    // The whole warp runs the loop (warp-uniform values stay in uniform
+    // registers) and one elected lane issues; descriptors are built once per
+    // operand and stepped by constant offsets.  MMA issue is close to
+    // synchronous, so scalar work between two MMAs idles the tensor pipe.
+    const bool leader = sm100::elect_one();
+    {
       uint32_t tq = 0, ik = 0;
       bool ok = true;
       const uint32_t kA = sbase + OFF_K, vA = sbase + OFF_V;
       auto qA = [&](int slot) { return sbase + OFF_QS + slot * QS_BYTES; };
       auto doA = [&](int slot) { return sbase + OFF_QS + slot * QS_BYTES + 16384; };
       auto dsA = [&](int b) { return sbase + OFF_DS + b * 16384; };
+      auto commit = [&](uint64_t* bar) {
+        if (leader) sm100::tc_commit(bar);
+        __syncwarp();
+      };
       // S^T (or dP^T) = A_keys[128 x d] * B_rows[64 x d]^T, both K-major
       auto issue_kmajor = [&](uint32_t dcol, uint32_t a, uint32_t b) {
+        const uint64_t ad = sm100::sdesc_sw128(a, 16, 1024);
+        const uint64_t bd = sm100::sdesc_sw128(b, 16, 1024);
+        if (leader) {
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          sm100::mma_ss(tmem + dcol,
-                        sm100::sdesc_sw128(a + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
-                        sm100::sdesc_sw128(b + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024),
-                        IDESC_S, k > 0);
+          for (int k = 0; k < D / 16; ++k)
+            sm100::mma_ss(tmem + dcol, ad + (((k >> 2) * 16384 + (k & 3) * 32) >> 4),
+                          bd + (((k >> 2) * 8192 + (k & 3) * 32) >> 4), IDESC_S, k > 0);
         }
       };
       for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x, ++ik) {
@@ -344,8 +350,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         sm100::tc_fence_after();
         if (it.T == 0) {
           if (!(ok = sm100::mbar_wait(dkv_empty, (ik & 1) ^ 1, abort_flag, p.status))) break;
-          sm100::tc_commit(dkv_full);
-          sm100::tc_commit(kv_empty);
+          commit(dkv_full);
+          commit(kv_empty);
           continue;
         }
         // Issue order per query tile t (buffers b = t & 1, nb = (t + 1) & 1):
@@ -358,13 +364,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             break;
           sm100::tc_fence_after();
           issue_kmajor(S_COL0 + b * 64, kA, qA(slot));
-          sm100::tc_commit(&s_full[b]);
+          commit(&s_full[b]);
           if (!(ok = sm100::mbar_wait(&dq_empty[b], ((tq >> 1) & 1) ^ 1, abort_flag, p.status)))
             break;
           sm100::tc_fence_after();
           issue_kmajor(DP_COL0 + b * 64, vA, doA(slot));
-          sm100::tc_commit(&dp_full[b]);
+          commit(&dp_full[b]);
         }
+        const uint64_t kd_mn = sm100::sdesc_sw128(kA, 16384, 1024);  // K as MN-major A (over d)
         for (int t = 0; t < it.T && ok; ++t) {
           const uint32_t cur = tq + t;
           const int slot = cur % NQS, b = cur & 1;
@@ -377,7 +384,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               break;
             sm100::tc_fence_after();
             issue_kmajor(S_COL0 + nb * 64, kA, qA(ns));
-            sm100::tc_commit(&s_full[nb]);
+            commit(&s_full[nb]);
           }
           if (!(ok = sm100::mbar_wait(&p_full[b], u & 1, abort_flag, p.status))) break;
           sm100::tc_fence_after();
@@ -385,44 +392,49 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!(ok = sm100::mbar_wait(dkv_empty, (ik & 1) ^ 1, abort_flag, p.status))) break;
             sm100::tc_fence_after();
           }
+          const uint64_t do_mn = sm100::sdesc_sw128(doA(slot), 8192, 1024);
+          const uint64_t q_mn = sm100::sdesc_sw128(qA(slot), 8192, 1024);
+          const uint64_t ds_k = sm100::sdesc_sw128(dsA(b), 16, 1024);
+          const uint64_t ds_mn = sm100::sdesc_sw128(dsA(b), 8192, 1024);
           // dV += P^T dO : A = P^T (TMEM, packed bf16), B = dO (MN-major)
+          if (leader) {
 #pragma unroll
-          for (int k = 0; k < BMQ / 16; ++k)
-            sm100::mma_ts(tmem + DV_COL, tmem + S_COL0 + b * 64 + k * 8,
-                          sm100::sdesc_sw128(doA(slot) + k * 2048, 8192, 1024), IDESC_DV,
-                          (t > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < BMQ / 16; ++k)
+              sm100::mma_ts(tmem + DV_COL, tmem + S_COL0 + b * 64 + k * 8, do_mn + ((k * 2048) >> 4),
+                            IDESC_DV, (t > 0 || k > 0) ? 1u : 0u);
+          }
           if (more) {
             if (!(ok = sm100::mbar_wait(&dq_empty[nb], ((nx >> 1) & 1) ^ 1, abort_flag,
                                         p.status)))
               break;
             sm100::tc_fence_after();
             issue_kmajor(DP_COL0 + nb * 64, vA, doA(ns));
-            sm100::tc_commit(&dp_full[nb]);
+            commit(&dp_full[nb]);
           }
           if (!(ok = sm100::mbar_wait(&ds_full[b], u & 1, abort_flag, p.status))) break;
           sm100::tc_fence_after();
-          // dK += dS^T Q : A = dS^T (K-major over rows), B = Q (MN-major)
+          if (leader) {
+            // dK += dS^T Q : A = dS^T (K-major over rows), B = Q (MN-major)
 #pragma unroll
-          for (int k = 0; k < BMQ / 16; ++k)
-            sm100::mma_ss(tmem + DK_COL, sm100::sdesc_sw128(dsA(b) + k * 32, 16, 1024),
-                          sm100::sdesc_sw128(qA(slot) + k * 2048, 8192, 1024), IDESC_DV,
-                          (t > 0 || k > 0) ? 1u : 0u);
-          // dQ^T = K^T dS^T : A = K (MN-major over d), B = dS^T (MN-major over rows)
+            for (int k = 0; k < BMQ / 16; ++k)
+              sm100::mma_ss(tmem + DK_COL, ds_k + ((k * 32) >> 4), q_mn + ((k * 2048) >> 4),
+                            IDESC_DV, (t > 0 || k > 0) ? 1u : 0u);
+            // dQ^T = K^T dS^T : A = K (MN-major over d), B = dS^T (MN-major over rows)
 #pragma unroll
-          for (int k = 0; k < BN / 16; ++k)
-            sm100::mma_ss(tmem + DP_COL0 + b * 64, sm100::sdesc_sw128(kA + k * 2048, 16384, 1024),
-                          sm100::sdesc_sw128(dsA(b) + k * 2048, 8192, 1024), IDESC_DQ,
-                          k > 0 ? 1u : 0u);
-          sm100::tc_commit(&dq_full[b]);
-          sm100::tc_commit(&ds_empty[b]);
-          sm100::tc_commit(&qdo_empty[slot]);
+            for (int k = 0; k < BN / 16; ++k)
+              sm100::mma_ss(tmem + DP_COL0 + b * 64, kd_mn + ((k * 2048) >> 4),
+                            ds_mn + ((k * 2048) >> 4), IDESC_DQ, k > 0 ? 1u : 0u);
+          }
+          commit(&dq_full[b]);
+          commit(&ds_empty[b]);
+          commit(&qdo_empty[slot]);
         }
         if (!ok) break;
         tq += it.T;
-        sm100::tc_commit(dkv_full);
-        sm100::tc_commit(kv_empty);
+        commit(dkv_full);
+        commit(kv_empty);
       }
-      sm100::tc_commit(drain);
+      commit(drain);
       sm100::mbar_wait_drain(drain, 0);
     }
   } else if (warp < 4) {
@@ -519,7 +531,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int q = 0; q < 8; ++q)
           *reinterpret_cast<uint4*>(line + ((q ^ (kl_ & 7)) << 4)) =
               make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        fence_proxy_async_smem();
+        sm100::fence_proxy_async_smem();
         sm100::tc_fence_before();
         sm100::mbar_arrive(&ds_full[b]);
       }
@@ -589,7 +601,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         sm100::named_bar_sync(1, 128);
 #pragma unroll
         for (int c = 0; c < 64; ++c) stage[c * D + dl] = __uint_as_float(v[c]);
-        fence_proxy_async_smem();
+        sm100::fence_proxy_async_smem();
         sm100::named_bar_sync(1, 128);
         if (threadIdx.x == 128) {
           const int qh = it.b * p.Hq + it.hkv * p.G + g;
