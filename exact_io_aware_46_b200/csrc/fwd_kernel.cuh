@@ -336,6 +336,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
           commit(&kv_empty[ks]);
         }
+        // Q is free once the item's last S has run: release it then, so the next
+        // item's Q loads while this item's last PV steps execute
+        if (it.nmax <= 1) commit(q_empty);
         for (int j = 0; j < it.nmax && ok; ++j) {
           const uint32_t vuse = use + 2 * j + 1;
           const int vs = vuse % C::NS;
@@ -372,6 +375,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!(ok = step(1, it.n1, pc1))) break;
           if (k_ready) commit(&kv_empty[ks]);
           commit(&kv_empty[vs]);
+          if (j + 2 == it.nmax) commit(q_empty);  // S_t(nmax - 1) were the last S
         }
         if (!ok) break;
         if (it.n0 == 0) {
@@ -382,7 +386,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!(ok = sm100::mbar_wait(&o_empty[1], oe_par, abort_flag, p.status))) break;
           commit(&o_full[1]);
         }
-        commit(q_empty);
         use += 2 * it.nmax;
       }
       // all issued tensor-core work (and its commits) must land before TMEM is freed
