@@ -299,9 +299,33 @@ def decode_leg(steps, warmup, world, flush):
     if st[0] != attn.ATTN_OK:
         raise RuntimeError(f"device status {st}")
     kv_bytes = float(np.sum(k_lens.astype(np.int64))) * c["Hkv"] * c["d"] * 2 * 2
+    # the same workload over a paged cache: 64-row pages in a seeded random order
+    page = 64
+    nb = c["Lmax"] // page
+    order = torch.from_numpy(
+        np.argsort(synth.uniform_u64(synth.workload_seed(4, "pages"), c["B"] * nb),
+                   kind="stable")).to(dev)
+    table = order.view(c["B"], nb).to(torch.int32).contiguous()
+
+    def to_pages(cache):
+        blocks = cache.view(c["B"], c["Hkv"], nb, page, c["d"]).permute(0, 2, 1, 3, 4)
+        out = torch.empty((c["B"] * nb, c["Hkv"], page, c["d"]), dtype=cache.dtype, device=dev)
+        out[order] = blocks.reshape(c["B"] * nb, c["Hkv"], page, c["d"])
+        return out
+
+    kp, vp = to_pages(kc), to_pages(vc)
     del kc, vc
     torch.cuda.empty_cache()
-    return ms, kv_bytes, k_lens
+    call_p = lambda: attn.attn_fwd_splitkv_decode_paged(q, kp, vp, table, kl, O=O, lse=lse,
+                                                        workspace=ws, stream=stream)
+    barrier(world)
+    pms = timed_loop(call_p, steps, warmup, stream, flush)
+    st = attn.attn_read_device_status(ws)
+    if st[0] != attn.ATTN_OK:
+        raise RuntimeError(f"device status {st}")
+    del kp, vp
+    torch.cuda.empty_cache()
+    return ms, kv_bytes, k_lens, (page, pms)
 
 
 def bwd_leg(steps, warmup, world, flush):
@@ -446,7 +470,7 @@ def main():
         if "fwd" in legs:
             ms, ms_e2e, h2d, d2h = fwd_leg(args.steps, args.warmup, world, flush)
         if "decode" in legs:
-            dms, kv_bytes, _ = decode_leg(args.steps, args.warmup, world, flush)
+            dms, kv_bytes, _, (page, pms) = decode_leg(args.steps, args.warmup, world, flush)
         if "bwd" in legs:
             bms = bwd_leg(max(3, args.steps // 2), args.warmup, world, flush)
         else:
@@ -457,6 +481,7 @@ def main():
         if "decode" in legs:
             rep["decode_ms"] = float(np.mean(dms))
             rep["decode_GBs"] = kv_bytes / (float(np.mean(dms)) * 1e-3) / 1e9
+            rep["decode_paged_GBs"] = kv_bytes / (float(np.mean(pms)) * 1e-3) / 1e9
         if bms is not None:
             rep["bwd_ms"] = float(np.mean(bms))
             rep["bwd_TFLOPs"] = bwd_flops(BWD) / (float(np.mean(bms)) * 1e-3) / 1e12
@@ -506,9 +531,16 @@ def main():
                          "traffic": traffic_per_launch(
                              "attn_decode_impl::decode_split_kernel<128,4>", kv_bytes),
                          "kernel": "attn_decode_impl::decode_split_kernel<128,4> + combine"},
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": 4 * args.steps,
         }
-        line["gpu_launches"] += 2 * args.steps
+        t_p = max_over_ranks(float(np.mean(pms)), world)
+        line["decode"]["paged"] = {
+            "workload": f"the same decode over a cache of {page}-row pages in a seeded random "
+                        f"order (block table [64, {DEC['Lmax'] // page}])",
+            "value": world * kv_bytes / (t_p * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": t_p,
+            "page_size": page,
+        }
+        line["gpu_launches"] += 4 * args.steps
     if bms is not None:
         bfl = bwd_flops(BWD)
         t_b = max_over_ranks(float(np.mean(bms)), world)

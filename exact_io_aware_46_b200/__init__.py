@@ -9,6 +9,7 @@ The functions carry the C entry points' names:
 
 * ``attn_fwd(Q, K, V, ...) -> (O, LSE)``
 * ``attn_fwd_splitkv_decode(Q, Kcache, Vcache, k_lens, ...) -> (O, LSE)``
+* ``attn_fwd_splitkv_decode_paged(Q, Kpages, Vpages, block_table, k_lens, ...) -> (O, LSE)``
 * ``attn_bwd(Q, K, V, O, dO, LSE, ...) -> (dQ, dK, dV)``
 * the ``*_workspace_size`` queries and the device-status helpers.
 """
@@ -30,7 +31,7 @@ LIB_PATH = os.path.join(_HERE, "libattn.so")
 #: size of the fixed device scratch used by attn_fwd_splitkv_decode_noalloc
 ATTN_NOALLOC_SCRATCH_BYTES = 16 << 20
 ATTN_MASK_NONE, ATTN_MASK_CAUSAL = 0, 1
-ATTN_DEV_BAD_KLEN, ATTN_DEV_TIMEOUT = 1, 2
+ATTN_DEV_BAD_KLEN, ATTN_DEV_TIMEOUT, ATTN_DEV_BAD_PAGE = 1, 2, 4
 
 _lock = threading.Lock()
 _lib = None
@@ -55,6 +56,8 @@ SIGNATURES = {
                       _i, _vp, _vp, _sz, _vp]),
     "attn_fwd_splitkv_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f,
                                              _vp, _vp]),
+    "attn_fwd_splitkv_decode_paged": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i,
+                                           _i, _f, _vp, _vp, _sz, _vp]),
     "attn_read_device_status": (_i, [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]),
     "attn_clear_device_status": (_i, [_vp, _vp]),
 }
@@ -188,6 +191,35 @@ def attn_fwd_splitkv_decode(Q, Kc, Vc, k_lens, scale=None, O=None, lse=None, wor
                                          Hkv, Lmax, d, float(scale), _ptr(k_lens),
                                          _ptr(workspace), workspace.numel(), _stream(stream))
     _check(code, "attn_fwd_splitkv_decode")
+    return O, lse
+
+
+def attn_fwd_splitkv_decode_paged(Q, Kp, Vp, block_table, k_lens, scale=None, O=None, lse=None,
+                                  workspace=None, stream=None, want_lse=True):
+    """Split-KV decode over a paged cache.  Q [B,Hq,1,d]; Kp/Vp [n_pages,Hkv,page,d] bf16;
+    block_table int32 [B,max_blocks] and k_lens int32 [B] on the device."""
+    for t, n in ((Q, "Q"), (Kp, "Kpages"), (Vp, "Vpages")):
+        _bf16(t, n)
+    if block_table.dtype != torch.int32 or block_table.dim() != 2 or not block_table.is_contiguous():
+        raise ValueError("block_table must be a contiguous int32 [B, max_blocks] tensor")
+    B, Hq, _, d = Q.shape
+    n_pages, Hkv, page = Kp.shape[0], Kp.shape[1], Kp.shape[2]
+    max_blocks = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if O is None:
+        O = torch.empty_like(Q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=Q.device)
+    if workspace is None:
+        workspace = _workspace(attn_decode_workspace_size(B, Hq, Hkv, max_blocks * page, d),
+                               Q.device, stream)
+    code = lib().attn_fwd_splitkv_decode_paged(_ptr(Q), _ptr(Kp), _ptr(Vp), _ptr(block_table),
+                                               max_blocks, page, n_pages, _ptr(O), _ptr(lse), B,
+                                               Hq, Hkv, d, float(scale), _ptr(k_lens),
+                                               _ptr(workspace), workspace.numel(),
+                                               _stream(stream))
+    _check(code, "attn_fwd_splitkv_decode_paged")
     return O, lse
 
 

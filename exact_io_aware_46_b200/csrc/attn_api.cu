@@ -193,6 +193,41 @@ attn_status_t attn_fwd_splitkv_decode(const attn_bf16_t* Q, const attn_bf16_t* K
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+attn_status_t attn_fwd_splitkv_decode_paged(const attn_bf16_t* Q, const attn_bf16_t* Kp,
+                                            const attn_bf16_t* Vp, const int32_t* block_table,
+                                            int max_blocks, int page_size, int n_pages,
+                                            attn_bf16_t* O, float* lse, int B, int Hq, int Hkv,
+                                            int d, float scale, const int32_t* k_lens,
+                                            void* workspace, size_t ws_bytes, void* stream) {
+  if (max_blocks <= 0 || n_pages <= 0 || page_size <= 0) return ATTN_ERR_INVALID;
+  int page_log2 = 0;
+  while ((1 << page_log2) < page_size && page_log2 < 17) ++page_log2;
+  if ((1 << page_log2) != page_size || page_size < 16 || page_size > 65536)
+    return ATTN_ERR_UNSUPPORTED;
+  const long long lmax = static_cast<long long>(max_blocks) * page_size;
+  if (lmax > (1 << 30)) return ATTN_ERR_INVALID;
+  const int Lmax = static_cast<int>(lmax);
+  if (!shapes_ok(B, Hq, Hkv, 1, Lmax)) return ATTN_ERR_INVALID;
+  if (!Q || !Kp || !Vp || !block_table || !O || !k_lens || !workspace) return ATTN_ERR_INVALID;
+  if (!aligned16(Q) || !aligned16(Kp) || !aligned16(Vp) || !aligned16(block_table) ||
+      !aligned16(O) || (lse && !aligned16(lse)) || !aligned16(k_lens) || !aligned256(workspace))
+    return ATTN_ERR_INVALID;
+  if (!(std::isfinite(scale) && scale > 0.f)) return ATTN_ERR_INVALID;
+  if (ws_bytes < attn_decode_workspace_size(B, Hq, Hkv, Lmax, d)) return ATTN_ERR_INVALID;
+  if (d != 128 && d != 64) return ATTN_ERR_UNSUPPORTED;
+  if (!attn_decode_impl::supported_group(Hq / Hkv)) return ATTN_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = device_sms();
+  if (sms <= 0) return ATTN_ERR_CUDA;
+  const attn_decode_impl::PagedKV pg{block_table, max_blocks, page_log2, n_pages};
+  cudaError_t e = attn_decode_impl::launch(
+      reinterpret_cast<const __nv_bfloat16*>(Q), reinterpret_cast<const __nv_bfloat16*>(Kp),
+      reinterpret_cast<const __nv_bfloat16*>(Vp), reinterpret_cast<__nv_bfloat16*>(O), lse, B, Hq,
+      Hkv, Lmax, d, scale, k_lens, reinterpret_cast<int*>(workspace),
+      reinterpret_cast<uint8_t*>(workspace) + kStatusBytes, sms, s, &pg);
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ backward
 
 size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d) {
@@ -255,7 +290,7 @@ attn_status_t attn_read_device_status(const void* workspace, void* stream, int32
   if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
   if (bits) *bits = v;
   if (v & ATTN_DEV_TIMEOUT) return ATTN_ERR_TIMEOUT;
-  if (v & ATTN_DEV_BAD_KLEN) return ATTN_ERR_INVALID;
+  if (v & (ATTN_DEV_BAD_KLEN | ATTN_DEV_BAD_PAGE)) return ATTN_ERR_INVALID;
   return ATTN_OK;
 }
 

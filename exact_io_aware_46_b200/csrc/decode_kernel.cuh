@@ -65,6 +65,10 @@ struct SplitParams {
   float* part_lse;  // [B*Hq][nsm] log2-sum-exp of the chunk (scaled scores)
   int B, Hq, Hkv, G, Lmax, nsm;
   float scale_log2;
+  // paged cache (block_table != nullptr): K/V are [n_pages][Hkv][page][D] and
+  // row r of sequence b lives in page block_table[b * max_blocks + r / page]
+  const int* block_table;
+  int max_blocks, page_log2, n_pages;
 };
 
 __device__ __forceinline__ int valid_klen(const int* k_lens, int b, int Lmax, int* status,
@@ -149,21 +153,62 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) decode_split_kernel(con
     *abort_flag = 0;
     sm100::fence_barrier_init();
   }
-  __syncthreads();
+  // paged cache: every block-table entry of this chunk is checked before any
+  // copy is issued; a chunk with a bad entry reads nothing and contributes an
+  // empty partial
+  const int* bt = p.block_table ? p.block_table + static_cast<size_t>(b) * p.max_blocks : nullptr;
+  bool bad_page = false;
+  if (bt) {
+    const int blk1 = (k0 + rows - 1) >> p.page_log2;
+    for (int bb = (k0 >> p.page_log2) + threadIdx.x; bb <= blk1; bb += NTHREADS) {
+      const int pg = __ldg(bt + bb);
+      if (pg < 0 || pg >= p.n_pages) bad_page = true;
+    }
+  }
+  if (__syncthreads_or(bad_page)) {
+    if (threadIdx.x == 0) atomicOr(p.status, ATTN_DEV_BAD_PAGE);
+    for (int e = threadIdx.x; e < p.G * D; e += NTHREADS) {
+      const size_t ph = (static_cast<size_t>(b) * p.Hq + hkv * p.G + e / D) * p.nsm + chunk;
+      p.part_o[ph * D + e % D] = 0.f;
+      if (e % D == 0) p.part_lse[ph] = -INFINITY;
+    }
+    return;
+  }
 
-  const size_t head_row0 = (static_cast<size_t>(b) * p.Hkv + hkv) * p.Lmax + k0;
   if (warp == NCW) {
     if (lane == 0) {
-      const uint8_t* gK = reinterpret_cast<const uint8_t*>(p.K) + head_row0 * ROWB;
-      const uint8_t* gV = reinterpret_cast<const uint8_t*>(p.V) + head_row0 * ROWB;
+      const uint8_t* gK = reinterpret_cast<const uint8_t*>(p.K);
+      const uint8_t* gV = reinterpret_cast<const uint8_t*>(p.V);
+      const size_t head_row0 = (static_cast<size_t>(b) * p.Hkv + hkv) * p.Lmax + k0;
+      const int page = 1 << p.page_log2;
       for (int s = 0; s < nstages; ++s) {
         const int slot = s % NST;
         if (!sm100::mbar_wait(&empty[slot], ((s / NST) & 1) ^ 1, abort_flag, p.status)) break;
         const int n = min(SR, rows - s * SR);
         const uint32_t bytes = static_cast<uint32_t>(n * ROWB);
         sm100::mbar_arrive_expect_tx(&full[slot], 2 * bytes);
-        bulk_g2s(sK + slot * STAGE, gK + static_cast<size_t>(s) * STAGE, bytes, &full[slot]);
-        bulk_g2s(sV + slot * STAGE, gV + static_cast<size_t>(s) * STAGE, bytes, &full[slot]);
+        if (!bt) {
+          const size_t off = (head_row0 + static_cast<size_t>(s) * SR) * ROWB;
+          bulk_g2s(sK + slot * STAGE, gK + off, bytes, &full[slot]);
+          bulk_g2s(sV + slot * STAGE, gV + off, bytes, &full[slot]);
+        } else {
+          // one copy per page segment of the stage's rows
+          int row = k0 + s * SR;
+          const int end = row + n;
+          uint32_t dst = static_cast<uint32_t>(slot * STAGE);
+          while (row < end) {
+            const int in_page = row & (page - 1);
+            const int seg = min(page - in_page, end - row);
+            const int pg = __ldg(bt + (row >> p.page_log2));
+            const size_t off =
+                ((static_cast<size_t>(pg) * p.Hkv + hkv) * page + in_page) * ROWB;
+            const uint32_t sb = static_cast<uint32_t>(seg * ROWB);
+            bulk_g2s(sK + dst, gK + off, sb, &full[slot]);
+            bulk_g2s(sV + dst, gV + off, sb, &full[slot]);
+            dst += sb;
+            row += seg;
+          }
+        }
       }
     }
     return;  // the producer takes no part in the merge below
@@ -394,11 +439,21 @@ cudaError_t launch_t(const SplitParams& sp, const CombineParams& cp, cudaStream_
   return cudaGetLastError();
 }
 
+// Paged cache description for launch(); Lmax is then max_blocks * page.
+struct PagedKV {
+  const int* block_table;  // device [B][max_blocks]
+  int max_blocks, page_log2, n_pages;
+};
+
 inline cudaError_t launch(const __nv_bfloat16* Q, const __nv_bfloat16* K, const __nv_bfloat16* V,
                           __nv_bfloat16* O, float* lse, int B, int Hq, int Hkv, int Lmax, int d,
                           float scale, const int* k_lens, int* status, uint8_t* scratch, int,
-                          cudaStream_t s) {
+                          cudaStream_t s, const PagedKV* paged = nullptr) {
   SplitParams sp;
+  sp.block_table = paged ? paged->block_table : nullptr;
+  sp.max_blocks = paged ? paged->max_blocks : 0;
+  sp.page_log2 = paged ? paged->page_log2 : 0;
+  sp.n_pages = paged ? paged->n_pages : 0;
   sp.Q = Q;
   sp.K = K;
   sp.V = V;

@@ -40,7 +40,8 @@
  * - Errors: argument errors are detected on the host before anything is
  *   launched and return ATTN_ERR_INVALID or ATTN_ERR_UNSUPPORTED.  A failed
  *   launch returns ATTN_ERR_CUDA.  Errors found on the device (a k_lens entry
- *   outside [0, Lk], an internal wait that timed out) set bits of a status
+ *   outside [0, Lk], a paged-cache block-table entry outside [0, n_pages), an
+ *   internal wait that timed out) set bits of a status
  *   word kept in the first 16 bytes of the workspace; the affected work units
  *   write zeros.  The word is sticky: read it with attn_read_device_status and
  *   clear it with attn_clear_device_status (a fresh workspace must be cleared
@@ -73,7 +74,7 @@ typedef enum {
 enum { ATTN_MASK_NONE = 0, ATTN_MASK_CAUSAL = 1 };
 
 /* Device status bits (first int32 of every workspace). */
-enum { ATTN_DEV_BAD_KLEN = 1, ATTN_DEV_TIMEOUT = 2 };
+enum { ATTN_DEV_BAD_KLEN = 1, ATTN_DEV_TIMEOUT = 2, ATTN_DEV_BAD_PAGE = 4 };
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* attn_status_string(attn_status_t s);
@@ -117,6 +118,32 @@ attn_status_t attn_fwd_splitkv_decode(const attn_bf16_t* Q, const attn_bf16_t* K
                                       int B, int Hq, int Hkv, int Lmax, int d, float scale,
                                       const int32_t* k_lens, void* workspace, size_t ws_bytes,
                                       void* stream);
+
+/* ------------------------------------------------------------------ paged decode
+ * The same split-KV decode over a paged cache: the KV-cache ledger of the
+ * three-ledgers page names paged attention as the decode-side companion of
+ * FlashAttention; what it computes is unchanged, only where row r of
+ * sequence b is read from.
+ *
+ *   Kpages/Vpages [n_pages, Hkv, page_size, d] bf16 (each head's rows of a
+ *   page are contiguous).  block_table device int32 [B, max_blocks]: row r of
+ *   sequence b is row r % page_size of page block_table[b, r / page_size].
+ *   Only the entries covering rows [0, k_lens[b]) are read; they must lie in
+ *   [0, n_pages).  k_lens device int32 [B], required, each in
+ *   [0, max_blocks * page_size].  page_size is a power of two in [16, 65536]
+ *   (else ATTN_ERR_UNSUPPORTED).  Q, O, lse, scale as attn_fwd_splitkv_decode.
+ *   The workspace is attn_decode_workspace_size(B, Hq, Hkv,
+ *   max_blocks * page_size, d) bytes.
+ *   A chunk whose block-table entries are out of range reads no page: it sets
+ *   ATTN_DEV_BAD_PAGE in the status word and contributes nothing to O.
+ */
+attn_status_t attn_fwd_splitkv_decode_paged(const attn_bf16_t* Q, const attn_bf16_t* Kpages,
+                                            const attn_bf16_t* Vpages,
+                                            const int32_t* block_table, int max_blocks,
+                                            int page_size, int n_pages, attn_bf16_t* O,
+                                            float* lse, int B, int Hq, int Hkv, int d,
+                                            float scale, const int32_t* k_lens,
+                                            void* workspace, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------ backward
  * Backward by recomputation: the three-ledgers page says the backward keeps only small row

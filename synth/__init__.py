@@ -95,7 +95,7 @@ def to_torch_bf16(bits: np.ndarray):
 
 # Workload seeds: 46 * 100 + workload number; each tensor draws its own stream.
 def workload_seed(workload: int, tensor: str) -> int:
-    tags = {"q": 1, "k": 2, "v": 3, "do": 4, "klen": 5}
+    tags = {"q": 1, "k": 2, "v": 3, "do": 4, "klen": 5, "pages": 6}
     return (4600 + workload) * 16 + tags[tensor]
 
 

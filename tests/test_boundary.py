@@ -96,6 +96,17 @@ def test_decode_and_bwd_reject_on_host(lib):
                         1 << 20, None) == 2
 
 
+def test_paged_decode_rejects_on_host(lib):
+    def call(bt=P, max_blocks=4, page=64, n_pages=8, d=128, ws_bytes=1 << 20, Hq=4):
+        return lib.attn_fwd_splitkv_decode_paged(P, P, P, bt, max_blocks, page, n_pages, P, None,
+                                                 1, Hq, 1, d, 0.1, P, P, ws_bytes, None)
+    assert call(bt=None) == 1
+    assert call(n_pages=0) == 1 and call(max_blocks=0) == 1
+    assert call(page=24) == 2 and call(page=8) == 2 and call(page=1 << 17) == 2
+    assert call(ws_bytes=64) == 1
+    assert call(d=96) == 2 and call(Hq=3) == 2
+
+
 def test_product_path_does_not_touch_oracle():
     """The CUDA binding must neither import nor load anything from oracle/."""
     pkg = os.path.join(ROOT, "exact_io_aware_46_b200")
