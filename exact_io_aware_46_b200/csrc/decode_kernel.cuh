@@ -28,14 +28,17 @@
 namespace attn_decode_impl {
 
 // Measured on B200 (B64 Hq32 Hkv8 d128, cache 32768, k_len ~ U[1024, 32768]):
-// chunk 1024 / 3 stages / 2 CTAs per SM 5.56 TB/s; 2 stages / 3 CTAs per SM
-// 5.98 TB/s; chunk 2048 with 2 stages / 3 CTAs per SM 6.11 TB/s (shipped);
-// chunk 4096 5.88 TB/s, chunk 512 5.01 TB/s.  More resident warps hide the
-// shared-memory and shuffle latency of the compute warps; longer chunks
-// amortise a CTA's start (query load, first copy) and its final merge.
+// chunk 1024 / 3 stages of 64 rows / 2 CTAs per SM 5.56 TB/s; 2 stages / 3
+// CTAs per SM 5.98 TB/s; chunk 2048, 2 x 64-row stages, 3 CTAs per SM 6.08-6.11
+// TB/s; chunk 2048, 4 x 32-row stages, 3 CTAs per SM 6.23 TB/s (shipped);
+// chunk 4096 5.88 TB/s, chunk 512 5.01 TB/s; 4 CTAs per SM (96 registers,
+// spills) 5.53-5.64 TB/s.  More resident warps hide the shared-memory and
+// shuffle latency of the compute warps, finer stages release ring space
+// sooner, and longer chunks amortise a CTA's start (query load, first copy)
+// and its final merge.
 constexpr int CH = 2048;  // keys per split
-constexpr int SR = 64;    // key rows per shared-memory stage
-constexpr int NST = 2;    // stages
+constexpr int SR = 32;    // key rows per shared-memory stage
+constexpr int NST = 4;    // stages
 constexpr int CTAS_PER_SM = 3;
 constexpr int NCW = 4;    // compute warps
 constexpr int NTHREADS = (NCW + 1) * 32;
