@@ -8,6 +8,7 @@ library is missing, every call raises.
 The functions carry the C entry points' names:
 
 * ``attn_fwd(Q, K, V, ...) -> (O, LSE)``
+* ``attn_fwd_varlen(Q, K, V, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, ...) -> (O, LSE)``
 * ``attn_fwd_splitkv_decode(Q, Kcache, Vcache, k_lens, ...) -> (O, LSE)``
 * ``attn_fwd_splitkv_decode_paged(Q, Kpages, Vpages, block_table, k_lens, ...) -> (O, LSE)``
 * ``attn_bwd(Q, K, V, O, dO, LSE, ...) -> (dQ, dK, dV)``
@@ -48,6 +49,9 @@ SIGNATURES = {
     "attn_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _vp, _sz,
                       _vp]),
+    "attn_fwd_varlen_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "attn_fwd_varlen": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
+                             _f, _i, _vp, _sz, _vp]),
     "attn_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "attn_fwd_splitkv_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _vp,
                                      _sz, _vp]),
@@ -128,6 +132,10 @@ def attn_fwd_workspace_size(B, Hq, Hkv, Lq, Lk, d) -> int:
     return int(lib().attn_fwd_workspace_size(B, Hq, Hkv, Lq, Lk, d))
 
 
+def attn_fwd_varlen_workspace_size(B, Hq, Hkv, max_seqlen_q, max_seqlen_k, d) -> int:
+    return int(lib().attn_fwd_varlen_workspace_size(B, Hq, Hkv, max_seqlen_q, max_seqlen_k, d))
+
+
 def attn_decode_workspace_size(B, Hq, Hkv, Lmax, d) -> int:
     return int(lib().attn_decode_workspace_size(B, Hq, Hkv, Lmax, d))
 
@@ -169,6 +177,36 @@ def attn_fwd(Q, K, V, scale=None, causal=False, k_lens=None, O=None, lse=None, w
                           float(scale), ATTN_MASK_CAUSAL if causal else ATTN_MASK_NONE,
                           _ptr(k_lens), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(code, "attn_fwd")
+    return O, lse
+
+
+def attn_fwd_varlen(Q, K, V, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                    scale=None, causal=False, O=None, lse=None, workspace=None, stream=None,
+                    want_lse=True):
+    """Forward over packed sequences.  Q [total_q,Hq,d], K/V [total_k,Hkv,d] bf16;
+    cu_seqlens_q / cu_seqlens_k int32 [B+1] on the device.  LSE is [Hq, total_q]."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _bf16(t, n)
+    total_q, Hq, d = Q.shape
+    total_k, Hkv = K.shape[0], K.shape[1]
+    B = cu_seqlens_q.numel() - 1
+    if cu_seqlens_k.numel() != B + 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must have the same length")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if O is None:
+        O = torch.empty_like(Q)
+    if lse is None and want_lse:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=Q.device)
+    if workspace is None:
+        workspace = _workspace(attn_fwd_varlen_workspace_size(B, Hq, Hkv, max_seqlen_q,
+                                                              max_seqlen_k, d), Q.device, stream)
+    code = lib().attn_fwd_varlen(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
+                                 _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B, Hq, Hkv,
+                                 int(max_seqlen_q), int(max_seqlen_k), total_q, total_k, d,
+                                 float(scale), ATTN_MASK_CAUSAL if causal else ATTN_MASK_NONE,
+                                 _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(code, "attn_fwd_varlen")
     return O, lse
 
 

@@ -53,6 +53,24 @@ bool make_tmap(CUtensorMap* m, const void* base, int d, int L, long long heads, 
   return r == CUDA_SUCCESS;
 }
 
+// 3-D bf16 view of a packed [T, H, d] tensor as [rows = T][heads = H][d] with the
+// kernels' coordinate order (column, row, head): dimension 1 steps over tokens
+// (stride H * d), dimension 2 over heads (stride d).
+bool make_tmap_packed(CUtensorMap* m, const void* base, int d, int T, int heads, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T > 0 ? T : 1),
+                        static_cast<cuuint64_t>(heads)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2 * static_cast<cuuint64_t>(heads),
+                           static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int device_sms() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -81,6 +99,44 @@ cudaError_t set_smem(K kernel, int bytes) {
 bool attn_bwd_impl::make_tmap_rows(CUtensorMap* m, const void* base, int L, long long heads,
                                    int box_rows) {
   return make_tmap(m, base, attn_bwd_impl::D, L, heads, box_rows);
+}
+
+// Shared launch of the forward kernel; p carries the layout-specific fields.
+static attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         attn_fwd_impl::Params p, attn_bf16_t* O, float* lse, int B, int Hq,
+                         int Hkv, int d, float scale, int mask_flags, void* workspace,
+                         void* stream) {
+  const int sms = device_sms();
+  if (sms <= 0) return ATTN_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int n_pairs = (p.Lq + 2 * attn_fwd_impl::BM - 1) / (2 * attn_fwd_impl::BM);
+  const int n_items = B * Hq * n_pairs;
+  p.O = reinterpret_cast<__nv_bfloat16*>(O);
+  p.lse = lse;
+  p.status = reinterpret_cast<int*>(workspace);
+  p.sched = reinterpret_cast<int*>(workspace) + 1;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = (mask_flags & ATTN_MASK_CAUSAL) ? 1 : 0;
+  p.n_pairs = n_pairs;
+  p.n_items = n_items;
+  const int grid = n_items < sms ? n_items : sms;
+  cudaError_t e;
+  if (d == 128) {
+    constexpr int smem = attn_fwd_impl::Cfg<128>::SMEM_BYTES;
+    e = set_smem(attn_fwd_impl::fwd_kernel<128>, smem);
+    if (e == cudaSuccess)
+      attn_fwd_impl::fwd_kernel<128><<<grid, attn_fwd_impl::NTHREADS, smem, s>>>(tq, tk, tv, p);
+  } else {
+    constexpr int smem = attn_fwd_impl::Cfg<64>::SMEM_BYTES;
+    e = set_smem(attn_fwd_impl::fwd_kernel<64>, smem);
+    if (e == cudaSuccess)
+      attn_fwd_impl::fwd_kernel<64><<<grid, attn_fwd_impl::NTHREADS, smem, s>>>(tq, tk, tv, p);
+  }
+  if (e != cudaSuccess) return ATTN_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 extern "C" {
@@ -118,48 +174,54 @@ attn_status_t attn_fwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (Lq == 0) return ATTN_OK;
 
-  const int sms = device_sms();
-  if (sms <= 0) return ATTN_ERR_CUDA;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int n_pairs = (Lq + 2 * attn_fwd_impl::BM - 1) / (2 * attn_fwd_impl::BM);
-  const int n_items = B * Hq * n_pairs;
-  cudaError_t e;
-  {
-    CUtensorMap tq, tk, tv;
-    if (!make_tmap(&tq, Q, d, Lq, static_cast<long long>(B) * Hq, 128) ||
-        !make_tmap(&tk, K, d, Lk, static_cast<long long>(B) * Hkv, 128) ||
-        !make_tmap(&tv, V, d, Lk, static_cast<long long>(B) * Hkv, 128))
-      return ATTN_ERR_CUDA;
-    attn_fwd_impl::Params p;
-    p.O = reinterpret_cast<__nv_bfloat16*>(O);
-    p.lse = lse;
-    p.k_lens = k_lens;
-    p.status = reinterpret_cast<int*>(workspace);
-    p.sched = reinterpret_cast<int*>(workspace) + 1;
-    p.B = B;
-    p.Hq = Hq;
-    p.Hkv = Hkv;
-    p.Lq = Lq;
-    p.Lk = Lk;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    p.causal = (mask_flags & ATTN_MASK_CAUSAL) ? 1 : 0;
-    p.n_pairs = n_pairs;
-    p.n_items = n_items;
-    const int grid = n_items < sms ? n_items : sms;
-    if (d == 128) {
-      constexpr int smem = attn_fwd_impl::Cfg<128>::SMEM_BYTES;
-      e = set_smem(attn_fwd_impl::fwd_kernel<128>, smem);
-      if (e == cudaSuccess)
-        attn_fwd_impl::fwd_kernel<128><<<grid, attn_fwd_impl::NTHREADS, smem, s>>>(tq, tk, tv, p);
-    } else {
-      constexpr int smem = attn_fwd_impl::Cfg<64>::SMEM_BYTES;
-      e = set_smem(attn_fwd_impl::fwd_kernel<64>, smem);
-      if (e == cudaSuccess)
-        attn_fwd_impl::fwd_kernel<64><<<grid, attn_fwd_impl::NTHREADS, smem, s>>>(tq, tk, tv, p);
-    }
-  }
-  if (e != cudaSuccess) return ATTN_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, Q, d, Lq, static_cast<long long>(B) * Hq, 128) ||
+      !make_tmap(&tk, K, d, Lk, static_cast<long long>(B) * Hkv, 128) ||
+      !make_tmap(&tv, V, d, Lk, static_cast<long long>(B) * Hkv, 128))
+    return ATTN_ERR_CUDA;
+  attn_fwd_impl::Params p{};
+  p.k_lens = k_lens;
+  p.Lq = Lq;
+  p.Lk = Lk;
+  return launch_fwd(tq, tk, tv, p, O, lse, B, Hq, Hkv, d, scale, mask_flags, workspace, stream);
+}
+
+size_t attn_fwd_varlen_workspace_size(int, int, int, int, int, int) { return kStatusBytes; }
+
+attn_status_t attn_fwd_varlen(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf16_t* V,
+                              attn_bf16_t* O, float* lse, const int32_t* cu_seqlens_q,
+                              const int32_t* cu_seqlens_k, int B, int Hq, int Hkv,
+                              int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                              int d, float scale, int mask_flags, void* workspace,
+                              size_t ws_bytes, void* stream) {
+  if (!shapes_ok(B, Hq, Hkv, max_seqlen_q, max_seqlen_k)) return ATTN_ERR_INVALID;
+  if (total_q < 0 || total_k < 0 || total_q > (1 << 30) || total_k > (1 << 30))
+    return ATTN_ERR_INVALID;
+  if (!Q || !K || !V || !O || !cu_seqlens_q || !cu_seqlens_k || !workspace)
+    return ATTN_ERR_INVALID;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) ||
+      (lse && !aligned16(lse)) || !aligned16(cu_seqlens_q) || !aligned16(cu_seqlens_k) ||
+      !aligned256(workspace))
+    return ATTN_ERR_INVALID;
+  if (!(std::isfinite(scale) && scale > 0.f)) return ATTN_ERR_INVALID;
+  if (mask_flags != ATTN_MASK_NONE && mask_flags != ATTN_MASK_CAUSAL) return ATTN_ERR_INVALID;
+  if (ws_bytes < attn_fwd_varlen_workspace_size(B, Hq, Hkv, max_seqlen_q, max_seqlen_k, d))
+    return ATTN_ERR_INVALID;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (max_seqlen_q == 0 || total_q == 0) return ATTN_OK;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_packed(&tq, Q, d, total_q, Hq, 128) ||
+      !make_tmap_packed(&tk, K, d, total_k, Hkv, 128) ||
+      !make_tmap_packed(&tv, V, d, total_k, Hkv, 128))
+    return ATTN_ERR_CUDA;
+  attn_fwd_impl::Params p{};
+  p.Lq = max_seqlen_q;
+  p.Lk = max_seqlen_k;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  return launch_fwd(tq, tk, tv, p, O, lse, B, Hq, Hkv, d, scale, mask_flags, workspace, stream);
 }
 
 // ------------------------------------------------------------------ decode

@@ -74,13 +74,26 @@ struct Params {
   int B, Hq, Hkv, Lq, Lk;
   float scale_log2;  // scale * log2(e)
   int causal;
-  int n_pairs;  // ceil(Lq / 256)
+  int n_pairs;  // ceil(Lq / 256) (ceil(max_seqlen_q / 256) for packed sequences)
   int n_items;  // B * Hq * n_pairs
+  // packed (variable-length) sequences: Q/O [total_q, Hq, D], K/V [total_k, Hkv, D],
+  // sequence b = rows [cu_q[b], cu_q[b+1]) and [cu_k[b], cu_k[b+1]); lse [Hq, total_q].
+  // nullptr for the batched layout.
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
 };
 
 struct Item {
   int b, h, row0;  // row0: first query row of tile 0; tile 1 starts at row0 + BM
-  int kv_len;
+  int lq;          // query rows of this sequence
+  int koff;        // Lk - Lq of this sequence (bottom-right causal alignment)
+  int kv_len;      // visible keys
+  int q_coord, k_coord;  // tensor-map row coordinate of the sequence's row 0
+  int q_head, kv_head;   // tensor-map head coordinates
+  size_t o_off;          // element offset of (row 0, head h) in O
+  size_t o_rstride;      // elements between consecutive rows of O
+  size_t lse_off;        // offset of row 0 in lse
   int n0, n1;  // key/value tiles each query tile visits
   int nmax;
 };
@@ -88,11 +101,11 @@ struct Item {
 constexpr int HEAD_GROUP = 8;  // heads whose items are interleaved (L2 reuse of their K/V)
 constexpr int NI = 4;          // depth of the shared-memory item ring
 
-__device__ __forceinline__ int tiles_for(const Params& p, int row0, int kv_len) {
-  if (row0 >= p.Lq) return 0;
-  const int last = min(row0 + BM - 1, p.Lq - 1);
-  int hi = kv_len;
-  if (p.causal) hi = min(hi, last + (p.Lk - p.Lq) + 1);
+__device__ __forceinline__ int tiles_for(const Params& p, const Item& it, int row0) {
+  if (row0 >= it.lq) return 0;
+  const int last = min(row0 + BM - 1, it.lq - 1);
+  int hi = it.kv_len;
+  if (p.causal) hi = min(hi, last + it.koff + 1);
   return hi <= 0 ? 0 : (hi + BN - 1) / BN;
 }
 
@@ -100,6 +113,7 @@ __device__ __forceinline__ int tiles_for(const Params& p, int row0, int kv_len) 
 // latest query rows (heaviest under a causal mask) first, heads interleaved.
 // Grouping keeps the concurrently streamed K/V within a few heads (L2-resident)
 // while dynamic fetching keeps the heaviest-first property for load balance.
+template <int D_OF_O>
 __device__ __forceinline__ Item get_item(const Params& p, int w, bool* bad) {
   Item it;
   const int BH = p.B * p.Hq;
@@ -112,17 +126,47 @@ __device__ __forceinline__ Item get_item(const Params& p, int w, bool* bad) {
   it.b = bh / p.Hq;
   it.h = bh % p.Hq;
   it.row0 = pair * 2 * BM;
-  int kl = p.Lk;
-  if (p.k_lens) {
-    kl = __ldg(p.k_lens + it.b);
-    if (kl < 0 || kl > p.Lk) {
-      if (bad) *bad = true;
-      kl = 0;
+  const int kvh = it.h / (p.Hq / p.Hkv);
+  if (!p.cu_q) {
+    int kl = p.Lk;
+    if (p.k_lens) {
+      kl = __ldg(p.k_lens + it.b);
+      if (kl < 0 || kl > p.Lk) {
+        if (bad) *bad = true;
+        kl = 0;
+      }
     }
+    it.lq = p.Lq;
+    it.koff = p.Lk - p.Lq;
+    it.kv_len = kl;
+    it.q_coord = 0;
+    it.k_coord = 0;
+    it.q_head = it.b * p.Hq + it.h;
+    it.kv_head = it.b * p.Hkv + kvh;
+    it.o_off = static_cast<size_t>(it.q_head) * p.Lq * D_OF_O;
+    it.o_rstride = D_OF_O;
+    it.lse_off = static_cast<size_t>(it.q_head) * p.Lq;
+  } else {
+    const int q0 = __ldg(p.cu_q + it.b), q1 = __ldg(p.cu_q + it.b + 1);
+    const int k0 = __ldg(p.cu_k + it.b), k1 = __ldg(p.cu_k + it.b + 1);
+    // a malformed sequence (offsets decreasing, past the totals, or longer than
+    // the stated maximum) is reported and skipped: nothing is read or written
+    const bool ok = 0 <= q0 && q0 <= q1 && q1 <= p.total_q && q1 - q0 <= p.Lq && 0 <= k0 &&
+                    k0 <= k1 && k1 <= p.total_k && k1 - k0 <= p.Lk;
+    if (!ok && bad) *bad = true;
+    it.lq = ok ? q1 - q0 : 0;
+    it.kv_len = ok ? k1 - k0 : 0;
+    it.koff = it.kv_len - it.lq;
+    it.q_coord = ok ? q0 : 0;
+    it.k_coord = ok ? k0 : 0;
+    it.q_head = it.h;
+    it.kv_head = kvh;
+    it.o_off = (static_cast<size_t>(it.q_coord) * p.Hq + it.h) * D_OF_O;
+    it.o_rstride = static_cast<size_t>(p.Hq) * D_OF_O;
+    it.lse_off = static_cast<size_t>(it.h) * p.total_q + it.q_coord;
   }
-  it.kv_len = kl;
-  it.n0 = tiles_for(p, it.row0, kl);
-  it.n1 = tiles_for(p, it.row0 + BM, kl);
+  it.n0 = tiles_for(p, it, it.row0);
+  it.n1 = tiles_for(p, it, it.row0 + BM);
   it.nmax = max(it.n0, it.n1);
   return it;
 }
@@ -248,16 +292,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         *reinterpret_cast<volatile int*>(&item_ring[k % NI]) = w;
         sm100::mbar_arrive(&item_full[k % NI]);
         if (w < 0) break;
-        const Item it = get_item(p, w, nullptr);
+        const Item it = get_item<D>(p, w, nullptr);
         if (!sm100::mbar_wait(q_empty, (k & 1) ^ 1, abort_flag, p.status)) break;
         sm100::mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
-        const int qh = it.b * p.Hq + it.h;
+        const int qh = it.q_head;
         for (int t = 0; t < 2; ++t)
           for (int c = 0; c < C::CHUNKS; ++c)
             sm100::tma_load_3d(&tmQ, q_full,
                                smem + C::OFF_Q + t * C::TILE_BYTES + c * CHUNK_BYTES, c * 64,
-                               it.row0 + t * BM, qh);
-        const int kvh = it.b * p.Hkv + it.h / (p.Hq / p.Hkv);
+                               it.q_coord + it.row0 + t * BM, qh);
+        const int kvh = it.kv_head;
         bool ok = true;
         for (int j = 0; j < it.nmax && ok; ++j) {
           for (int kv = 0; kv < 2; ++kv, ++use) {
@@ -271,7 +315,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int c = 0; c < C::CHUNKS; ++c)
               sm100::tma_load_3d(kv == 0 ? &tmK : &tmV, &kv_full[slot],
                                  smem + C::OFF_KV + slot * C::TILE_BYTES + c * CHUNK_BYTES,
-                                 c * 64, j * BN, kvh);
+                                 c * 64, it.k_coord + j * BN, kvh);
           }
         }
         if (!ok) break;
@@ -317,7 +361,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
         if (leader) sm100::mbar_arrive(&item_empty[k % NI]);
         if (w < 0) break;
-        const Item it = get_item(p, w, nullptr);
+        const Item it = get_item<D>(p, w, nullptr);
         if (!(ok = sm100::mbar_wait(q_full, k & 1, abort_flag, p.status))) break;
         sm100::tc_fence_after();
         const uint32_t oe_par = (k & 1) ^ 1;
@@ -414,12 +458,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int w;
       if (!(ok = next_item(k, w)) || w < 0) break;
       bool bad = false;
-      const Item it = get_item(p, w, &bad);
+      const Item it = get_item<D>(p, w, &bad);
       if (bad && threadIdx.x == 0) atomicOr(p.status, 1);
       const int n_t = t ? it.n1 : it.n0;
       const int row0 = it.row0 + t * BM;
       const int row = row0 + r;
-      const int diag = row + (p.Lk - p.Lq);  // last visible key under the causal mask
+      const int diag = row + it.koff;  // last visible key under the causal mask
       float m_use = -INFINITY, l = 0.f;
       for (int j = 0; j < n_t; ++j) {
         if (!(ok = sm100::mbar_wait(&s_full[t], s_cnt & 1, abort_flag, p.status))) break;
@@ -433,7 +477,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
         const int k0 = j * BN + 64 * hf;
         const bool need_mask =
-            (k0 + 64 > it.kv_len) || (p.causal && (k0 + 63 > row0 + (p.Lk - p.Lq)));
+            (k0 + 64 > it.kv_len) || (p.causal && (k0 + 63 > row0 + it.koff));
         if (need_mask) {
           const int lim = p.causal ? min(it.kv_len - 1, diag) : it.kv_len - 1;
 #pragma unroll
@@ -511,10 +555,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         sm100::named_bar_sync(bar_id, 64);
         l += lx[(hf ^ 1) * BM + r];
       }
-      const bool live = row < p.Lq;
+      const bool live = row < it.lq;
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       __nv_bfloat16* orow =
-          p.O + ((static_cast<size_t>(it.b) * p.Hq + it.h) * p.Lq + (live ? row : 0)) * D + DH * hf;
+          p.O + it.o_off + (live ? row : 0) * it.o_rstride + DH * hf;
       if (n_t > 0) {
 #pragma unroll 1
         for (int c = 0; c < DH / 32; ++c) {
@@ -538,7 +582,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int v = 0; v < DH / 8; ++v) dst[v] = make_uint4(0, 0, 0, 0);
       }
       if (live && p.lse && hf == 0)
-        p.lse[(static_cast<size_t>(it.b) * p.Hq + it.h) * p.Lq + row] =
+        p.lse[it.lse_off + row] =
             (l > 0.f) ? (m_use + log2f(l)) * 0.69314718055994531f : -INFINITY;
       sm100::tc_fence_before();
       __syncwarp();

@@ -97,6 +97,31 @@ attn_status_t attn_fwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf
                        int d, float scale, int mask_flags, const int32_t* k_lens,
                        void* workspace, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------ packed forward
+ * The forward over variable-length sequences packed back to back (no padding):
+ * the same attention per sequence as attn_fwd, with the batch given by
+ * offsets instead of a common length.  The pages name varlen batching as the
+ * prefill-side partner of the KV-cache ledger; the layout and the offset
+ * convention are ours.
+ *
+ *   Q, O [total_q, Hq, d] bf16; K, V [total_k, Hkv, d] bf16.  cu_seqlens_q and
+ *   cu_seqlens_k: device int32 [B + 1], non-decreasing, starting at 0; sequence
+ *   b is rows [cu_q[b], cu_q[b+1]) of Q and [cu_k[b], cu_k[b+1]) of K and V,
+ *   at most max_seqlen_q / max_seqlen_k rows long and inside total_q / total_k.
+ *   lse [Hq, total_q] fp32 (may be NULL).  mask_flags as attn_fwd (the causal
+ *   mask is aligned to each sequence's bottom-right corner); no k_lens (the
+ *   offsets give each sequence's keys).  A sequence whose offsets break these
+ *   rules is skipped (nothing read or written) and sets ATTN_DEV_BAD_KLEN.
+ */
+size_t attn_fwd_varlen_workspace_size(int B, int Hq, int Hkv, int max_seqlen_q,
+                                      int max_seqlen_k, int d);
+attn_status_t attn_fwd_varlen(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf16_t* V,
+                              attn_bf16_t* O, float* lse, const int32_t* cu_seqlens_q,
+                              const int32_t* cu_seqlens_k, int B, int Hq, int Hkv,
+                              int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                              int d, float scale, int mask_flags, void* workspace,
+                              size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------ decode
  * Split-KV decode (one query token per sequence over a contiguous KV cache):
  * the "short query scans a long history" case of the three-ledgers page

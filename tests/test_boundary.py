@@ -107,6 +107,16 @@ def test_paged_decode_rejects_on_host(lib):
     assert call(d=96) == 2 and call(Hq=3) == 2
 
 
+def test_varlen_fwd_rejects_on_host(lib):
+    def call(cu=P, B=2, Hq=4, Hkv=2, mq=64, mk=64, tq=100, tk=100, d=128, mask=1, ws_bytes=256):
+        return lib.attn_fwd_varlen(P, P, P, P, None, cu, cu, B, Hq, Hkv, mq, mk, tq, tk, d, 0.1,
+                                   mask, P, ws_bytes, None)
+    assert call(cu=None) == 1 and call(Hq=3) == 1 and call(tq=-1) == 1 and call(mask=5) == 1
+    assert call(ws_bytes=16) == 1 and call(B=0) == 1
+    assert call(d=80) == 2
+    assert call(mq=0) == 0 and call(tq=0) == 0  # nothing to compute: returns at once
+
+
 def test_product_path_does_not_touch_oracle():
     """The CUDA binding must neither import nor load anything from oracle/."""
     pkg = os.path.join(ROOT, "exact_io_aware_46_b200")
