@@ -271,7 +271,43 @@ def fwd_leg(steps, warmup, world, flush):
     ms_e2e = timed_loop(e2e_call, max(3, steps // 2), 2, stream, flush)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = hO.numel() * hO.element_size() + hL.numel() * hL.element_size()
-    return ms, ms_e2e, h2d, d2h
+    del q, k, v, O, lse, hq, hk, hv, hO, hL
+    torch.cuda.empty_cache()
+    return ms, ms_e2e, h2d, d2h, varlen_leg(steps, warmup, world, flush)
+
+
+VARLEN = dict(n_seq=16, lo=256, hi=4096, H=16, d=128)
+
+
+def varlen_leg(steps, warmup, world, flush):
+    """Packed causal prefill: 16 sequences with seeded lengths ~ U[256, 4096] back to
+    back, Hq = Hkv = 16, d = 128.  FLOPs count each sequence's visible pairs."""
+    import torch
+
+    import exact_io_aware_46_b200 as attn
+
+    c = VARLEN
+    dev = torch.device("cuda")
+    lens = synth.uniform_int(synth.workload_seed(6, "klen"), c["n_seq"], c["lo"], c["hi"])
+    total = int(np.sum(lens.astype(np.int64)))
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=dev)
+    q = synth.normal_bf16_device(synth.workload_seed(6, "q"), (total, c["H"], c["d"]), dev)
+    k = synth.normal_bf16_device(synth.workload_seed(6, "k"), (total, c["H"], c["d"]), dev)
+    v = synth.normal_bf16_device(synth.workload_seed(6, "v"), (total, c["H"], c["d"]), dev)
+    O = torch.empty_like(q)
+    lse = torch.empty((c["H"], total), dtype=torch.float32, device=dev)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    mx = int(lens.max())
+    call = lambda: attn.attn_fwd_varlen(q, k, v, cu, cu, mx, mx, causal=True, O=O, lse=lse,
+                                        workspace=ws, stream=stream)
+    barrier(world)
+    ms = timed_loop(call, steps, warmup, stream, flush)
+    st = attn.attn_read_device_status(ws)
+    if st[0] != attn.ATTN_OK:
+        raise RuntimeError(f"device status {st}")
+    flops = sum(4.0 * c["d"] * causal_pairs(int(L), int(L), True) * c["H"] for L in lens)
+    return ms, flops, total
 
 
 def decode_leg(steps, warmup, world, flush):
@@ -468,7 +504,8 @@ def main():
     DEC["Lmax"] = args.decode_lmax
     with Clocks(gpu_idx) as clk:
         if "fwd" in legs:
-            ms, ms_e2e, h2d, d2h = fwd_leg(args.steps, args.warmup, world, flush)
+            ms, ms_e2e, h2d, d2h, (vms, vflops, vtotal) = fwd_leg(args.steps, args.warmup,
+                                                                  world, flush)
         if "decode" in legs:
             dms, kv_bytes, _, (page, pms) = decode_leg(args.steps, args.warmup, world, flush)
         if "bwd" in legs:
@@ -494,7 +531,8 @@ def main():
     t_e2e = max_over_ranks(float(np.mean(ms_e2e)), world)
     value = world * flops / (t_step * 1e-3) / 1e12
     achieved = flops / (float(np.mean(ms)) * 1e-3) / 1e12
-    launches = args.steps  # one persistent forward kernel per step
+    # one persistent forward kernel per step: timed forward, e2e and packed-prefill loops
+    launches = args.steps + max(3, args.steps // 2) + args.steps
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -517,6 +555,14 @@ def main():
                 "ms_per_step": t_e2e},
         "gpu_launches": launches,
         "clocks": clocks,
+    }
+    t_v = max_over_ranks(float(np.mean(vms)), world)
+    line["varlen"] = {
+        "workload": f"packed causal prefill: {VARLEN['n_seq']} sequences with lengths "
+                    f"~U[{VARLEN['lo']},{VARLEN['hi']}] back to back ({vtotal} tokens), "
+                    f"Hq=Hkv={VARLEN['H']}, d={VARLEN['d']}",
+        "value": world * vflops / (t_v * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": t_v,
+        "flops_per_step": vflops,
     }
     if "decode" in legs:
         t_d = max_over_ranks(float(np.mean(dms)), world)
