@@ -13,6 +13,11 @@ Parity status of each function (what pins it, see ``tests/test_oracle_pins.py``)
   FlashAttention-2 tutorial (2.1.9), row sums, constant V, key permutation,
   causal row 0, closed forms (one key, Q = 0), the fully masked row, and an
   independent library witness (torch fp64 softmax) on small shapes.
+* the sliding-window mask (``window`` > 0 with ``causal``) -- pinned: a window
+  wider than the sequence equals the causal mask (forward exactly, backward to
+  rounding), W = 1 closed forms (O_i = V_{i+off}, LSE_i = scale q_i.k_{i+off},
+  dQ = dK = 0, dV = the routed dO), W = 2 as a two-term softmax, and brute force
+  over each row's visible key set.
 * ``bwd`` / ``bwd_sampled`` -- pinned: central finite differences of the
   forward's loss on tiny shapes, gradient invariants (columns of dS sum to
   zero, sum_j dV_j = sum_i dO_i), grouped-query equality to the sum of
@@ -61,18 +66,16 @@ def _load():
             lib = ctypes.CDLL(build())
             lib.oracle_set_threads.argtypes = [ctypes.c_int]
             lib.oracle_get_threads.restype = ctypes.c_int
-            lib.oracle_fwd_head.argtypes = [_dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                            ctypes.c_double, ctypes.c_int, ctypes.c_int, _ip,
-                                            ctypes.c_int, _dp, _dp]
-            lib.oracle_probs_head.argtypes = [_dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                              ctypes.c_double, ctypes.c_int, ctypes.c_int, _dp, _dp]
-            lib.oracle_bwd_head.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
-                                            ctypes.c_int, ctypes.c_double, ctypes.c_int,
-                                            ctypes.c_int, _dp, _dp, _dp]
-            lib.oracle_bwd_head_sampled.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
-                                                    ctypes.c_int, ctypes.c_double, ctypes.c_int,
-                                                    ctypes.c_int, _ip, ctypes.c_int, _ip,
-                                                    ctypes.c_int, _dp, _dp, _dp]
+            _c = ctypes.c_int
+            lib.oracle_fwd_head.argtypes = [_dp, _dp, _dp, _c, _c, _c, ctypes.c_double, _c, _c, _c,
+                                            _ip, _c, _dp, _dp]
+            lib.oracle_probs_head.argtypes = [_dp, _dp, _c, _c, _c, ctypes.c_double, _c, _c, _c,
+                                              _dp, _dp]
+            lib.oracle_bwd_head.argtypes = [_dp, _dp, _dp, _dp, _c, _c, _c, ctypes.c_double, _c, _c,
+                                            _c, _dp, _dp, _dp]
+            lib.oracle_bwd_head_sampled.argtypes = [_dp, _dp, _dp, _dp, _c, _c, _c,
+                                                    ctypes.c_double, _c, _c, _c, _ip, _c, _ip, _c,
+                                                    _dp, _dp, _dp]
             lib.oracle_online_row.argtypes = [_dp, _dp, ctypes.c_int, ctypes.c_int, _ip, ctypes.c_int,
                                               _dp, _dp, _dp, _dp, _dp]
             lib.oracle_merge.argtypes = [ctypes.c_double, ctypes.c_double, _dp, ctypes.c_double,
@@ -112,8 +115,17 @@ def _kv_len(k_lens, b, Lk):
     return int(Lk if k_lens is None else k_lens[b])
 
 
-def fwd(Q, K, V, scale: float, causal: bool = False, k_lens=None, rows=None, heads=None):
+def _window(causal, window):
+    w = int(window or 0)
+    if w > 0 and not causal:
+        raise ValueError("a sliding window needs the causal mask")
+    return w
+
+
+def fwd(Q, K, V, scale: float, causal: bool = False, k_lens=None, rows=None, heads=None,
+        window: int = 0):
     """Forward of every (b, h) head, or of the listed ``heads`` [(b, h), ...].
+    ``window`` > 0 (with ``causal``): each query row sees only its ``window`` latest keys.
 
     Q [B,Hq,Lq,d]; K, V [B,Hkv,Lk,d] (fp64 or bf16 bits); query head h reads
     key/value head h // (Hq // Hkv).  ``rows`` restricts the query rows.
@@ -136,13 +148,14 @@ def fwd(Q, K, V, scale: float, causal: bool = False, k_lens=None, rows=None, hea
         o = np.zeros((R, d))
         lse = np.zeros(R)
         lib.oracle_fwd_head(_p(q), _p(k), _p(v), Lq, Lk, d, float(scale), int(bool(causal)),
-                            _kv_len(k_lens, b, Lk), _pi(rows_a), R, _p(o), _p(lse))
+                            _window(causal, window), _kv_len(k_lens, b, Lk), _pi(rows_a), R,
+                            _p(o), _p(lse))
         O[b, h] = o
         L[b, h] = lse
     return O, L
 
 
-def probs(Q, K, scale: float, causal: bool = False, kv_len=None):
+def probs(Q, K, scale: float, causal: bool = False, kv_len=None, window: int = 0):
     """Full probability matrix P [Lq,Lk] and LSE [Lq] of one head (Q [Lq,d], K [Lk,d])."""
     lib = _load()
     q = _f64(Q)
@@ -152,11 +165,12 @@ def probs(Q, K, scale: float, causal: bool = False, kv_len=None):
     P = np.zeros((Lq, Lk))
     lse = np.zeros(Lq)
     lib.oracle_probs_head(_p(q), _p(k), Lq, Lk, d, float(scale), int(bool(causal)),
-                          int(Lk if kv_len is None else kv_len), _p(P), _p(lse))
+                          _window(causal, window), int(Lk if kv_len is None else kv_len), _p(P),
+                          _p(lse))
     return P, lse
 
 
-def bwd(Q, K, V, dO, scale: float, causal: bool = False, k_lens=None):
+def bwd(Q, K, V, dO, scale: float, causal: bool = False, k_lens=None, window: int = 0):
     """Full backward: returns (dQ [B,Hq,Lq,d], dK [B,Hkv,Lk,d], dV [B,Hkv,Lk,d]) in fp64.
 
     Grouped query heads accumulate into their shared key/value head."""
@@ -178,15 +192,16 @@ def bwd(Q, K, V, dO, scale: float, causal: bool = False, k_lens=None):
                 g = _f64(dO[b, h])
                 dq = np.zeros((Lq, d))
                 lib.oracle_bwd_head(_p(q), _p(k), _p(v), _p(g), Lq, Lk, d, float(scale),
-                                    int(bool(causal)), _kv_len(k_lens, b, Lk), _p(dq), _p(dk),
-                                    _p(dv))
+                                    int(bool(causal)), _window(causal, window),
+                                    _kv_len(k_lens, b, Lk), _p(dq), _p(dk), _p(dv))
                 dQ[b, h] = dq
             dK[b, hk] = dk
             dV[b, hk] = dv
     return dQ, dK, dV
 
 
-def bwd_sampled(Q, K, V, dO, scale: float, causal: bool, k_lens, b: int, hk: int, qrows, kcols):
+def bwd_sampled(Q, K, V, dO, scale: float, causal: bool, k_lens, b: int, hk: int, qrows, kcols,
+                window: int = 0):
     """Backward of key/value head (b, hk) at sampled outputs.
 
     Returns (dQ [G,nq,d] for the G query heads of hk at rows ``qrows``,
@@ -207,8 +222,9 @@ def bwd_sampled(Q, K, V, dO, scale: float, causal: bool, k_lens, b: int, hk: int
         g = _f64(dO[b, h])
         dq = np.zeros((len(qa), d))
         lib.oracle_bwd_head_sampled(_p(q), _p(k), _p(v), _p(g), Lq, Lk, d, float(scale),
-                                    int(bool(causal)), _kv_len(k_lens, b, Lk), _pi(qa), len(qa),
-                                    _pi(ka), len(ka), _p(dq), _p(dKs), _p(dVs))
+                                    int(bool(causal)), _window(causal, window),
+                                    _kv_len(k_lens, b, Lk), _pi(qa), len(qa), _pi(ka), len(ka),
+                                    _p(dq), _p(dKs), _p(dVs))
         dQs[gi] = dq
     return dQs, dKs, dVs
 

@@ -20,6 +20,10 @@
  *     causal : key j is visible to query i iff j <= i + (Lk - Lq)
  *              (bottom-right alignment; ordinary lower triangle when Lq == Lk)
  *     padding: key j is visible iff j < kv_len (per-sequence key length)
+ *     sliding window (with causal, window W > 0): additionally
+ *              j > i + (Lk - Lq) - W, i.e. each query sees its W latest keys
+ *              (the local causal mask of the pages' mask discussion; W <= 0
+ *              means no window)
  *     a row with no visible key has O = 0 and LSE = -inf.
  *
  *   LSE_i = m_i + ln(sum_j exp(S_ij - m_i)) over visible j: the per-row
@@ -59,22 +63,23 @@ int oracle_get_threads(void) {
 #endif
 }
 
-static int is_visible(int i, int j, int Lq, int Lk, int causal, int kv_len) {
+static int is_visible(int i, int j, int Lq, int Lk, int causal, int window, int kv_len) {
   if (j >= kv_len) return 0;
   if (causal && j > i + (Lk - Lq)) return 0;
+  if (causal && window > 0 && j <= i + (Lk - Lq) - window) return 0;
   return 1;
 }
 
 /* One query row i of one head: fills s[0..Lk) (scaled, -inf where masked) and
  * p[0..Lk) (softmax), returns the number of visible keys; *lse receives LSE_i. */
 static int row_probs(const double* Qh, const double* Kh, int i, int Lq, int Lk, int d,
-                     double scale, int causal, int kv_len, double* s, double* p,
+                     double scale, int causal, int window, int kv_len, double* s, double* p,
                      double* lse) {
   const double* q = Qh + (size_t)i * d;
   double m = -INFINITY;
   int nvis = 0;
   for (int j = 0; j < Lk; ++j) {
-    if (!is_visible(i, j, Lq, Lk, causal, kv_len)) {
+    if (!is_visible(i, j, Lq, Lk, causal, window, kv_len)) {
       s[j] = -INFINITY;
       continue;
     }
@@ -104,7 +109,7 @@ static int row_probs(const double* Qh, const double* Kh, int i, int Lq, int Lk, 
  * rows: the query rows to compute (NULL = all Lq rows, then n_rows = Lq).
  * O_rows [n_rows,d], lse_rows [n_rows]. */
 void oracle_fwd_head(const double* Qh, const double* Kh, const double* Vh, int Lq, int Lk,
-                     int d, double scale, int causal, int kv_len, const int* rows,
+                     int d, double scale, int causal, int window, int kv_len, const int* rows,
                      int n_rows, double* O_rows, double* lse_rows) {
   if (rows == NULL) n_rows = Lq;
 #pragma omp parallel num_threads(oracle_get_threads())
@@ -115,7 +120,7 @@ void oracle_fwd_head(const double* Qh, const double* Kh, const double* Vh, int L
     for (int r = 0; r < n_rows; ++r) {
       int i = rows ? rows[r] : r;
       double lse;
-      row_probs(Qh, Kh, i, Lq, Lk, d, scale, causal, kv_len, s, p, &lse);
+      row_probs(Qh, Kh, i, Lq, Lk, d, scale, causal, window, kv_len, s, p, &lse);
       double* o = O_rows + (size_t)r * d;
       for (int c = 0; c < d; ++c) o[c] = 0.0;
       for (int j = 0; j < Lk; ++j) {
@@ -132,17 +137,17 @@ void oracle_fwd_head(const double* Qh, const double* Kh, const double* Vh, int L
 
 /* Full probability matrix of one head, P [Lq,Lk] (for row-sum and tiny-case pins). */
 void oracle_probs_head(const double* Qh, const double* Kh, int Lq, int Lk, int d, double scale,
-                       int causal, int kv_len, double* P, double* lse) {
+                       int causal, int window, int kv_len, double* P, double* lse) {
   double* s = (double*)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
   for (int i = 0; i < Lq; ++i)
-    row_probs(Qh, Kh, i, Lq, Lk, d, scale, causal, kv_len, s, P + (size_t)i * Lk, lse + i);
+    row_probs(Qh, Kh, i, Lq, Lk, d, scale, causal, window, kv_len, s, P + (size_t)i * Lk, lse + i);
   free(s);
 }
 
 /* Backward for one (b, h) head, all rows.  dQh [Lq,d] is overwritten; dKh and
  * dVh [Lk,d] are ACCUMULATED into (+=) so grouped query heads sum naturally. */
 void oracle_bwd_head(const double* Qh, const double* Kh, const double* Vh, const double* dOh,
-                     int Lq, int Lk, int d, double scale, int causal, int kv_len,
+                     int Lq, int Lk, int d, double scale, int causal, int window, int kv_len,
                      double* dQh, double* dKh, double* dVh) {
   int nt = oracle_get_threads();
   double* dK_part = (double*)calloc((size_t)nt * Lk * d + 1, sizeof(double));
@@ -165,7 +170,7 @@ void oracle_bwd_head(const double* Qh, const double* Kh, const double* Vh, const
       const double* g = dOh + (size_t)i * d;
       double* dq = dQh + (size_t)i * d;
       for (int c = 0; c < d; ++c) dq[c] = 0.0;
-      if (row_probs(Qh, Kh, i, Lq, Lk, d, scale, causal, kv_len, s, p, &lse) == 0) continue;
+      if (row_probs(Qh, Kh, i, Lq, Lk, d, scale, causal, window, kv_len, s, p, &lse) == 0) continue;
       /* dP_ij = dO_i . V_j ; D_i = sum_j P_ij dP_ij */
       double D = 0.0;
       for (int j = 0; j < Lk; ++j) {
@@ -211,6 +216,7 @@ void oracle_bwd_head(const double* Qh, const double* Kh, const double* Vh, const
  * definition requires); only the outputs are restricted. */
 void oracle_bwd_head_sampled(const double* Qh, const double* Kh, const double* Vh,
                              const double* dOh, int Lq, int Lk, int d, double scale, int causal,
+                             int window,
                              int kv_len, const int* qrows, int nq, const int* kcols, int nk,
                              double* dQ_rows, double* dK_cols, double* dV_cols) {
   double* lse = (double*)malloc(sizeof(double) * (size_t)(Lq > 0 ? Lq : 1));
@@ -223,7 +229,7 @@ void oracle_bwd_head_sampled(const double* Qh, const double* Kh, const double* V
     double* p = (double*)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
 #pragma omp for schedule(dynamic, 8)
     for (int i = 0; i < Lq; ++i) {
-      has[i] = row_probs(Qh, Kh, i, Lq, Lk, d, scale, causal, kv_len, s, p, &lse[i]) > 0;
+      has[i] = row_probs(Qh, Kh, i, Lq, Lk, d, scale, causal, window, kv_len, s, p, &lse[i]) > 0;
       double acc_D = 0.0;
       const double* g = dOh + (size_t)i * d;
       for (int j = 0; j < Lk; ++j) {
@@ -248,7 +254,7 @@ void oracle_bwd_head_sampled(const double* Qh, const double* Kh, const double* V
     for (int c = 0; c < d; ++c) dq[c] = 0.0;
     if (!has[i]) continue;
     for (int j = 0; j < Lk; ++j) {
-      if (!is_visible(i, j, Lq, Lk, causal, kv_len)) continue;
+      if (!is_visible(i, j, Lq, Lk, causal, window, kv_len)) continue;
       const double* k = Kh + (size_t)j * d;
       const double* v = Vh + (size_t)j * d;
       double sc = 0.0, dp = 0.0;
@@ -267,7 +273,7 @@ void oracle_bwd_head_sampled(const double* Qh, const double* Kh, const double* V
     double* dk = dK_cols + (size_t)r * d;
     double* dv = dV_cols + (size_t)r * d;
     for (int i = 0; i < Lq; ++i) {
-      if (!has[i] || !is_visible(i, j, Lq, Lk, causal, kv_len)) continue;
+      if (!has[i] || !is_visible(i, j, Lq, Lk, causal, window, kv_len)) continue;
       const double* q = Qh + (size_t)i * d;
       const double* g = dOh + (size_t)i * d;
       double sc = 0.0, dp = 0.0;

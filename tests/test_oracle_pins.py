@@ -406,3 +406,73 @@ def test_torch_fp64_autograd_witness_backward(causal):
     assert np.max(np.abs(dQ - q.grad.numpy())) <= 1e-12
     assert np.max(np.abs(dK - k.grad.numpy())) <= 1e-12
     assert np.max(np.abs(dV - v.grad.numpy())) <= 1e-12
+
+
+# ---------------------------------------------------------------- sliding window
+
+
+@pytest.mark.parametrize("Lq,Lk", [(12, 12), (7, 12)])
+def test_window_wider_than_the_sequence_is_causal(Lq, Lk):
+    Q, K, V, dO = (_rand(900 + i, s) for i, s in enumerate(
+        [(1, 2, Lq, 16), (1, 1, Lk, 16), (1, 1, Lk, 16), (1, 2, Lq, 16)]))
+    O1, L1 = oracle.fwd(Q, K, V, 0.3, causal=True)
+    O2, L2 = oracle.fwd(Q, K, V, 0.3, causal=True, window=Lk + 1)
+    assert np.array_equal(O1, O2) and np.array_equal(L1, L2)
+    g1 = oracle.bwd(Q, K, V, dO, 0.3, causal=True)
+    g2 = oracle.bwd(Q, K, V, dO, 0.3, causal=True, window=Lk + 1)
+    for a, b in zip(g1, g2):  # dK, dV sum over threads in any order: equal to rounding
+        assert np.allclose(a, b, rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("Lq,Lk", [(9, 9), (6, 10)])
+def test_window_one_sees_only_the_diagonal_key(Lq, Lk):
+    """W = 1: each row's softmax has one term, so O_i = V_{i+off} and
+    LSE_i = scale * q_i . k_{i+off}; then P is one-hot, dS = P (dP - D) = 0, so
+    dQ = dK = 0 and dV_j gathers dO of the row that sees key j."""
+    off = Lk - Lq
+    Q, K, V, dO = (_rand(920 + i, s) for i, s in enumerate(
+        [(1, 1, Lq, 8), (1, 1, Lk, 8), (1, 1, Lk, 8), (1, 1, Lq, 8)]))
+    O, L = oracle.fwd(Q, K, V, 0.25, causal=True, window=1)
+    for i in range(Lq):
+        j = i + off
+        assert np.allclose(O[0, 0, i], V[0, 0, j], rtol=0, atol=1e-15)
+        assert math.isclose(L[0, 0, i], 0.25 * float(Q[0, 0, i] @ K[0, 0, j]), rel_tol=1e-13)
+    dQ, dK, dV = oracle.bwd(Q, K, V, dO, 0.25, causal=True, window=1)
+    assert np.allclose(dQ, 0.0, atol=1e-13) and np.allclose(dK, 0.0, atol=1e-13)
+    want = np.zeros_like(dV)
+    for i in range(Lq):
+        want[0, 0, i + off] = dO[0, 0, i]
+    assert np.allclose(dV, want, rtol=0, atol=1e-13)
+
+
+def test_window_two_is_a_two_term_softmax():
+    Lq = Lk = 10
+    Q, K, V = (_rand(940 + i, (1, 1, Lq, 8)) for i in range(3))
+    O, _ = oracle.fwd(Q, K, V, 0.5, causal=True, window=2)
+    for i in range(1, Lq):
+        a = 0.5 * float(Q[0, 0, i] @ K[0, 0, i - 1])
+        b = 0.5 * float(Q[0, 0, i] @ K[0, 0, i])
+        wa, wb = 1.0 / (1.0 + math.exp(b - a)), 1.0 / (1.0 + math.exp(a - b))
+        assert np.allclose(O[0, 0, i], wa * V[0, 0, i - 1] + wb * V[0, 0, i], rtol=1e-12,
+                           atol=1e-14)
+    assert np.allclose(O[0, 0, 0], V[0, 0, 0], rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("W", [1, 3, 5])
+def test_window_visible_set_per_row(W):
+    """Brute force on the probability matrix: row i has exactly the keys
+    (i + off - W, i + off] that exist, each with positive probability."""
+    Lq, Lk = 7, 11
+    off = Lk - Lq
+    Q, K = _rand(960, (Lq, 8)), _rand(961, (Lk, 8))
+    P, _ = oracle.probs(Q, K, 0.4, causal=True, window=W)
+    for i in range(Lq):
+        want = {j for j in range(Lk) if i + off - W < j <= i + off}
+        assert {j for j in range(Lk) if P[i, j] > 0} == want
+        assert math.isclose(P[i].sum(), 1.0, rel_tol=1e-13)
+
+
+def test_window_requires_causal():
+    with pytest.raises(ValueError):
+        oracle.fwd(_rand(1, (1, 1, 4, 8)), _rand(2, (1, 1, 4, 8)), _rand(3, (1, 1, 4, 8)), 1.0,
+                   causal=False, window=2)
