@@ -271,9 +271,21 @@ def fwd_leg(steps, warmup, world, flush):
     ms_e2e = timed_loop(e2e_call, max(3, steps // 2), 2, stream, flush)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = hO.numel() * hO.element_size() + hL.numel() * hL.element_size()
+    # the same workload with a sliding window of 1024 keys (key tiles outside skipped)
+    W = WINDOW
+    call_w = lambda: attn.attn_fwd_sliding(q, k, v, W, O=O, lse=lse, workspace=ws, stream=stream)
+    barrier(world)
+    wms = timed_loop(call_w, steps, warmup, stream, flush)
+    st = attn.attn_read_device_status(ws)
+    if st[0] != attn.ATTN_OK:
+        raise RuntimeError(f"device status {st}")
+    wflops = 4.0 * c["d"] * c["B"] * c["Hq"] * sum(min(i + 1, W) for i in range(c["L"]))
     del q, k, v, O, lse, hq, hk, hv, hO, hL
     torch.cuda.empty_cache()
-    return ms, ms_e2e, h2d, d2h, varlen_leg(steps, warmup, world, flush)
+    return ms, ms_e2e, h2d, d2h, varlen_leg(steps, warmup, world, flush), (W, wms, wflops)
+
+
+WINDOW = 1024
 
 
 VARLEN = dict(n_seq=16, lo=256, hi=4096, H=16, d=128)
@@ -504,8 +516,8 @@ def main():
     DEC["Lmax"] = args.decode_lmax
     with Clocks(gpu_idx) as clk:
         if "fwd" in legs:
-            ms, ms_e2e, h2d, d2h, (vms, vflops, vtotal) = fwd_leg(args.steps, args.warmup,
-                                                                  world, flush)
+            (ms, ms_e2e, h2d, d2h, (vms, vflops, vtotal),
+             (W, wms, wflops)) = fwd_leg(args.steps, args.warmup, world, flush)
         if "decode" in legs:
             dms, kv_bytes, _, (page, pms) = decode_leg(args.steps, args.warmup, world, flush)
         if "bwd" in legs:
@@ -532,7 +544,7 @@ def main():
     value = world * flops / (t_step * 1e-3) / 1e12
     achieved = flops / (float(np.mean(ms)) * 1e-3) / 1e12
     # one persistent forward kernel per step: timed forward, e2e and packed-prefill loops
-    launches = args.steps + max(3, args.steps // 2) + args.steps
+    launches = args.steps + max(3, args.steps // 2) + args.steps + args.steps
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -563,6 +575,13 @@ def main():
                     f"Hq=Hkv={VARLEN['H']}, d={VARLEN['d']}",
         "value": world * vflops / (t_v * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": t_v,
         "flops_per_step": vflops,
+    }
+    t_w = max_over_ranks(float(np.mean(wms)), world)
+    line["sliding_window"] = {
+        "workload": f"the causal prefill forward B4 H16 L4096 d128 with a sliding window of {W} "
+                    f"keys (FLOPs over visible pairs)",
+        "value": world * wflops / (t_w * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": t_w,
+        "flops_per_step": wflops,
     }
     if "decode" in legs:
         t_d = max_over_ranks(float(np.mean(dms)), world)

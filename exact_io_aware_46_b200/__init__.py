@@ -12,6 +12,7 @@ The functions carry the C entry points' names:
 * ``attn_fwd_splitkv_decode(Q, Kcache, Vcache, k_lens, ...) -> (O, LSE)``
 * ``attn_fwd_splitkv_decode_paged(Q, Kpages, Vpages, block_table, k_lens, ...) -> (O, LSE)``
 * ``attn_bwd(Q, K, V, O, dO, LSE, ...) -> (dQ, dK, dV)``
+* ``attn_fwd_sliding`` / ``attn_bwd_sliding``: the same with a sliding-window causal mask
 * the ``*_workspace_size`` queries and the device-status helpers.
 """
 
@@ -49,6 +50,10 @@ SIGNATURES = {
     "attn_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _vp, _sz,
                       _vp]),
+    "attn_fwd_sliding": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _vp,
+                              _sz, _vp]),
+    "attn_bwd_sliding": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                              _f, _i, _vp, _vp, _sz, _vp]),
     "attn_fwd_varlen_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "attn_fwd_varlen": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
                              _f, _i, _vp, _sz, _vp]),
@@ -178,6 +183,50 @@ def attn_fwd(Q, K, V, scale=None, causal=False, k_lens=None, O=None, lse=None, w
                           _ptr(k_lens), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(code, "attn_fwd")
     return O, lse
+
+
+def attn_fwd_sliding(Q, K, V, window, scale=None, k_lens=None, O=None, lse=None, workspace=None,
+                     stream=None, want_lse=True):
+    """Sliding-window causal forward: row i sees its ``window`` latest keys."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _bf16(t, n)
+    B, Hq, Lq, d = Q.shape
+    Hkv, Lk = K.shape[1], K.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if O is None:
+        O = torch.empty_like(Q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=Q.device)
+    if workspace is None:
+        workspace = _workspace(attn_fwd_workspace_size(B, Hq, Hkv, Lq, Lk, d), Q.device, stream)
+    code = lib().attn_fwd_sliding(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse), B, Hq, Hkv, Lq,
+                                  Lk, d, float(scale), int(window), _ptr(k_lens), _ptr(workspace),
+                                  workspace.numel(), _stream(stream))
+    _check(code, "attn_fwd_sliding")
+    return O, lse
+
+
+def attn_bwd_sliding(Q, K, V, O, dO, lse, window, scale=None, k_lens=None, dQ=None, dK=None,
+                     dV=None, workspace=None, stream=None):
+    """Backward of attn_fwd_sliding.  Returns (dQ, dK, dV) bf16."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V"), (O, "O"), (dO, "dO")):
+        _bf16(t, n)
+    B, Hq, Lq, d = Q.shape
+    Hkv, Lk = K.shape[1], K.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dQ = torch.empty_like(Q) if dQ is None else dQ
+    dK = torch.empty_like(K) if dK is None else dK
+    dV = torch.empty_like(V) if dV is None else dV
+    if workspace is None:
+        workspace = _workspace(attn_bwd_workspace_size(B, Hq, Hkv, Lq, Lk, d), Q.device, stream)
+    code = lib().attn_bwd_sliding(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(lse),
+                                  _ptr(dQ), _ptr(dK), _ptr(dV), B, Hq, Hkv, Lq, Lk, d,
+                                  float(scale), int(window), _ptr(k_lens), _ptr(workspace),
+                                  workspace.numel(), _stream(stream))
+    _check(code, "attn_bwd_sliding")
+    return dQ, dK, dV
 
 
 def attn_fwd_varlen(Q, K, V, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,

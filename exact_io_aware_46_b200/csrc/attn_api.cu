@@ -123,17 +123,24 @@ static attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, co
   p.n_pairs = n_pairs;
   p.n_items = n_items;
   const int grid = n_items < sms ? n_items : sms;
-  cudaError_t e;
+  const int mode = p.cu_q ? attn_fwd_impl::MODE_VARLEN
+                          : (p.window > 0 ? attn_fwd_impl::MODE_WINDOW : attn_fwd_impl::MODE_PLAIN);
+  cudaError_t e = cudaSuccess;
+  auto run = [&](auto kernel, int smem) {
+    e = set_smem(kernel, smem);
+    if (e == cudaSuccess) kernel<<<grid, attn_fwd_impl::NTHREADS, smem, s>>>(tq, tk, tv, p);
+  };
+  using namespace attn_fwd_impl;
   if (d == 128) {
-    constexpr int smem = attn_fwd_impl::Cfg<128>::SMEM_BYTES;
-    e = set_smem(attn_fwd_impl::fwd_kernel<128>, smem);
-    if (e == cudaSuccess)
-      attn_fwd_impl::fwd_kernel<128><<<grid, attn_fwd_impl::NTHREADS, smem, s>>>(tq, tk, tv, p);
+    constexpr int smem = Cfg<128>::SMEM_BYTES;
+    if (mode == MODE_PLAIN) run(fwd_kernel<128, MODE_PLAIN>, smem);
+    else if (mode == MODE_WINDOW) run(fwd_kernel<128, MODE_WINDOW>, smem);
+    else run(fwd_kernel<128, MODE_VARLEN>, smem);
   } else {
-    constexpr int smem = attn_fwd_impl::Cfg<64>::SMEM_BYTES;
-    e = set_smem(attn_fwd_impl::fwd_kernel<64>, smem);
-    if (e == cudaSuccess)
-      attn_fwd_impl::fwd_kernel<64><<<grid, attn_fwd_impl::NTHREADS, smem, s>>>(tq, tk, tv, p);
+    constexpr int smem = Cfg<64>::SMEM_BYTES;
+    if (mode == MODE_PLAIN) run(fwd_kernel<64, MODE_PLAIN>, smem);
+    else if (mode == MODE_WINDOW) run(fwd_kernel<64, MODE_WINDOW>, smem);
+    else run(fwd_kernel<64, MODE_VARLEN>, smem);
   }
   if (e != cudaSuccess) return ATTN_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -159,10 +166,11 @@ int attn_num_sms(void) { return device_sms(); }
 
 size_t attn_fwd_workspace_size(int, int, int, int, int, int) { return kStatusBytes; }
 
-attn_status_t attn_fwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf16_t* V,
-                       attn_bf16_t* O, float* lse, int B, int Hq, int Hkv, int Lq, int Lk, int d,
-                       float scale, int mask_flags, const int32_t* k_lens, void* workspace,
-                       size_t ws_bytes, void* stream) {
+static attn_status_t fwd_batched(const attn_bf16_t* Q, const attn_bf16_t* K,
+                                 const attn_bf16_t* V, attn_bf16_t* O, float* lse, int B, int Hq,
+                                 int Hkv, int Lq, int Lk, int d, float scale, int mask_flags,
+                                 int window, const int32_t* k_lens, void* workspace,
+                                 size_t ws_bytes, void* stream) {
   if (!shapes_ok(B, Hq, Hkv, Lq, Lk)) return ATTN_ERR_INVALID;
   if (!Q || !K || !V || !O || !workspace) return ATTN_ERR_INVALID;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) ||
@@ -183,7 +191,25 @@ attn_status_t attn_fwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf
   p.k_lens = k_lens;
   p.Lq = Lq;
   p.Lk = Lk;
+  p.window = window;
   return launch_fwd(tq, tk, tv, p, O, lse, B, Hq, Hkv, d, scale, mask_flags, workspace, stream);
+}
+
+attn_status_t attn_fwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf16_t* V,
+                       attn_bf16_t* O, float* lse, int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                       float scale, int mask_flags, const int32_t* k_lens, void* workspace,
+                       size_t ws_bytes, void* stream) {
+  return fwd_batched(Q, K, V, O, lse, B, Hq, Hkv, Lq, Lk, d, scale, mask_flags, 0, k_lens,
+                     workspace, ws_bytes, stream);
+}
+
+attn_status_t attn_fwd_sliding(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf16_t* V,
+                               attn_bf16_t* O, float* lse, int B, int Hq, int Hkv, int Lq, int Lk,
+                               int d, float scale, int window, const int32_t* k_lens,
+                               void* workspace, size_t ws_bytes, void* stream) {
+  if (window < 1) return ATTN_ERR_INVALID;
+  return fwd_batched(Q, K, V, O, lse, B, Hq, Hkv, Lq, Lk, d, scale, ATTN_MASK_CAUSAL, window,
+                     k_lens, workspace, ws_bytes, stream);
 }
 
 size_t attn_fwd_varlen_workspace_size(int, int, int, int, int, int) { return kStatusBytes; }
@@ -296,11 +322,13 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d) {
   return kStatusBytes + attn_bwd_impl::scratch_bytes(B, Hq, Hkv, Lq, Lk, d);
 }
 
-attn_status_t attn_bwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf16_t* V,
-                       const attn_bf16_t* O, const attn_bf16_t* dO, const float* lse,
-                       attn_bf16_t* dQ, attn_bf16_t* dK, attn_bf16_t* dV, int B, int Hq, int Hkv,
-                       int Lq, int Lk, int d, float scale, int mask_flags, const int32_t* k_lens,
-                       void* workspace, size_t ws_bytes, void* stream) {
+static attn_status_t bwd_batched(const attn_bf16_t* Q, const attn_bf16_t* K,
+                                 const attn_bf16_t* V, const attn_bf16_t* O,
+                                 const attn_bf16_t* dO, const float* lse, attn_bf16_t* dQ,
+                                 attn_bf16_t* dK, attn_bf16_t* dV, int B, int Hq, int Hkv, int Lq,
+                                 int Lk, int d, float scale, int mask_flags, int window,
+                                 const int32_t* k_lens, void* workspace, size_t ws_bytes,
+                                 void* stream) {
   if (!shapes_ok(B, Hq, Hkv, Lq, Lk)) return ATTN_ERR_INVALID;
   if (!Q || !K || !V || !O || !dO || !lse || !dQ || !dK || !dV || !workspace)
     return ATTN_ERR_INVALID;
@@ -334,11 +362,32 @@ attn_status_t attn_bwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf
   a.d = d;
   a.scale = scale;
   a.causal = (mask_flags & ATTN_MASK_CAUSAL) ? 1 : 0;
+  a.window = window;
   a.k_lens = k_lens;
   a.status = reinterpret_cast<int*>(workspace);
   a.scratch = reinterpret_cast<uint8_t*>(workspace) + kStatusBytes;
   a.sms = sms;
   return attn_bwd_impl::launch(a, s);
+}
+
+attn_status_t attn_bwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf16_t* V,
+                       const attn_bf16_t* O, const attn_bf16_t* dO, const float* lse,
+                       attn_bf16_t* dQ, attn_bf16_t* dK, attn_bf16_t* dV, int B, int Hq, int Hkv,
+                       int Lq, int Lk, int d, float scale, int mask_flags, const int32_t* k_lens,
+                       void* workspace, size_t ws_bytes, void* stream) {
+  return bwd_batched(Q, K, V, O, dO, lse, dQ, dK, dV, B, Hq, Hkv, Lq, Lk, d, scale, mask_flags, 0,
+                     k_lens, workspace, ws_bytes, stream);
+}
+
+attn_status_t attn_bwd_sliding(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf16_t* V,
+                               const attn_bf16_t* O, const attn_bf16_t* dO, const float* lse,
+                               attn_bf16_t* dQ, attn_bf16_t* dK, attn_bf16_t* dV, int B, int Hq,
+                               int Hkv, int Lq, int Lk, int d, float scale, int window,
+                               const int32_t* k_lens, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  if (window < 1) return ATTN_ERR_INVALID;
+  return bwd_batched(Q, K, V, O, dO, lse, dQ, dK, dV, B, Hq, Hkv, Lq, Lk, d, scale,
+                     ATTN_MASK_CAUSAL, window, k_lens, workspace, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------------ status

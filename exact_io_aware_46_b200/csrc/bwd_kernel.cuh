@@ -68,6 +68,7 @@ struct Args {
   int B, Hq, Hkv, Lq, Lk, d;
   float scale;
   int causal;
+  int window;  // > 0: sliding window (with causal)
   const int* k_lens;
   int* status;
   uint8_t* scratch;
@@ -93,6 +94,7 @@ struct Params {
   int B, Hq, Hkv, G, Lq, Lk, Lqp;
   float scale, scale_log2;
   int causal;
+  int window;  // > 0: a query row sees only its `window` latest keys
   int n_kv;     // ceil(Lk / 128)
   int n_qt;     // Lqp / 64
   int n_items;  // B * Hkv * n_kv
@@ -138,8 +140,14 @@ __device__ __forceinline__ Item get_item(const Params& p, int w, bool* bad) {
   if (p.causal) r_min = max(0, k0 - (p.Lk - p.Lq));  // first row that sees key k0
   if (r_min >= p.Lq) return it;
   it.i_lo = r_min / BMQ;
-  const int nq = (p.Lq + BMQ - 1) / BMQ;
-  it.T = p.G * (nq - it.i_lo);
+  int i_end = (p.Lq + BMQ - 1) / BMQ;  // one past the last query tile
+  if (p.window > 0) {
+    // the last row that sees a key of this tile: i + off - W < k0 + BN - 1
+    const int r_max = k0 + BN - 2 - (p.Lk - p.Lq) + p.window;
+    if (r_max < r_min) return it;
+    i_end = min(i_end, r_max / BMQ + 1);
+  }
+  it.T = p.G * (i_end - it.i_lo);
   return it;
 }
 
@@ -479,12 +487,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         sm100::tmem_ld32(tmem + lane_base + S_COL0 + b * 64 + 32,
                          *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
         sm100::tmem_ld_wait();
-        // key visible to query row r0 + c iff key <= lim_key and c >= cmin
+        // key visible to query row r0 + c iff key <= lim_key, c >= cmin and
+        // (sliding window) c <= cmax
         const int r0 = i * BMQ;
         const bool key_ok = key <= lim;
         const int cmin = p.causal ? key - r0 - off : -1;
+        const int cmax = p.window > 0 ? key - off + p.window - 1 - r0 : BMQ;
         // whole tile visible: no per-element test (warp-uniform; usual case)
-        const bool all_vis = __all_sync(0xffffffffu, key_ok && cmin <= 0);
+        const bool all_vis = __all_sync(0xffffffffu, key_ok && cmin <= 0 && cmax >= BMQ - 1);
         const float4* l2v = reinterpret_cast<const float4*>(l2s);
         const float2 sl2x2 = make_float2(p.scale_log2, p.scale_log2);
         float pr[64];
@@ -505,7 +515,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!all_vis) {
 #pragma unroll
           for (int c = 0; c < 64; ++c)
-            if (!key_ok || c < cmin) pr[c] = 0.f;
+            if (!key_ok || c < cmin || c > cmax) pr[c] = 0.f;
         }
         uint32_t pk[32];
 #pragma unroll
@@ -653,6 +663,7 @@ inline attn_status_t launch(const Args& a, cudaStream_t s) {
   p.scale = a.scale;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.causal = a.causal;
+  p.window = a.window;
   p.k_lens = a.k_lens;
   p.status = a.status;
   const size_t rows = static_cast<size_t>(a.B) * a.Hq * p.Lqp;

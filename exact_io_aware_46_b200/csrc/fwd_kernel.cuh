@@ -31,6 +31,8 @@
 //    becomes rare.
 #pragma once
 
+#include <climits>
+
 #include "sm100.cuh"
 
 namespace attn_fwd_impl {
@@ -82,6 +84,7 @@ struct Params {
   const int* cu_q;
   const int* cu_k;
   int total_q, total_k;
+  int window;  // > 0: sliding window (with causal): a row sees its `window` latest keys
 };
 
 struct Item {
@@ -94,9 +97,19 @@ struct Item {
   size_t o_off;          // element offset of (row 0, head h) in O
   size_t o_rstride;      // elements between consecutive rows of O
   size_t lse_off;        // offset of row 0 in lse
-  int n0, n1;  // key/value tiles each query tile visits
-  int nmax;
+  int n0, n1;    // one past the last key/value tile each query tile visits
+  int lo0, lo1;  // first key/value tile each query tile visits (0 without a window)
+  int jb, nmax;  // the item's key/value tiles: [jb, nmax)
 };
+
+// Kernel variants, fixed at compile time so that the plain batched forward
+// carries none of the others' per-item state (measured: a single kernel with
+// runtime switches ran the plain workload 7 % slower -- register spills in the
+// MMA-issuing warp):
+//   MODE_PLAIN   [B, H, L, d] tensors, optional causal mask and key padding;
+//   MODE_WINDOW  the same with a sliding-window causal mask (p.window keys);
+//   MODE_VARLEN  packed sequences [T, H, d] with cu_seqlens offsets.
+enum : int { MODE_PLAIN = 0, MODE_WINDOW = 1, MODE_VARLEN = 2 };
 
 constexpr int HEAD_GROUP = 8;  // heads whose items are interleaved (L2 reuse of their K/V)
 constexpr int NI = 4;          // depth of the shared-memory item ring
@@ -113,7 +126,7 @@ __device__ __forceinline__ int tiles_for(const Params& p, const Item& it, int ro
 // latest query rows (heaviest under a causal mask) first, heads interleaved.
 // Grouping keeps the concurrently streamed K/V within a few heads (L2-resident)
 // while dynamic fetching keeps the heaviest-first property for load balance.
-template <int D_OF_O>
+template <int D_OF_O, int MODE>
 __device__ __forceinline__ Item get_item(const Params& p, int w, bool* bad) {
   Item it;
   const int BH = p.B * p.Hq;
@@ -127,7 +140,7 @@ __device__ __forceinline__ Item get_item(const Params& p, int w, bool* bad) {
   it.h = bh % p.Hq;
   it.row0 = pair * 2 * BM;
   const int kvh = it.h / (p.Hq / p.Hkv);
-  if (!p.cu_q) {
+  if constexpr (MODE != MODE_VARLEN) {
     int kl = p.Lk;
     if (p.k_lens) {
       kl = __ldg(p.k_lens + it.b);
@@ -143,9 +156,9 @@ __device__ __forceinline__ Item get_item(const Params& p, int w, bool* bad) {
     it.k_coord = 0;
     it.q_head = it.b * p.Hq + it.h;
     it.kv_head = it.b * p.Hkv + kvh;
-    it.o_off = static_cast<size_t>(it.q_head) * p.Lq * D_OF_O;
+    it.o_off = 0;  // the epilogue addresses [B, H, L, d] directly in this layout
     it.o_rstride = D_OF_O;
-    it.lse_off = static_cast<size_t>(it.q_head) * p.Lq;
+    it.lse_off = 0;
   } else {
     const int q0 = __ldg(p.cu_q + it.b), q1 = __ldg(p.cu_q + it.b + 1);
     const int k0 = __ldg(p.cu_k + it.b), k1 = __ldg(p.cu_k + it.b + 1);
@@ -167,7 +180,17 @@ __device__ __forceinline__ Item get_item(const Params& p, int w, bool* bad) {
   }
   it.n0 = tiles_for(p, it, it.row0);
   it.n1 = tiles_for(p, it, it.row0 + BM);
+  // sliding window: key tiles entirely below the first row's window are skipped
+  it.lo0 = it.lo1 = 0;
+  if constexpr (MODE == MODE_WINDOW) {
+    const int f0 = it.row0 + it.koff - p.window + 1, f1 = f0 + BM;
+    it.lo0 = f0 > 0 ? f0 / BN : 0;
+    it.lo1 = f1 > 0 ? f1 / BN : 0;
+    if (it.lo0 >= it.n0) it.n0 = it.lo0 = 0;  // no row of the tile sees a key
+    if (it.lo1 >= it.n1) it.n1 = it.lo1 = 0;
+  }
   it.nmax = max(it.n0, it.n1);
+  it.jb = it.n0 > 0 ? it.lo0 : it.lo1;  // tile 1 never starts before tile 0
   return it;
 }
 
@@ -207,7 +230,7 @@ __device__ __forceinline__ void issue_pv_tile(uint32_t o_tmem, uint32_t p_tmem, 
                   (acc || k > 0) ? 1u : 0u);
 }
 
-template <int D>
+template <int D, int MODE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -292,7 +315,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         *reinterpret_cast<volatile int*>(&item_ring[k % NI]) = w;
         sm100::mbar_arrive(&item_full[k % NI]);
         if (w < 0) break;
-        const Item it = get_item<D>(p, w, nullptr);
+        const Item it = get_item<D, MODE>(p, w, nullptr);
         if (!sm100::mbar_wait(q_empty, (k & 1) ^ 1, abort_flag, p.status)) break;
         sm100::mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
         const int qh = it.q_head;
@@ -303,7 +326,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                it.q_coord + it.row0 + t * BM, qh);
         const int kvh = it.kv_head;
         bool ok = true;
-        for (int j = 0; j < it.nmax && ok; ++j) {
+        for (int j = it.jb; j < it.nmax && ok; ++j) {
           for (int kv = 0; kv < 2; ++kv, ++use) {
             const int slot = use % C::NS;
             if (!sm100::mbar_wait(&kv_empty[slot], ((use / C::NS) & 1) ^ 1, abort_flag,
@@ -361,20 +384,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
         if (leader) sm100::mbar_arrive(&item_empty[k % NI]);
         if (w < 0) break;
-        const Item it = get_item<D>(p, w, nullptr);
+        const Item it = get_item<D, MODE>(p, w, nullptr);
         if (!(ok = sm100::mbar_wait(q_full, k & 1, abort_flag, p.status))) break;
         sm100::tc_fence_after();
         const uint32_t oe_par = (k & 1) ^ 1;
-        if (it.nmax > 0) {
+        const int jb = it.jb;
+        const int lo[2] = {it.lo0, it.lo1};
+        if (it.nmax > jb) {
           const int ks = use % C::NS;
           if (!(ok = sm100::mbar_wait(&kv_full[ks], (use / C::NS) & 1, abort_flag, p.status)))
             break;
           sm100::tc_fence_after();
-          if (it.n0 > 0) {
+          if (it.n0 > jb && lo[0] == jb) {
             issue_s(0, ks);
             commit(&s_full[0]);
           }
-          if (it.n1 > 0) {
+          if (it.n1 > jb && lo[1] == jb) {
             issue_s(1, ks);
             commit(&s_full[1]);
           }
@@ -382,9 +407,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         // Q is free once the item's last S has run: release it then, so the next
         // item's Q loads while this item's last PV steps execute
-        if (it.nmax <= 1) commit(q_empty);
-        for (int j = 0; j < it.nmax && ok; ++j) {
-          const uint32_t vuse = use + 2 * j + 1;
+        if (it.nmax - jb <= 1) commit(q_empty);
+        for (int j = jb; j < it.nmax && ok; ++j) {
+          const uint32_t vuse = use + 2 * (j - jb) + 1;
           const int vs = vuse % C::NS;
           const uint32_t kuse = vuse + 1;
           const int ks = kuse % C::NS;
@@ -394,16 +419,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           sm100::tc_fence_after();
           // one query tile's step: O_t += P_t V_j, then S_t = Q_t K_{j+1}^T
           auto step = [&](int t, int n_t, uint32_t& pc) -> bool {
-            if (j < n_t) {
-              if (j == 0 && !sm100::mbar_wait(&o_empty[t], oe_par, abort_flag, p.status))
+            if (lo[t] <= j && j < n_t) {
+              if (j == lo[t] && !sm100::mbar_wait(&o_empty[t], oe_par, abort_flag, p.status))
                 return false;
               if (!sm100::mbar_wait(&p_full[t], pc & 1, abort_flag, p.status)) return false;
               ++pc;
               sm100::tc_fence_after();
-              issue_pv(t, vs, j > 0);
+              issue_pv(t, vs, j > lo[t]);
               if (j == n_t - 1) commit(&o_full[t]);
             }
-            if (j + 1 < n_t) {
+            if (lo[t] <= j + 1 && j + 1 < n_t) {
               if (!k_ready) {
                 if (!sm100::mbar_wait(&kv_full[ks], (kuse / C::NS) & 1, abort_flag, p.status))
                   return false;
@@ -430,7 +455,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!(ok = sm100::mbar_wait(&o_empty[1], oe_par, abort_flag, p.status))) break;
           commit(&o_full[1]);
         }
-        use += 2 * it.nmax;
+        use += 2 * (it.nmax - jb);
       }
       // all issued tensor-core work (and its commits) must land before TMEM is freed
       commit(drain);
@@ -458,14 +483,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int w;
       if (!(ok = next_item(k, w)) || w < 0) break;
       bool bad = false;
-      const Item it = get_item<D>(p, w, &bad);
+      const Item it = get_item<D, MODE>(p, w, &bad);
       if (bad && threadIdx.x == 0) atomicOr(p.status, 1);
       const int n_t = t ? it.n1 : it.n0;
       const int row0 = it.row0 + t * BM;
       const int row = row0 + r;
       const int diag = row + it.koff;  // last visible key under the causal mask
       float m_use = -INFINITY, l = 0.f;
-      for (int j = 0; j < n_t; ++j) {
+      const int lo_t = t ? it.lo1 : it.lo0;
+      for (int j = lo_t; j < n_t; ++j) {
         if (!(ok = sm100::mbar_wait(&s_full[t], s_cnt & 1, abort_flag, p.status))) break;
         float* red_w = red + ((s_cnt & 1) * 4 + t * 2) * BM;
         ++s_cnt;
@@ -476,13 +502,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         sm100::tmem_ld_wait();
 
         const int k0 = j * BN + 64 * hf;
+        // sliding window: keys at or below the last row's window edge may be masked
+        const bool win_edge =
+            MODE == MODE_WINDOW && k0 <= row0 + (BM - 1) + it.koff - p.window;
         const bool need_mask =
-            (k0 + 64 > it.kv_len) || (p.causal && (k0 + 63 > row0 + it.koff));
+            (k0 + 64 > it.kv_len) || (p.causal && (k0 + 63 > row0 + it.koff)) || win_edge;
         if (need_mask) {
           const int lim = p.causal ? min(it.kv_len - 1, diag) : it.kv_len - 1;
+          const int lo_key = MODE == MODE_WINDOW ? diag - p.window + 1 : INT_MIN;
 #pragma unroll
           for (int c = 0; c < 64; ++c)
-            if (k0 + c > lim) s[c] = __float_as_uint(-INFINITY);
+            if (k0 + c > lim || k0 + c < lo_key) s[c] = __float_as_uint(-INFINITY);
         }
         float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
@@ -499,7 +529,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const float m_upd = fmaxf(m_use, m_new);
           const float alpha = (m_use == -INFINITY) ? 0.f : sm100::ex2(m_use - m_upd);
           l *= alpha;
-          if (j > 0) {
+          if (j > lo_t) {
             // O holds PV of the previous tiles (complete: S of this tile was
             // committed after them); rescale this thread's half in place
 #pragma unroll 1
@@ -557,8 +587,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       const bool live = row < it.lq;
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
-      __nv_bfloat16* orow =
-          p.O + it.o_off + (live ? row : 0) * it.o_rstride + DH * hf;
+      __nv_bfloat16* orow;
+      if constexpr (MODE == MODE_VARLEN)
+        orow = p.O + it.o_off + (live ? row : 0) * it.o_rstride + DH * hf;
+      else
+        orow = p.O + ((static_cast<size_t>(it.b) * p.Hq + it.h) * p.Lq + (live ? row : 0)) * D +
+               DH * hf;
       if (n_t > 0) {
 #pragma unroll 1
         for (int c = 0; c < DH / 32; ++c) {
@@ -582,7 +616,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int v = 0; v < DH / 8; ++v) dst[v] = make_uint4(0, 0, 0, 0);
       }
       if (live && p.lse && hf == 0)
-        p.lse[it.lse_off + row] =
+        p.lse[MODE == MODE_VARLEN ? it.lse_off + row
+                                  : (static_cast<size_t>(it.b) * p.Hq + it.h) * p.Lq + row] =
             (l > 0.f) ? (m_use + log2f(l)) * 0.69314718055994531f : -INFINITY;
       sm100::tc_fence_before();
       __syncwarp();

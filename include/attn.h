@@ -97,6 +97,29 @@ attn_status_t attn_fwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf
                        int d, float scale, int mask_flags, const int32_t* k_lens,
                        void* workspace, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------ sliding window
+ * Local causal (sliding-window) attention: the causal mask of attn_fwd /
+ * attn_bwd plus a lower edge, so query row i sees only keys j with
+ *   i + (Lk - Lq) - window < j <= i + (Lk - Lq)   (and j < k_lens[b]).
+ * The pages name local / causal / padding masks as variants of M; the window
+ * convention (the `window` latest keys, the diagonal included) is ours.  Key
+ * tiles entirely outside a query tile's window are skipped, so the work
+ * grows with window, not with Lk.  window >= 1 (else ATTN_ERR_INVALID); all
+ * other arguments, layouts and errors as attn_fwd / attn_bwd with
+ * mask_flags = ATTN_MASK_CAUSAL (attn_bwd_sliding takes the lse that
+ * attn_fwd_sliding wrote for the same window).
+ */
+attn_status_t attn_fwd_sliding(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf16_t* V,
+                               attn_bf16_t* O, float* lse, int B, int Hq, int Hkv, int Lq, int Lk,
+                               int d, float scale, int window, const int32_t* k_lens,
+                               void* workspace, size_t ws_bytes, void* stream);
+attn_status_t attn_bwd_sliding(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf16_t* V,
+                               const attn_bf16_t* O, const attn_bf16_t* dO, const float* lse,
+                               attn_bf16_t* dQ, attn_bf16_t* dK, attn_bf16_t* dV, int B, int Hq,
+                               int Hkv, int Lq, int Lk, int d, float scale, int window,
+                               const int32_t* k_lens, void* workspace, size_t ws_bytes,
+                               void* stream);
+
 /* ------------------------------------------------------------------ packed forward
  * The forward over variable-length sequences packed back to back (no padding):
  * the same attention per sequence as attn_fwd, with the batch given by

@@ -117,6 +117,15 @@ def test_varlen_fwd_rejects_on_host(lib):
     assert call(mq=0) == 0 and call(tq=0) == 0  # nothing to compute: returns at once
 
 
+def test_sliding_rejects_on_host(lib):
+    assert lib.attn_fwd_sliding(P, P, P, P, None, 1, 2, 1, 8, 8, 128, 0.1, 0, None, P, 256,
+                                None) == 1
+    assert lib.attn_fwd_sliding(P, P, P, P, None, 1, 2, 1, 8, 8, 96, 0.1, 4, None, P, 256,
+                                None) == 2
+    assert lib.attn_bwd_sliding(P, P, P, P, P, P, P, P, P, 1, 1, 1, 8, 8, 128, 0.1, -3, None, P,
+                                1 << 20, None) == 1
+
+
 def test_product_path_does_not_touch_oracle():
     """The CUDA binding must neither import nor load anything from oracle/."""
     pkg = os.path.join(ROOT, "exact_io_aware_46_b200")
