@@ -30,6 +30,7 @@ FWD_CASES = [
     (1, 2, 2, 600, 600, 128, 300, [600]),
     (1, 2, 2, 300, 900, 128, 256, None),        # Lq < Lk: bottom-right alignment
     (2, 2, 2, 513, 513, 64, 200, [513, 301]),   # d = 64, key padding
+    (1, 2, 2, 500, 300, 128, 64, None),         # Lq > Lk: the first 200 rows see no key
 ]
 
 
