@@ -22,6 +22,13 @@ Parity status of each function (what pins it, see ``tests/test_oracle_pins.py``)
   forward's loss on tiny shapes, gradient invariants (columns of dS sum to
   zero, sum_j dV_j = sum_i dO_i), grouped-query equality to the sum of
   per-head gradients, and a torch fp64 autograd witness.
+* ``e4m3_to_f64`` / ``dequant_tiles`` / ``fwd_fp8`` -- pinned: all 256 codes
+  against torch's float8_e4m3fn widening (an independent library witness) and
+  the format's landmark values (448, 2^-6, 2^-9, NaN), the row-to-tile scale
+  assignment on constant codes with ragged tails, and invariances of the
+  scales (a factor on v_scale scales O, a factor on q_scale traded against the
+  softmax scale, a per-tile factor moved between codes and scales); the
+  forward itself is ``fwd`` on the dequantised values.
 * ``online_row`` / ``merge`` -- pinned: the worked example's block statistics
   (block A: m = 5, S = 1.0498; ratio 0.7312; block C = [10] rescale e^-5) and
   brute-force equality with the one-pass softmax over every block split.
@@ -258,3 +265,48 @@ def merge(m_a, l_a, O_a, m_b, l_b, O_b):
     lib.oracle_merge(float(m_a), float(l_a), _p(Oa), float(m_b), float(l_b), _p(Ob), d, _p(m),
                      _p(l), _p(O))
     return float(m[0]), float(l[0]), O
+
+
+# ---------------------------------------------------------------- 8-bit (E4M3) inputs
+# The low-precision forward of the FlashAttention line ("FlashAttention" blog,
+# section 10 on FlashAttention-3: new-hardware features and low-precision
+# execution) takes Q, K and V as 8-bit floats.  The oracle decodes them exactly
+# and runs the fp64 forward above on the dequantised values: it is the exact
+# attention of the inputs the low-precision path is given.
+
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    """Exact values of E4M3 8-bit floats (the OCP 8-bit floating-point format):
+    bit 7 sign, bits 6-3 exponent with bias 7, bits 2-0 mantissa.  Exponent
+    field 0 holds zero and the subnormals (m / 8) * 2^-6; otherwise the value is
+    (1 + m / 8) * 2^(e - 7).  There are no infinities: S.1111.111 is NaN, so the
+    largest finite magnitude is S.1111.110 = 448."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & (c & 0x7 == 7), np.nan, mag)
+    return sign * mag
+
+
+def dequant_tiles(codes, scales, tile: int = 128) -> np.ndarray:
+    """Dequantise [..., L, d] E4M3 codes with one scale per ``tile`` rows:
+    row i of every head is multiplied by scales[..., i // tile]."""
+    x = e4m3_to_f64(codes)
+    L = x.shape[-2]
+    sc = np.asarray(scales, dtype=np.float64)
+    if sc.shape[-1] != (L + tile - 1) // tile:
+        raise ValueError("one scale per row tile expected")
+    return x * sc[..., np.arange(L) // tile][..., None]
+
+
+def fwd_fp8(Q8, K8, V8, q_scale, k_scale, v_scale, scale: float, causal: bool = False,
+            k_lens=None, rows=None, heads=None, tile: int = 128):
+    """Forward of E4M3 inputs with per-tile scales: Q8 [B,Hq,Lq,d] with q_scale
+    [B,Hq,ceil(Lq/tile)], K8/V8 [B,Hkv,Lk,d] with k_scale/v_scale
+    [B,Hkv,ceil(Lk/tile)].  Exact attention (``fwd``) of the dequantised tensors;
+    returns (O, LSE) like ``fwd``."""
+    return fwd(dequant_tiles(Q8, q_scale, tile), dequant_tiles(K8, k_scale, tile),
+               dequant_tiles(V8, v_scale, tile), scale, causal=causal, k_lens=k_lens, rows=rows,
+               heads=heads)

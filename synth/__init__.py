@@ -16,6 +16,8 @@ Generator
 
 The workloads' tensors are i.i.d. N(0, 1) in bf16, laid out ``[B, H, L, d]``
 row-major; per-request key lengths are integers uniform in ``[lo, hi]``.
+8-bit inputs are those bf16 tensors quantised to E4M3 with one fp32 scale per
+128-row tile of each head (the tile's largest magnitude maps to 448).
 """
 
 from __future__ import annotations
@@ -93,6 +95,37 @@ def to_torch_bf16(bits: np.ndarray):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
 
 
+def quantize_e4m3_tiles(x, tile: int = 128):
+    """Quantise a float32 torch tensor [..., L, d] to E4M3 codes with one scale per
+    ``tile`` rows (scale = the tile's largest magnitude / 448, the format's
+    largest finite value); the rounding is torch's float8_e4m3fn conversion.
+    Returns (codes uint8 [..., L, d], scales float32 [..., ceil(L / tile)]) as
+    tensors on x's device."""
+    import torch
+
+    L, d = x.shape[-2], x.shape[-1]
+    nt = (L + tile - 1) // tile
+    lead = x.shape[:-2]
+    xp = torch.zeros(*lead, nt * tile, d, dtype=torch.float32, device=x.device)
+    xp[..., :L, :] = x
+    xt = xp.view(*lead, nt, tile, d)
+    amax = xt.abs().amax(dim=(-1, -2))
+    scale = torch.clamp(amax, min=2.0 ** -100) / 448.0
+    y = torch.clamp(xt / scale[..., None, None], -448.0, 448.0)
+    codes = y.to(torch.float8_e4m3fn).view(torch.uint8).view(*lead, nt * tile, d)[..., :L, :]
+    return codes.contiguous(), scale.contiguous()
+
+
+def normal_e4m3(seed: int, shape, tile: int = 128):
+    """The bf16 N(0,1) tensor of :func:`normal_bf16` quantised per row tile with
+    :func:`quantize_e4m3_tiles`; returns numpy (codes uint8, scales float32)."""
+    import torch
+
+    x = torch.from_numpy(bf16_bits_to_f64(normal_bf16(seed, shape)).astype(np.float32))
+    c, s = quantize_e4m3_tiles(x, tile)
+    return c.numpy(), s.numpy()
+
+
 # Workload seeds: 46 * 100 + workload number; each tensor draws its own stream.
 def workload_seed(workload: int, tensor: str) -> int:
     tags = {"q": 1, "k": 2, "v": 3, "do": 4, "klen": 5, "pages": 6}
@@ -105,6 +138,8 @@ __all__ = [
     "f64_to_bf16_bits",
     "bf16_bits_to_f64",
     "normal_bf16",
+    "quantize_e4m3_tiles",
+    "normal_e4m3",
     "uniform_int",
     "to_torch_bf16",
     "workload_seed",
@@ -152,3 +187,10 @@ def normal_bf16_device(seed: int, shape, device, chunk: int = 1 << 25):
         x = torch.sqrt(-2.0 * torch.log(u1)) * torch.cos(2.0 * np.pi * u2)
         out[s:s + m] = x.to(torch.float32).to(torch.bfloat16)
     return out.view(*shape)
+
+
+def normal_e4m3_device(seed: int, shape, device, tile: int = 128):
+    """Device twin of :func:`normal_e4m3` (drawn with :func:`normal_bf16_device`);
+    returns torch (codes uint8, scales float32) on ``device``."""
+    x = normal_bf16_device(seed, shape, device).float()
+    return quantize_e4m3_tiles(x, tile)

@@ -476,3 +476,96 @@ def test_window_requires_causal():
     with pytest.raises(ValueError):
         oracle.fwd(_rand(1, (1, 1, 4, 8)), _rand(2, (1, 1, 4, 8)), _rand(3, (1, 1, 4, 8)), 1.0,
                    causal=False, window=2)
+
+
+# ---------------------------------------------------------------- 8-bit (E4M3) inputs
+
+
+def test_e4m3_decode_matches_torch_on_every_code():
+    """Library witness: torch's float8_e4m3fn widening of all 256 codes."""
+    import torch
+
+    c = np.arange(256, dtype=np.uint8)
+    got = oracle.e4m3_to_f64(c)
+    ref = torch.from_numpy(c).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan) and nan.sum() == 2  # 0x7F and 0xFF
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def test_e4m3_landmark_values():
+    """The format's fixed points: zero, smallest subnormal and normal, one, the
+    largest finite value, the sign bit."""
+    v = oracle.e4m3_to_f64(np.array([0x00, 0x01, 0x07, 0x08, 0x38, 0x3F, 0x7E, 0xFE, 0xC0],
+                                    dtype=np.uint8))
+    assert list(v) == [0.0, 2.0 ** -9, 7 * 2.0 ** -9, 2.0 ** -6, 1.0, 1.875, 448.0, -448.0, -2.0]
+    assert np.signbit(oracle.e4m3_to_f64(np.array([0x80], dtype=np.uint8)))[0]
+
+
+@pytest.mark.parametrize("L", [1, 128, 129, 300])
+def test_dequant_assigns_each_row_its_tile_scale(L):
+    """Constant codes 0x38 (= 1.0): every dequantised row equals the scale of
+    tile i // 128, including the ragged last tile."""
+    nt = (L + 127) // 128
+    codes = np.full((2, 3, L, 8), 0x38, dtype=np.uint8)
+    scales = (np.arange(2 * 3 * nt, dtype=np.float32).reshape(2, 3, nt) + 1.0) * 0.125
+    x = oracle.dequant_tiles(codes, scales)
+    for i in range(L):
+        assert np.all(x[:, :, i, :] == scales[:, :, i // 128][..., None])
+    with pytest.raises(ValueError):
+        oracle.dequant_tiles(codes, scales[..., :nt - 1] if nt > 1 else np.zeros((2, 3, 2)))
+
+
+def _fp8_case(seed, B=1, Hq=2, Hkv=1, Lq=200, Lk=300, d=16):
+    Q8, qs = synth.normal_e4m3(seed, (B, Hq, Lq, d))
+    K8, ks = synth.normal_e4m3(seed + 1, (B, Hkv, Lk, d))
+    V8, vs = synth.normal_e4m3(seed + 2, (B, Hkv, Lk, d))
+    return Q8, K8, V8, qs, ks, vs
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_scale_invariances(causal):
+    """A factor c on every V scale multiplies O by c and leaves LSE; a factor on
+    the Q scales traded against the softmax scale changes nothing; a per-tile
+    power of two moved from K's codes into K's scales changes nothing (catches a
+    Q/K/V scale mix-up or a wrong tile index)."""
+    Q8, K8, V8, qs, ks, vs = _fp8_case(931)
+    sc = 0.25
+    O, L = oracle.fwd_fp8(Q8, K8, V8, qs, ks, vs, sc, causal=causal)
+    O2, L2 = oracle.fwd_fp8(Q8, K8, V8, qs, ks, vs.astype(np.float64) * 3.0, sc, causal=causal)
+    assert np.allclose(O2, 3.0 * O, rtol=1e-13, atol=1e-14) and np.allclose(L2, L, atol=1e-13)
+    O3, L3 = oracle.fwd_fp8(Q8, K8, V8, qs.astype(np.float64) * 3.0, ks, vs, sc / 3.0, causal=causal)
+    assert np.allclose(O3, O, atol=1e-13) and np.allclose(L3, L, atol=1e-13)
+    # halve the codes of K tile 1 (exponent field - 1 on normal codes) and double its scale
+    K8b, ksb = K8.copy(), ks.copy()
+    t1 = K8b[:, :, 128:256, :]
+    e = (t1 >> 3) & 0xF
+    assert np.all((e >= 2) | (t1 & 0x7F == 0)), "test codes must stay normal when halved"
+    t1[...] = np.where(t1 & 0x7F == 0, t1, t1 - 8)
+    ksb[:, :, 1] *= 2.0
+    O4, L4 = oracle.fwd_fp8(Q8, K8b, V8, qs, ksb, vs, sc, causal=causal)
+    assert np.allclose(O4, O, atol=1e-13) and np.allclose(L4, L, atol=1e-13)
+
+
+def test_fp8_brute_force_against_torch():
+    """Tiny case: decode with torch, assign tile scales row by row, softmax in
+    torch fp64 -- against the oracle."""
+    import torch
+
+    Q8, K8, V8, qs, ks, vs = _fp8_case(977, B=2, Hq=2, Hkv=2, Lq=140, Lk=260, d=8)
+
+    def deq(c, s):
+        x = torch.from_numpy(c).view(torch.float8_e4m3fn).to(torch.float64)
+        out = torch.empty_like(x)
+        for i in range(x.shape[2]):
+            out[:, :, i, :] = x[:, :, i, :] * torch.from_numpy(s[:, :, i // 128].astype(np.float64))[..., None]
+        return out
+
+    q, k, v = deq(Q8, qs), deq(K8, ks), deq(V8, vs)
+    s = q @ k.transpose(-1, -2) * 0.3
+    i = torch.arange(140)[:, None]
+    j = torch.arange(260)[None, :]
+    s = s.masked_fill(~(j <= i + 120), float("-inf"))
+    O, L = oracle.fwd_fp8(Q8, K8, V8, qs, ks, vs, 0.3, causal=True)
+    assert np.max(np.abs(O - (torch.softmax(s, -1) @ v).numpy())) <= 1e-12
+    assert np.max(np.abs(L - torch.logsumexp(s, -1).numpy())) <= 1e-12
