@@ -280,9 +280,24 @@ def fwd_leg(steps, warmup, world, flush):
     if st[0] != attn.ATTN_OK:
         raise RuntimeError(f"device status {st}")
     wflops = 4.0 * c["d"] * c["B"] * c["Hq"] * sum(min(i + 1, W) for i in range(c["L"]))
-    del q, k, v, O, lse, hq, hk, hv, hO, hL
+    # the same workload with E4M3 inputs: these tensors quantised per 128-row tile
+    del hq, hk, hv, hO, hL
+    q8, qs = synth.quantize_e4m3_tiles(q.float())
+    k8, ks = synth.quantize_e4m3_tiles(k.float())
+    v8, vs = synth.quantize_e4m3_tiles(v.float())
+    del q, k, v
     torch.cuda.empty_cache()
-    return ms, ms_e2e, h2d, d2h, varlen_leg(steps, warmup, world, flush), (W, wms, wflops)
+    call_8 = lambda: attn.attn_fwd_fp8(q8, k8, v8, qs, ks, vs, causal=True, O=O, lse=lse,
+                                       workspace=ws, stream=stream)
+    barrier(world)
+    fms = timed_loop(call_8, steps, warmup, stream, flush)
+    st = attn.attn_read_device_status(ws)
+    if st[0] != attn.ATTN_OK:
+        raise RuntimeError(f"device status {st}")
+    del q8, k8, v8, qs, ks, vs, O, lse
+    torch.cuda.empty_cache()
+    return (ms, ms_e2e, h2d, d2h, varlen_leg(steps, warmup, world, flush), (W, wms, wflops),
+            fms)
 
 
 WINDOW = 1024
@@ -517,7 +532,7 @@ def main():
     with Clocks(gpu_idx) as clk:
         if "fwd" in legs:
             (ms, ms_e2e, h2d, d2h, (vms, vflops, vtotal),
-             (W, wms, wflops)) = fwd_leg(args.steps, args.warmup, world, flush)
+             (W, wms, wflops), fms) = fwd_leg(args.steps, args.warmup, world, flush)
         if "decode" in legs:
             dms, kv_bytes, _, (page, pms) = decode_leg(args.steps, args.warmup, world, flush)
         if "bwd" in legs:
@@ -544,7 +559,9 @@ def main():
     value = world * flops / (t_step * 1e-3) / 1e12
     achieved = flops / (float(np.mean(ms)) * 1e-3) / 1e12
     # one persistent forward kernel per step: timed forward, e2e and packed-prefill loops
-    launches = args.steps + max(3, args.steps // 2) + args.steps + args.steps
+    # one persistent forward kernel per step: timed forward, e2e, sliding-window, 8-bit and
+    # packed-prefill loops
+    launches = args.steps + max(3, args.steps // 2) + args.steps + args.steps + args.steps
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -582,6 +599,21 @@ def main():
                     f"keys (FLOPs over visible pairs)",
         "value": world * wflops / (t_w * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": t_w,
         "flops_per_step": wflops,
+    }
+    t_8 = max_over_ranks(float(np.mean(fms)), world)
+    ach8 = flops / (float(np.mean(fms)) * 1e-3) / 1e12
+    peak8 = 2.0 * pk["bf16_tflops"]
+    line["fp8"] = {
+        "workload": "the causal prefill forward B4 H16 L4096 d128 with E4M3 Q, K, V (the same "
+                    "tensors quantised with one scale per 128-row tile), O bf16 + LSE fp32",
+        "value": world * flops / (t_8 * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": t_8,
+        "flops_per_step": flops, "dtype": "e4m3 (fp32 accumulate)",
+        "roofline": {"bound": "tensor", "achieved": ach8, "peak": peak8, "unit": "TFLOP/s",
+                     "frac": ach8 / peak8,
+                     "traffic": traffic_per_launch("attn_fwd_impl::fwd_kernel<128,MODE_FP8>"),
+                     "peak_source": f"{pk['source']} burst bf16 x 2 (the nominal 8-bit:bf16 "
+                                    f"dense ratio, 4.5 : 2.25 PFLOP/s)",
+                     "kernel": "attn_fwd_impl::fwd_kernel<128,MODE_FP8>"},
     }
     if "decode" in legs:
         t_d = max_over_ranks(float(np.mean(dms)), world)

@@ -13,6 +13,8 @@ The functions carry the C entry points' names:
 * ``attn_fwd_splitkv_decode_paged(Q, Kpages, Vpages, block_table, k_lens, ...) -> (O, LSE)``
 * ``attn_bwd(Q, K, V, O, dO, LSE, ...) -> (dQ, dK, dV)``
 * ``attn_fwd_sliding`` / ``attn_bwd_sliding``: the same with a sliding-window causal mask
+* ``attn_fwd_fp8(Q8, K8, V8, q_scale, k_scale, v_scale, ...) -> (O, LSE)``: E4M3 inputs with
+  one scale per 128-row tile
 * the ``*_workspace_size`` queries and the device-status helpers.
 """
 
@@ -33,7 +35,7 @@ LIB_PATH = os.path.join(_HERE, "libattn.so")
 #: size of the fixed device scratch used by attn_fwd_splitkv_decode_noalloc
 ATTN_NOALLOC_SCRATCH_BYTES = 16 << 20
 ATTN_MASK_NONE, ATTN_MASK_CAUSAL = 0, 1
-ATTN_DEV_BAD_KLEN, ATTN_DEV_TIMEOUT, ATTN_DEV_BAD_PAGE = 1, 2, 4
+ATTN_DEV_BAD_KLEN, ATTN_DEV_TIMEOUT, ATTN_DEV_BAD_PAGE, ATTN_DEV_BAD_SCALE = 1, 2, 4, 8
 
 _lock = threading.Lock()
 _lib = None
@@ -52,6 +54,8 @@ SIGNATURES = {
                       _vp]),
     "attn_fwd_sliding": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _vp,
                               _sz, _vp]),
+    "attn_fwd_fp8": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i,
+                          _vp, _vp, _sz, _vp]),
     "attn_bwd_sliding": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                               _f, _i, _vp, _vp, _sz, _vp]),
     "attn_fwd_varlen_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
@@ -182,6 +186,47 @@ def attn_fwd(Q, K, V, scale=None, causal=False, k_lens=None, O=None, lse=None, w
                           float(scale), ATTN_MASK_CAUSAL if causal else ATTN_MASK_NONE,
                           _ptr(k_lens), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(code, "attn_fwd")
+    return O, lse
+
+
+def _u8(t, name):
+    if t.dtype != torch.uint8 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA uint8 tensor of E4M3 codes")
+
+
+def _f32(t, name):
+    if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA float32 tensor")
+
+
+def attn_fwd_fp8(Q8, K8, V8, q_scale, k_scale, v_scale, scale=None, causal=False, k_lens=None,
+                 O=None, lse=None, workspace=None, stream=None, want_lse=True):
+    """Forward of E4M3 inputs.  Q8 [B,Hq,Lq,d], K8/V8 [B,Hkv,Lk,d] uint8 codes;
+    q_scale [B,Hq,ceil(Lq/128)], k_scale/v_scale [B,Hkv,ceil(Lk/128)] fp32 (one
+    scale per 128-row tile).  Returns (O bf16 [B,Hq,Lq,d], LSE fp32 [B,Hq,Lq])."""
+    for t, n in ((Q8, "Q8"), (K8, "K8"), (V8, "V8")):
+        _u8(t, n)
+    for t, n in ((q_scale, "q_scale"), (k_scale, "k_scale"), (v_scale, "v_scale")):
+        _f32(t, n)
+    B, Hq, Lq, d = Q8.shape
+    Hkv, Lk = K8.shape[1], K8.shape[2]
+    if tuple(q_scale.shape) != (B, Hq, (Lq + 127) // 128) or \
+            tuple(k_scale.shape) != (B, Hkv, (Lk + 127) // 128) or \
+            tuple(v_scale.shape) != (B, Hkv, (Lk + 127) // 128):
+        raise ValueError("one scale per 128-row tile of each head expected")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if O is None:
+        O = torch.empty((B, Hq, Lq, d), dtype=torch.bfloat16, device=Q8.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=Q8.device)
+    if workspace is None:
+        workspace = _workspace(attn_fwd_workspace_size(B, Hq, Hkv, Lq, Lk, d), Q8.device, stream)
+    code = lib().attn_fwd_fp8(_ptr(Q8), _ptr(K8), _ptr(V8), _ptr(q_scale), _ptr(k_scale),
+                              _ptr(v_scale), _ptr(O), _ptr(lse), B, Hq, Hkv, Lq, Lk, d,
+                              float(scale), ATTN_MASK_CAUSAL if causal else ATTN_MASK_NONE,
+                              _ptr(k_lens), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(code, "attn_fwd_fp8")
     return O, lse
 
 

@@ -71,6 +71,23 @@ bool make_tmap_packed(CUtensorMap* m, const void* base, int d, int T, int heads,
   return r == CUDA_SUCCESS;
 }
 
+// 3-D 8-bit view [heads][rows][d] of a [B, H, L, d] E4M3 tensor, boxes of
+// 128 columns (128 bytes) x `box_rows` rows x 1 head, 128-byte swizzle.
+bool make_tmap_u8(CUtensorMap* m, const void* base, int d, int L, long long heads, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L > 0 ? L : 1),
+                        static_cast<cuuint64_t>(heads)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d),
+                           static_cast<cuuint64_t>(d) * static_cast<cuuint64_t>(L > 0 ? L : 1)};
+  cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int device_sms() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -123,8 +140,10 @@ static attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, co
   p.n_pairs = n_pairs;
   p.n_items = n_items;
   const int grid = n_items < sms ? n_items : sms;
-  const int mode = p.cu_q ? attn_fwd_impl::MODE_VARLEN
-                          : (p.window > 0 ? attn_fwd_impl::MODE_WINDOW : attn_fwd_impl::MODE_PLAIN);
+  const int mode = p.cu_q      ? attn_fwd_impl::MODE_VARLEN
+                   : p.q_scale ? attn_fwd_impl::MODE_FP8
+                   : p.window > 0 ? attn_fwd_impl::MODE_WINDOW
+                                  : attn_fwd_impl::MODE_PLAIN;
   cudaError_t e = cudaSuccess;
   auto run = [&](auto kernel, int smem) {
     e = set_smem(kernel, smem);
@@ -135,8 +154,10 @@ static attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, co
     constexpr int smem = Cfg<128>::SMEM_BYTES;
     if (mode == MODE_PLAIN) run(fwd_kernel<128, MODE_PLAIN>, smem);
     else if (mode == MODE_WINDOW) run(fwd_kernel<128, MODE_WINDOW>, smem);
+    else if (mode == MODE_FP8) run(fwd_kernel<128, MODE_FP8>, Cfg<128, 1>::SMEM_BYTES);
     else run(fwd_kernel<128, MODE_VARLEN>, smem);
   } else {
+    if (mode == MODE_FP8) return ATTN_ERR_UNSUPPORTED;
     constexpr int smem = Cfg<64>::SMEM_BYTES;
     if (mode == MODE_PLAIN) run(fwd_kernel<64, MODE_PLAIN>, smem);
     else if (mode == MODE_WINDOW) run(fwd_kernel<64, MODE_WINDOW>, smem);
@@ -210,6 +231,40 @@ attn_status_t attn_fwd_sliding(const attn_bf16_t* Q, const attn_bf16_t* K, const
   if (window < 1) return ATTN_ERR_INVALID;
   return fwd_batched(Q, K, V, O, lse, B, Hq, Hkv, Lq, Lk, d, scale, ATTN_MASK_CAUSAL, window,
                      k_lens, workspace, ws_bytes, stream);
+}
+
+attn_status_t attn_fwd_fp8(const void* Q8, const void* K8, const void* V8, const float* q_scale,
+                           const float* k_scale, const float* v_scale, attn_bf16_t* O, float* lse,
+                           int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale,
+                           int mask_flags, const int32_t* k_lens, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  if (!shapes_ok(B, Hq, Hkv, Lq, Lk)) return ATTN_ERR_INVALID;
+  if (!Q8 || !K8 || !V8 || !q_scale || !k_scale || !v_scale || !O || !workspace)
+    return ATTN_ERR_INVALID;
+  if (!aligned16(Q8) || !aligned16(K8) || !aligned16(V8) || !aligned16(O) ||
+      !aligned16(q_scale) || !aligned16(k_scale) || !aligned16(v_scale) ||
+      (lse && !aligned16(lse)) || (k_lens && !aligned16(k_lens)) || !aligned256(workspace))
+    return ATTN_ERR_INVALID;
+  if (!(std::isfinite(scale) && scale > 0.f)) return ATTN_ERR_INVALID;
+  if (mask_flags != ATTN_MASK_NONE && mask_flags != ATTN_MASK_CAUSAL) return ATTN_ERR_INVALID;
+  if (ws_bytes < attn_fwd_workspace_size(B, Hq, Hkv, Lq, Lk, d)) return ATTN_ERR_INVALID;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (Lq == 0) return ATTN_OK;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_u8(&tq, Q8, d, Lq, static_cast<long long>(B) * Hq, 128) ||
+      !make_tmap_u8(&tk, K8, d, Lk, static_cast<long long>(B) * Hkv, 128) ||
+      !make_tmap_u8(&tv, V8, d, Lk, static_cast<long long>(B) * Hkv, 128))
+    return ATTN_ERR_CUDA;
+  attn_fwd_impl::Params p{};
+  p.k_lens = k_lens;
+  p.Lq = Lq;
+  p.Lk = Lk;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.n_qt = (Lq + attn_fwd_impl::BM - 1) / attn_fwd_impl::BM;
+  p.n_kt = (Lk + attn_fwd_impl::BN - 1) / attn_fwd_impl::BN;
+  return launch_fwd(tq, tk, tv, p, O, lse, B, Hq, Hkv, d, scale, mask_flags, workspace, stream);
 }
 
 size_t attn_fwd_varlen_workspace_size(int, int, int, int, int, int) { return kStatusBytes; }
@@ -401,7 +456,7 @@ attn_status_t attn_read_device_status(const void* workspace, void* stream, int32
   if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
   if (bits) *bits = v;
   if (v & ATTN_DEV_TIMEOUT) return ATTN_ERR_TIMEOUT;
-  if (v & (ATTN_DEV_BAD_KLEN | ATTN_DEV_BAD_PAGE)) return ATTN_ERR_INVALID;
+  if (v & (ATTN_DEV_BAD_KLEN | ATTN_DEV_BAD_PAGE | ATTN_DEV_BAD_SCALE)) return ATTN_ERR_INVALID;
   return ATTN_OK;
 }
 

@@ -46,11 +46,14 @@ constexpr int W_MMA = NSMX + 1;
 constexpr int CHUNK_BYTES = 128 * 128;  // one 128-row x 64-column bf16 swizzle panel
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 
-template <int D>
+// EB: bytes per element of Q, K and V (2: bf16, 1: E4M3)
+template <int D, int EB = 2>
 struct Cfg {
-  static constexpr int CHUNKS = D / 64;
-  static constexpr int TILE_BYTES = BM * D * 2;
-  static constexpr int NS = (D == 128) ? 4 : 8;
+  static constexpr int PANEL = 128 / EB;  // elements per 128-byte swizzle panel row
+  static constexpr int CHUNKS = D / PANEL;
+  static constexpr int KSTEP = 32 / EB;   // K elements per MMA instruction (32 bytes)
+  static constexpr int TILE_BYTES = BM * D * EB;
+  static constexpr int NS = (TILE_BYTES == 32768) ? 4 : 8;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * TILE_BYTES;
   // row-max exchange [parity][tile][half][row] and row-sum exchange (same shape)
@@ -59,12 +62,14 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_LSUM + 2 * 2 * 2 * BM * 4;
   static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;  // barriers, item ring + alignment slack
   // TMEM columns: S_0, S_1 (128 fp32 columns each), then O_0, O_1 (D columns
-  // each).  The P of key half h (64 keys, packed bf16 pairs) overwrites the
-  // first 32 of the 64 S columns that half h was read from.
+  // each).  The P of key half h (64 keys: packed bf16 pairs, or E4M3 quads)
+  // overwrites the first 32 (16) of the 64 S columns that half h was read from.
   __device__ static constexpr uint32_t s_col(int t) { return t * 128u; }
   __device__ static constexpr uint32_t o_col(int t) { return 256u + t * D; }
-  static constexpr uint32_t IDESC_S = sm100::idesc_bf16_f32(128, BN, false, false);
-  static constexpr uint32_t IDESC_PV = sm100::idesc_bf16_f32(128, D, false, true);
+  static constexpr uint32_t IDESC_S = EB == 2 ? sm100::idesc_bf16_f32(128, BN, false, false)
+                                               : sm100::idesc_e4m3_f32(128, BN, false, false);
+  static constexpr uint32_t IDESC_PV = EB == 2 ? sm100::idesc_bf16_f32(128, D, false, true)
+                                                : sm100::idesc_e4m3_f32(128, D, false, true);
 };
 
 struct Params {
@@ -85,6 +90,12 @@ struct Params {
   const int* cu_k;
   int total_q, total_k;
   int window;  // > 0: sliding window (with causal): a row sees its `window` latest keys
+  // 8-bit inputs: one fp32 scale per 128-row tile of each head; a dequantised
+  // row i is code * scale[head][i / 128].  nullptr for bf16 inputs.
+  const float* q_scale;  // [B * Hq][n_qt]
+  const float* k_scale;  // [B * Hkv][n_kt]
+  const float* v_scale;  // [B * Hkv][n_kt]
+  int n_qt, n_kt;
 };
 
 struct Item {
@@ -108,8 +119,11 @@ struct Item {
 // MMA-issuing warp):
 //   MODE_PLAIN   [B, H, L, d] tensors, optional causal mask and key padding;
 //   MODE_WINDOW  the same with a sliding-window causal mask (p.window keys);
-//   MODE_VARLEN  packed sequences [T, H, d] with cu_seqlens offsets.
-enum : int { MODE_PLAIN = 0, MODE_WINDOW = 1, MODE_VARLEN = 2 };
+//   MODE_VARLEN  packed sequences [T, H, d] with cu_seqlens offsets;
+//   MODE_FP8     the plain layout with E4M3 Q, K, V and per-tile scales.
+enum : int { MODE_PLAIN = 0, MODE_WINDOW = 1, MODE_VARLEN = 2, MODE_FP8 = 3 };
+
+constexpr int DEV_BAD_SCALE = 8;  // device status bit: a scale that is not finite and > 0
 
 constexpr int HEAD_GROUP = 8;  // heads whose items are interleaved (L2 reuse of their K/V)
 constexpr int NI = 4;          // depth of the shared-memory item ring
@@ -202,39 +216,53 @@ __device__ __forceinline__ Item get_item(const Params& p, int w, bool* bad) {
 __device__ __forceinline__ constexpr bool poly_pair(int cp) { return (cp & 7) == 7; }
 
 // S_t = Q_t K_j^T: 128 x 128 (keys) x D, both operands K-major SW128 panels.
-// One base descriptor per operand; the K-steps add constant offsets (>> 4) to
-// the start-address field.  Inlined: an out-of-line call put its argument and
-// descriptor set-up between consecutive MMAs.
-template <int D>
+// One base descriptor per operand; the K-steps (32 bytes each: 16 bf16 or 32
+// E4M3 elements) add constant offsets (>> 4) to the start-address field.
+// Inlined: an out-of-line call put its argument and descriptor set-up between
+// consecutive MMAs.
+template <int D, int EB>
 __device__ __forceinline__ void issue_s_tile(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+  using C = Cfg<D, EB>;
   const uint64_t qd = sm100::sdesc_sw128(q_smem, 16, 1024);
   const uint64_t kd = sm100::sdesc_sw128(k_smem, 16, 1024);
 #pragma unroll
-  for (int k = 0; k < D / 16; ++k) {
+  for (int k = 0; k < D / C::KSTEP; ++k) {
     const uint64_t off = static_cast<uint64_t>(((k >> 2) * CHUNK_BYTES + (k & 3) * 32) >> 4);
-    sm100::mma_ss(d_tmem, qd + off, kd + off, Cfg<D>::IDESC_S, k > 0 ? 1u : 0u);
+    if constexpr (EB == 2)
+      sm100::mma_ss(d_tmem, qd + off, kd + off, C::IDESC_S, k > 0 ? 1u : 0u);
+    else
+      sm100::mma_ss_f8(d_tmem, qd + off, kd + off, C::IDESC_S, k > 0 ? 1u : 0u);
   }
 }
 
-// O_t (+)= P_t V_j: A = P_t from TMEM (packed bf16, 8 columns per 16 keys;
-// keys 64..127 start 64 columns further on), B = V_j MN-major (LBO = next
-// 64-column panel, SBO = next 8 keys).
-template <int D>
+// O_t (+)= P_t V_j: A = P_t from TMEM (8 columns per instruction: 16 keys of
+// packed bf16 or 32 keys of E4M3; keys 64..127 start 64 columns further on),
+// B = V_j MN-major (LBO = next 128-byte panel of columns, SBO = next 8 keys);
+// consecutive instructions start 16 (bf16) or 32 (E4M3) key rows further on.
+template <int D, int EB>
 __device__ __forceinline__ void issue_pv_tile(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem,
                                               bool acc) {
+  using C = Cfg<D, EB>;
+  constexpr int KS = C::KSTEP;        // keys per instruction
+  constexpr int PER_HALF = 64 / KS;   // instructions per 64-key half
   const uint64_t vd = sm100::sdesc_sw128(v_smem, CHUNK_BYTES, 1024);
 #pragma unroll
-  for (int k = 0; k < BN / 16; ++k)
-    sm100::mma_ts(o_tmem, p_tmem + (k >> 2) * 64 + (k & 3) * 8,
-                  vd + static_cast<uint64_t>((k * 2048) >> 4), Cfg<D>::IDESC_PV,
-                  (acc || k > 0) ? 1u : 0u);
+  for (int k = 0; k < BN / KS; ++k) {
+    const uint32_t a = p_tmem + (k / PER_HALF) * 64 + (k % PER_HALF) * 8;
+    const uint64_t b = vd + static_cast<uint64_t>((k * KS * 128) >> 4);
+    if constexpr (EB == 2)
+      sm100::mma_ts(o_tmem, a, b, C::IDESC_PV, (acc || k > 0) ? 1u : 0u);
+    else
+      sm100::mma_ts_f8(o_tmem, a, b, C::IDESC_PV, (acc || k > 0) ? 1u : 0u);
+  }
 }
 
 template <int D, int MODE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const Params p) {
-  using C = Cfg<D>;
+  constexpr int EB = MODE == MODE_FP8 ? 1 : 2;
+  using C = Cfg<D, EB>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle panels
   const uint32_t raw_addr = sm100::smem_u32(smem_raw);
@@ -322,8 +350,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int t = 0; t < 2; ++t)
           for (int c = 0; c < C::CHUNKS; ++c)
             sm100::tma_load_3d(&tmQ, q_full,
-                               smem + C::OFF_Q + t * C::TILE_BYTES + c * CHUNK_BYTES, c * 64,
-                               it.q_coord + it.row0 + t * BM, qh);
+                               smem + C::OFF_Q + t * C::TILE_BYTES + c * CHUNK_BYTES,
+                               c * C::PANEL, it.q_coord + it.row0 + t * BM, qh);
         const int kvh = it.kv_head;
         bool ok = true;
         for (int j = it.jb; j < it.nmax && ok; ++j) {
@@ -338,7 +366,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int c = 0; c < C::CHUNKS; ++c)
               sm100::tma_load_3d(kv == 0 ? &tmK : &tmV, &kv_full[slot],
                                  smem + C::OFF_KV + slot * C::TILE_BYTES + c * CHUNK_BYTES,
-                                 c * 64, it.k_coord + j * BN, kvh);
+                                 c * C::PANEL, it.k_coord + j * BN, kvh);
           }
         }
         if (!ok) break;
@@ -368,12 +396,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       };
       auto issue_s = [&](int t, int slot) {
         if (leader)
-          issue_s_tile<D>(tmem + C::s_col(t), q_addr + t * C::TILE_BYTES,
+          issue_s_tile<D, EB>(tmem + C::s_col(t), q_addr + t * C::TILE_BYTES,
                           kv_addr + slot * C::TILE_BYTES);
       };
       auto issue_pv = [&](int t, int slot, bool acc) {
         if (leader)
-          issue_pv_tile<D>(tmem + C::o_col(t), tmem + C::s_col(t),
+          issue_pv_tile<D, EB>(tmem + C::o_col(t), tmem + C::s_col(t),
                            kv_addr + slot * C::TILE_BYTES, acc);
       };
 
@@ -475,7 +503,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     float* lsum_x = reinterpret_cast<float*>(smem + C::OFF_LSUM);  // [2][2][2][BM]
     const int bar_id = 1 + t * 4 + qd;  // named barrier of the two warps sharing these rows
     const float sl2 = p.scale_log2;
-    const float2 sl2x2 = make_float2(sl2, sl2);
     uint32_t s_cnt = 0, e_cnt = 0;
     bool ok = true;
 
@@ -491,7 +518,42 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int diag = row + it.koff;  // last visible key under the causal mask
       float m_use = -INFINITY, l = 0.f;
       const int lo_t = t ? it.lo1 : it.lo0;
+      // 8-bit inputs: the scores of tile j are S_acc * q_scale * k_scale[j], so
+      // the log2-domain factor is per tile; V's per-tile scale is folded into P
+      // through the exponent, relative to the item's largest V scale v_ref so
+      // that P stays within the E4M3 range (at most 2^8 with the stale max)
+      float sl2_t = sl2, v_ref = 1.f;
+      const float* ks_row = nullptr;
+      const float* vs_row = nullptr;
+      if constexpr (MODE == MODE_FP8) {
+        if (n_t > 0) {
+          ks_row = p.k_scale + static_cast<size_t>(it.kv_head) * p.n_kt;
+          vs_row = p.v_scale + static_cast<size_t>(it.kv_head) * p.n_kt;
+          const float sq = __ldg(p.q_scale + static_cast<size_t>(it.q_head) * p.n_qt + row0 / BM);
+          bool good = sq > 0.f && sq < INFINITY;
+          float vm = 0.f;
+          for (int jj = lo_t + sm100::lane_id(); jj < n_t; jj += 32) {
+            const float kv = __ldg(ks_row + jj), vv = __ldg(vs_row + jj);
+            good = good && kv > 0.f && kv < INFINITY && vv > 0.f && vv < INFINITY;
+            vm = fmaxf(vm, vv);
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, o));
+          if (!__all_sync(0xffffffffu, good) && sm100::lane_id() == 0)
+            atomicOr(p.status, DEV_BAD_SCALE);
+          sl2_t = sl2 * sq;
+          v_ref = vm;
+        }
+      }
       for (int j = lo_t; j < n_t; ++j) {
+        float sl2j = sl2_t, u_j = 0.f, rv = 1.f;
+        if constexpr (MODE == MODE_FP8) {
+          const float skj = __ldg(ks_row + j), svj = __ldg(vs_row + j);
+          sl2j = sl2_t * skj;
+          rv = v_ref / svj;       // >= 1: P of this tile is stored as p / rv
+          u_j = -sm100::lg2(rv);
+        }
+        const float2 sl2x2 = make_float2(sl2j, sl2j);
         if (!(ok = sm100::mbar_wait(&s_full[t], s_cnt & 1, abort_flag, p.status))) break;
         float* red_w = red + ((s_cnt & 1) * 4 + t * 2) * BM;
         ++s_cnt;
@@ -523,7 +585,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // the row max over all 128 keys: exchange with the warp holding the other half
         red_w[hf * BM + r] = fmaxf(mx0, mx1);
         sm100::named_bar_sync(bar_id, 64);
-        const float m_new = fmaxf(fmaxf(mx0, mx1), red_w[(hf ^ 1) * BM + r]) * sl2;
+        const float m_new = fmaxf(fmaxf(mx0, mx1), red_w[(hf ^ 1) * BM + r]) * sl2j;
         const bool need = m_new > m_use + RESCALE_THRESHOLD;
         if (__any_sync(0xffffffffu, need)) {
           const float m_upd = fmaxf(m_use, m_new);
@@ -545,30 +607,46 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           m_use = m_upd;
         }
         const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
-        const float2 negm = make_float2(-m_sub, -m_sub);
+        const float2 negm = make_float2(u_j - m_sub, u_j - m_sub);
         float2 lsum = make_float2(0.f, 0.f);
-        // exponentials in two 32-column chunks; each chunk's P (packed bf16)
-        // is stored to TMEM while the next chunk is computed
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-#pragma unroll
-          for (int cp = 16 * q; cp < 16 * q + 16; ++cp) {
-            const float2 x = __ffma2_rn(
-                make_float2(__uint_as_float(s[2 * cp]), __uint_as_float(s[2 * cp + 1])), sl2x2,
-                negm);
-            float2 e;
-            if (poly_pair(cp)) {
-              e = sm100::ex2_poly2(x);
-            } else {
-              e.x = sm100::ex2(x.x);
-              e.y = sm100::ex2(x.y);
-            }
-            lsum = __fadd2_rn(lsum, e);
-            s[cp] = sm100::pack_bf16x2(e.x, e.y);
+        auto exp_pair = [&](int cp) -> float2 {
+          const float2 x = __ffma2_rn(
+              make_float2(__uint_as_float(s[2 * cp]), __uint_as_float(s[2 * cp + 1])), sl2x2,
+              negm);
+          float2 e;
+          if (poly_pair(cp)) {
+            e = sm100::ex2_poly2(x);
+          } else {
+            e.x = sm100::ex2(x.x);
+            e.y = sm100::ex2(x.y);
           }
-          sm100::tmem_st16(s_addr + 16 * q, &s[16 * q]);
+          lsum = __fadd2_rn(lsum, e);
+          return e;
+        };
+        // exponentials in two 32-column chunks; each chunk's P is stored to
+        // TMEM while the next chunk is computed
+        if constexpr (EB == 2) {
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+#pragma unroll
+            for (int cp = 16 * q; cp < 16 * q + 16; ++cp) {
+              const float2 e = exp_pair(cp);
+              s[cp] = sm100::pack_bf16x2(e.x, e.y);
+            }
+            sm100::tmem_st16(s_addr + 16 * q, &s[16 * q]);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+#pragma unroll
+            for (int cw = 8 * q; cw < 8 * q + 8; ++cw) {
+              const float2 e0 = exp_pair(2 * cw), e1 = exp_pair(2 * cw + 1);
+              s[cw] = sm100::pack_e4m3x4(e0.x, e0.y, e1.x, e1.y);
+            }
+            sm100::tmem_st8(s_addr + 8 * q, &s[8 * q]);
+          }
         }
-        l += lsum.x + lsum.y;
+        l += (lsum.x + lsum.y) * rv;
         sm100::tmem_st_wait();
         sm100::tc_fence_before();
         __syncwarp();
@@ -586,7 +664,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         l += lx[(hf ^ 1) * BM + r];
       }
       const bool live = row < it.lq;
-      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      const float inv = (l > 0.f) ? v_ref / l : 0.f;  // v_ref: P of 8-bit inputs is relative to it
       __nv_bfloat16* orow;
       if constexpr (MODE == MODE_VARLEN)
         orow = p.O + it.o_off + (live ? row : 0) * it.o_rstride + DH * hf;

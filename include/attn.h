@@ -74,7 +74,7 @@ typedef enum {
 enum { ATTN_MASK_NONE = 0, ATTN_MASK_CAUSAL = 1 };
 
 /* Device status bits (first int32 of every workspace). */
-enum { ATTN_DEV_BAD_KLEN = 1, ATTN_DEV_TIMEOUT = 2, ATTN_DEV_BAD_PAGE = 4 };
+enum { ATTN_DEV_BAD_KLEN = 1, ATTN_DEV_TIMEOUT = 2, ATTN_DEV_BAD_PAGE = 4, ATTN_DEV_BAD_SCALE = 8 };
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* attn_status_string(attn_status_t s);
@@ -96,6 +96,34 @@ attn_status_t attn_fwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf
                        attn_bf16_t* O, float* lse, int B, int Hq, int Hkv, int Lq, int Lk,
                        int d, float scale, int mask_flags, const int32_t* k_lens,
                        void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ 8-bit forward
+ * The forward of attn_fwd on 8-bit inputs: the low-precision execution that the
+ * "FlashAttention" blog (section 10, FlashAttention-3) names, with Q, K and V as
+ * E4M3 floats (OCP 8-bit format: 1 sign, 4 exponent bits with bias 7, 3
+ * mantissa bits, max 448, no infinities) and one fp32 scale per 128-row tile of
+ * each head.  The attention computed is that of the dequantised tensors
+ *   Q[b,h,i,:] = Q8[b,h,i,:] * q_scale[b,h,i/128]   (K and V likewise),
+ * with S = Q K^T on the 8-bit tensor cores (exact products, fp32 sums) and the
+ * probabilities rounded to E4M3 for O += P V; the softmax statistics, O and
+ * LSE are kept in fp32.  Accuracy against exact attention of the dequantised
+ * inputs: the rounding of P (3 mantissa bits) bounds each O element's error
+ * by 2^-4 max|V| and typically gives a relative L2 error of ~2 %; LSE is as
+ * accurate as attn_fwd's.
+ *
+ *   Q8 [B,Hq,Lq,d], K8/V8 [B,Hkv,Lk,d] E4M3 bytes (read only, 16-byte aligned);
+ *   q_scale [B,Hq,ceil(Lq/128)], k_scale/v_scale [B,Hkv,ceil(Lk/128)] fp32
+ *   device arrays (16-byte aligned), each finite and > 0 -- a scale that is
+ *   not sets ATTN_DEV_BAD_SCALE in the status word (results then undefined,
+ *   nothing outside the buffers is touched).
+ *   O, lse, scale, mask_flags, k_lens, workspace: as attn_fwd.
+ *   d must be 128 (else ATTN_ERR_UNSUPPORTED).
+ */
+attn_status_t attn_fwd_fp8(const void* Q8, const void* K8, const void* V8, const float* q_scale,
+                           const float* k_scale, const float* v_scale, attn_bf16_t* O,
+                           float* lse, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale,
+                           int mask_flags, const int32_t* k_lens, void* workspace,
+                           size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------ sliding window
  * Local causal (sliding-window) attention: the causal mask of attn_fwd /
@@ -249,7 +277,8 @@ attn_status_t attn_fwd_splitkv_decode_noalloc(const attn_bf16_t* Q, const attn_b
 /* ------------------------------------------------------------------ status
  * Reads (after synchronising `stream`) the device status word of `workspace`:
  * ATTN_OK when clear, ATTN_ERR_TIMEOUT if any wait expired, ATTN_ERR_INVALID
- * if a k_lens entry was out of range.  *bits (may be NULL) receives the raw
+ * if a k_lens entry, a block-table entry, a sequence offset or an 8-bit scale
+ * was out of range.  *bits (may be NULL) receives the raw
  * ATTN_DEV_* bits.  Returns ATTN_ERR_CUDA if the copy itself fails. */
 attn_status_t attn_read_device_status(const void* workspace, void* stream, int32_t* bits);
 

@@ -126,6 +126,17 @@ def test_sliding_rejects_on_host(lib):
                                 1 << 20, None) == 1
 
 
+def test_fp8_fwd_rejects_on_host(lib):
+    def call(q=P, qs=P, d=128, mask=1, scale=0.1, ws_bytes=256, Lq=8, Hq=2):
+        return lib.attn_fwd_fp8(q, P, P, qs, P, P, P, None, 1, Hq, 1, Lq, 8, d, scale, mask, None,
+                                P, ws_bytes, None)
+    assert call(q=None) == 1 and call(qs=None) == 1 and call(mask=3) == 1
+    assert call(scale=-1.0) == 1 and call(ws_bytes=8) == 1 and call(Hq=0) == 1
+    assert call(qs=ctypes.c_void_p(256 * 1024 + 4)) == 1  # scales must be 16-byte aligned
+    assert call(d=64) == 2 and call(d=96) == 2
+    assert call(Lq=0) == 0
+
+
 def test_product_path_does_not_touch_oracle():
     """The CUDA binding must neither import nor load anything from oracle/."""
     pkg = os.path.join(ROOT, "exact_io_aware_46_b200")
