@@ -391,6 +391,68 @@ def decode_leg(steps, warmup, world, flush):
     return ms, kv_bytes, k_lens, (page, pms)
 
 
+RING = dict(world=4, B=1, Hq=32, Hkv=8, L=16384, d=128)
+
+
+def ring_leg(steps, warmup, world, flush):
+    """Ring attention's decomposition on one GPU: the long-context causal workload
+    B1 Hq32 Hkv8 L16384 d128 split into 4 chunks of 4096; every emulated rank's
+    ring steps (attn_fwd on each visible chunk, attn_merge_partial into the fp32
+    accumulator) run back to back, without the exchange (one GPU).  Also times
+    attn_merge_partial alone on one chunk's rows (HBM-bound)."""
+    import torch
+
+    import exact_io_aware_46_b200 as attn
+    from exact_io_aware_46_b200.ring import fold_chunk, ring_steps
+
+    c = RING
+    W, Lc = c["world"], c["L"] // c["world"]
+    dev = torch.device("cuda")
+    q = synth.normal_bf16_device(synth.workload_seed(3, "q"), (c["B"], c["Hq"], c["L"], c["d"]), dev)
+    k = synth.normal_bf16_device(synth.workload_seed(3, "k"), (c["B"], c["Hkv"], c["L"], c["d"]), dev)
+    v = synth.normal_bf16_device(synth.workload_seed(3, "v"), (c["B"], c["Hkv"], c["L"], c["d"]), dev)
+    qs = [q[:, :, r * Lc:(r + 1) * Lc].contiguous() for r in range(W)]
+    ks = [k[:, :, r * Lc:(r + 1) * Lc].contiguous() for r in range(W)]
+    vs = [v[:, :, r * Lc:(r + 1) * Lc].contiguous() for r in range(W)]
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    # the undivided sequence in one call, for comparison
+    O1 = torch.empty_like(q)
+    whole = lambda: attn.attn_fwd(q, k, v, causal=True, O=O1, workspace=ws)
+    barrier(world)
+    wms = timed_loop(whole, steps, warmup, torch.cuda.current_stream(), flush)
+    del q, k, v, O1
+    acc = [(torch.empty((c["B"], c["Hq"], Lc, c["d"]), dtype=torch.float32, device=dev),
+            torch.empty((c["B"], c["Hq"], Lc), dtype=torch.float32, device=dev),
+            torch.empty((c["B"], c["Hq"], Lc, c["d"]), dtype=torch.bfloat16, device=dev))
+           for _ in range(W)]
+    plans = [ring_steps(r, W, True) for r in range(W)]
+
+    def step():
+        for r in range(W):
+            last = max(s for s, _, kind in plans[r] if kind != "skip")
+            for s, src, kind in plans[r]:
+                fold_chunk(qs[r], ks[src], vs[src], kind, acc[r][0], acc[r][1], first=(s == 0),
+                           O_out=acc[r][2] if s == last else None, workspace=ws)
+
+    barrier(world)
+    ms = timed_loop(step, steps, warmup, torch.cuda.current_stream(), flush)
+    st = attn.attn_read_device_status(ws)
+    if st[0] != attn.ATTN_OK:
+        raise RuntimeError(f"device status {st}")
+    flops = 4.0 * c["d"] * causal_pairs(c["L"], c["L"], True) * c["Hq"] * c["B"]
+    n_fold = sum(1 for p in plans for _, _, kind in p if kind != "skip")
+    # the merge kernel alone: one chunk's rows folded into an accumulator
+    Op = acc[0][2]
+    lp = torch.zeros_like(acc[0][1])
+    merge = lambda: attn.attn_merge_partial(Op, lp, acc[0][0], acc[0][1], init=False)
+    mms = timed_loop(merge, steps, warmup, torch.cuda.current_stream(), flush)
+    rows = Op.numel() // c["d"]
+    mbytes = rows * (4 * c["d"] * 2 + 2 * c["d"] + 12)  # acc read + write, partial, LSEs
+    del qs, ks, vs, acc
+    torch.cuda.empty_cache()
+    return ms, flops, n_fold, mms, mbytes, wms
+
+
 def bwd_leg(steps, warmup, world, flush):
     import torch
 
@@ -502,7 +564,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--legs", default="fwd,decode,bwd",
+    ap.add_argument("--legs", default="fwd,decode,bwd,ring",
                     help="comma list of fwd, decode, bwd (subsets are for profiling runs)")
     ap.add_argument("--decode-lmax", type=int, default=DEC["Lmax"],
                     help="smaller KV cache for profiling captures (k_len ~ U[1024, Lmax])")
@@ -539,6 +601,7 @@ def main():
             bms = bwd_leg(max(3, args.steps // 2), args.warmup, world, flush)
         else:
             bms = None
+        ring = ring_leg(args.steps, args.warmup, world, flush) if "ring" in legs else None
     clocks = clk.summary()
     if "fwd" not in legs:  # profiling runs of single legs: report what ran
         rep = {"legs": legs, "clocks": clocks}
@@ -549,6 +612,10 @@ def main():
         if bms is not None:
             rep["bwd_ms"] = float(np.mean(bms))
             rep["bwd_TFLOPs"] = bwd_flops(BWD) / (float(np.mean(bms)) * 1e-3) / 1e12
+        if ring is not None:
+            rep["ring_ms"] = float(np.mean(ring[0]))
+            rep["ring_TFLOPs"] = ring[1] / (float(np.mean(ring[0])) * 1e-3) / 1e12
+            rep["merge_GBs"] = ring[4] / (float(np.mean(ring[3])) * 1e-3) / 1e9
         if rank == 0:
             print(json.dumps(rep), flush=True)
         return
@@ -558,7 +625,6 @@ def main():
     t_e2e = max_over_ranks(float(np.mean(ms_e2e)), world)
     value = world * flops / (t_step * 1e-3) / 1e12
     achieved = flops / (float(np.mean(ms)) * 1e-3) / 1e12
-    # one persistent forward kernel per step: timed forward, e2e and packed-prefill loops
     # one persistent forward kernel per step: timed forward, e2e, sliding-window, 8-bit and
     # packed-prefill loops
     launches = args.steps + max(3, args.steps // 2) + args.steps + args.steps + args.steps
@@ -650,6 +716,26 @@ def main():
                          "traffic": traffic_per_launch("attn_bwd_impl::bwd_main_kernel")},
         }
         line["gpu_launches"] += 3 * max(3, args.steps // 2)
+    if ring is not None:
+        rms, rflops, n_fold, mms, mbytes, wholems = ring
+        t_r = max_over_ranks(float(np.mean(rms)), world)
+        gbs = mbytes / (float(np.mean(mms)) * 1e-3) / 1e9
+        line["ring"] = {
+            "workload": f"ring attention's decomposition of the causal B1 Hq32 Hkv8 L16384 d128 "
+                        f"forward into {RING['world']} chunks, every rank's steps run on this "
+                        f"GPU (attn_fwd per visible chunk + attn_merge_partial; no exchange: "
+                        f"one GPU)",
+            "value": world * rflops / (t_r * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": t_r, "flops_per_step": rflops, "chunk_folds_per_step": n_fold,
+            "undivided_ms": float(np.mean(wholems)),
+            "undivided_TFLOPs": rflops / (float(np.mean(wholems)) * 1e-3) / 1e12,
+            "merge": {"kernel": "attn_merge_impl::merge_kernel", "rows": RING["B"] * RING["Hq"]
+                      * (RING["L"] // RING["world"]), "ms": float(np.mean(mms)),
+                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"],
+                                   "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                                   "traffic": None}},
+        }
+        line["gpu_launches"] += 2 * n_fold * args.steps + 2 * args.steps
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:

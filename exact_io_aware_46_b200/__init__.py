@@ -54,6 +54,7 @@ SIGNATURES = {
                       _vp]),
     "attn_fwd_sliding": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _vp,
                               _sz, _vp]),
+    "attn_merge_partial": (_i, [_vp, _vp, _vp, _vp, _vp, ctypes.c_longlong, _i, _i, _vp]),
     "attn_fwd_fp8": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i,
                           _vp, _vp, _sz, _vp]),
     "attn_bwd_sliding": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
@@ -228,6 +229,25 @@ def attn_fwd_fp8(Q8, K8, V8, q_scale, k_scale, v_scale, scale=None, causal=False
                               _ptr(k_lens), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(code, "attn_fwd_fp8")
     return O, lse
+
+
+def attn_merge_partial(O_part, lse_part, O_acc, lse_acc, init, O_out=None, stream=None):
+    """Fold a partial result (O_part bf16 [..., d], lse_part fp32 [...]) into the
+    fp32 accumulator (O_acc, lse_acc) in place (``init``: overwrite it instead);
+    ``O_out`` (bf16, optional) also receives the merged O."""
+    _bf16(O_part, "O_part")
+    for t, n in ((lse_part, "lse_part"), (O_acc, "O_acc"), (lse_acc, "lse_acc")):
+        _f32(t, n)
+    if O_out is not None:
+        _bf16(O_out, "O_out")
+    d = O_part.shape[-1]
+    rows = O_part.numel() // d if d else 0
+    if O_acc.shape != O_part.shape or lse_part.numel() != rows or lse_acc.numel() != rows or \
+            (O_out is not None and O_out.shape != O_part.shape):
+        raise ValueError("partial, accumulator and output shapes differ")
+    code = lib().attn_merge_partial(_ptr(O_part), _ptr(lse_part), _ptr(O_acc), _ptr(lse_acc),
+                                    _ptr(O_out), rows, d, 1 if init else 0, _stream(stream))
+    _check(code, "attn_merge_partial")
 
 
 def attn_fwd_sliding(Q, K, V, window, scale=None, k_lens=None, O=None, lse=None, workspace=None,

@@ -14,6 +14,7 @@
 #include "bwd_kernel.cuh"
 #include "decode_kernel.cuh"
 #include "fwd_kernel.cuh"
+#include "merge_kernel.cuh"
 
 namespace {
 
@@ -303,6 +304,39 @@ attn_status_t attn_fwd_varlen(const attn_bf16_t* Q, const attn_bf16_t* K, const 
   p.total_q = total_q;
   p.total_k = total_k;
   return launch_fwd(tq, tk, tv, p, O, lse, B, Hq, Hkv, d, scale, mask_flags, workspace, stream);
+}
+
+// ------------------------------------------------------------------ merge of partials
+
+attn_status_t attn_merge_partial(const attn_bf16_t* O_part, const float* lse_part, float* O_acc,
+                                 float* lse_acc, attn_bf16_t* O_out, long long rows, int d,
+                                 int init, void* stream) {
+  if (rows < 0 || !(d == 8 || d == 16 || d == 32 || d == 64 || d == 128 || d == 256))
+    return ATTN_ERR_INVALID;
+  if (init != 0 && init != 1) return ATTN_ERR_INVALID;
+  if (!O_part || !lse_part || !O_acc || !lse_acc) return ATTN_ERR_INVALID;
+  if (!aligned16(O_part) || !aligned16(O_acc) || (O_out && !aligned16(O_out)) ||
+      !aligned16(lse_part) || !aligned16(lse_acc))
+    return ATTN_ERR_INVALID;
+  if (rows == 0) return ATTN_OK;
+  const int sms = device_sms();
+  if (sms <= 0) return ATTN_ERR_CUDA;
+  attn_merge_impl::Params p;
+  p.O_part = reinterpret_cast<const __nv_bfloat16*>(O_part);
+  p.lse_part = lse_part;
+  p.O_acc = O_acc;
+  p.lse_acc = lse_acc;
+  p.O_out = reinterpret_cast<__nv_bfloat16*>(O_out);
+  p.rows = rows;
+  p.d = d;
+  p.init = init;
+  const long long rpb = attn_merge_impl::NTHREADS / (d / 8);
+  const long long need = (rows + rpb - 1) / rpb;
+  const long long cap = static_cast<long long>(sms) * 8;  // 8 resident blocks per SM
+  const int grid = static_cast<int>(need < cap ? need : cap);
+  attn_merge_impl::merge_kernel<<<grid, attn_merge_impl::NTHREADS, 0,
+                                  reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------ decode

@@ -1,0 +1,121 @@
+"""Ring attention: the forward over a sequence split across the ranks of a
+process group (context parallelism, the third ledger of "FlashAttention and
+long context: separate the three ledgers", where RingAttention passes K/V
+blocks around the devices and computes blockwise attention).
+
+Rank r holds one contiguous chunk of the sequence: its query rows and its
+keys/values, all chunks of equal length.  In ``world`` steps every K/V chunk
+visits every rank: at step s rank r holds the chunk of rank (r - s) mod world,
+computes the partial attention of its queries against it with ``attn_fwd``
+(on the GPU kernels) and folds the partial into an fp32 accumulator with
+``attn_merge_partial`` (the normalised merge rule in LSE form).  While a step
+computes, the next chunk is already in flight: each rank sends the chunk it
+holds to rank r + 1 and receives the next from rank r - 1 with point-to-point
+operations of ``torch.distributed`` (NCCL between GPUs over NVLink; gloo on
+CPU), into a second buffer.  Under the causal mask a chunk from a later rank is
+entirely masked and skipped (its exchange still runs, so every rank takes the
+same collective steps in the same order), the diagonal chunk is causal and the
+earlier chunks are fully visible.
+
+The exchange moves K/V between ranks and the kernels compute; there is no
+compute on the host and no fallback: ``ring_attn_fwd`` needs the CUDA library.
+"""
+
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+FULL, CAUSAL, SKIP = "full", "causal", "skip"
+
+
+def ring_steps(rank: int, world: int, causal: bool):
+    """The schedule of one rank: a list of (step, source rank, kind), where
+    kind is FULL (every key of the chunk visible), CAUSAL (the rank's own
+    chunk, the causal mask inside it) or SKIP (every key masked)."""
+    if not 0 <= rank < world:
+        raise ValueError("rank out of range")
+    out = []
+    for s in range(world):
+        src = (rank - s) % world
+        if not causal or src < rank:
+            kind = FULL
+        elif src == rank:
+            kind = CAUSAL
+        else:
+            kind = SKIP
+        out.append((s, src, kind))
+    return out
+
+
+class RingExchange:
+    """Double-buffered ring pass of a tuple of tensors: ``start()`` posts the
+    send of the held tensors to rank + 1 and the receive of the next ones from
+    rank - 1; ``finish()`` waits for both and makes the received tensors the
+    held ones.  Works on any backend with point-to-point operations."""
+
+    def __init__(self, tensors, group=None):
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.cur = [t.contiguous() for t in tensors]
+        self.nxt = [torch.empty_like(t) for t in self.cur]
+        self.reqs = None
+
+    def _peer(self, r):
+        return dist.get_global_rank(self.group, r) if self.group is not None else r
+
+    def start(self):
+        if self.reqs is not None:
+            raise RuntimeError("a ring step is already in flight")
+        to = self._peer((self.rank + 1) % self.world)
+        frm = self._peer((self.rank - 1) % self.world)
+        ops = [dist.P2POp(dist.isend, t, to, self.group) for t in self.cur]
+        ops += [dist.P2POp(dist.irecv, t, frm, self.group) for t in self.nxt]
+        self.reqs = dist.batch_isend_irecv(ops)
+
+    def finish(self):
+        for r in self.reqs:
+            r.wait()
+        self.reqs = None
+        self.cur, self.nxt = self.nxt, self.cur
+
+
+def fold_chunk(q, kc, vc, kind, O_acc, lse_acc, first, O_out=None, scale=None, workspace=None):
+    """One ring step's compute: the partial attention of q against the K/V chunk
+    (kc, vc) held at this step (kind FULL or CAUSAL), folded into the fp32
+    accumulator (O_acc, lse_acc); ``first`` initialises it, ``O_out`` (bf16)
+    receives the merged O at the last step."""
+    from . import attn_fwd, attn_merge_partial
+
+    if kind == SKIP:
+        return
+    Op, lp = attn_fwd(q, kc, vc, scale=scale, causal=(kind == CAUSAL), workspace=workspace)
+    attn_merge_partial(Op, lp, O_acc, lse_acc, init=first, O_out=O_out)
+
+
+def ring_attn_fwd(q, k, v, group=None, causal=True, scale=None):
+    """Ring-attention forward.  q [B, Hq, Lc, d], k/v [B, Hkv, Lc, d] bf16 CUDA
+    tensors: this rank's chunk (rows [rank * Lc, (rank + 1) * Lc) of the whole
+    sequence); every rank passes the same shapes.  Returns this rank's
+    (O bf16 [B, Hq, Lc, d], LSE fp32 [B, Hq, Lc]) of attention over the whole
+    sequence."""
+    if not q.is_cuda:
+        raise ValueError("ring_attn_fwd runs on the CUDA kernels")
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    steps = ring_steps(rank, world, causal)
+    last = max(s for s, _, kind in steps if kind != SKIP)
+    O_acc = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    lse_acc = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    O = torch.empty_like(q)
+    ex = RingExchange((k, v), group)
+    for s, _, kind in steps:
+        if s + 1 < world:
+            ex.start()
+        kc, vc = ex.cur
+        fold_chunk(q, kc, vc, kind, O_acc, lse_acc, first=(s == 0),
+                   O_out=O if s == last else None, scale=scale)
+        if s + 1 < world:
+            ex.finish()
+    return O, lse_acc

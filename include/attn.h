@@ -125,6 +125,26 @@ attn_status_t attn_fwd_fp8(const void* Q8, const void* K8, const void* V8, const
                            int mask_flags, const int32_t* k_lens, void* workspace,
                            size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------ merge of partial results
+ * Combines partial attention results of the same query rows over disjoint key
+ * sets with the normalised merge rule of the FlashAttention-2 tutorial (2.1.3),
+ * in LSE form:  LSE = ln(e^{LSE_a} + e^{LSE_b}),
+ *               O = e^{LSE_a - LSE} O_a + e^{LSE_b - LSE} O_b.
+ * Used by ring (context-parallel) attention to fold in one key chunk per step.
+ *
+ *   O_part [rows, d] bf16 and lse_part [rows] fp32 (natural log, as attn_fwd
+ *   writes them; -inf = no visible key): the partial to fold in (read only).
+ *   O_acc [rows, d] fp32 and lse_acc [rows] fp32: the accumulator (in/out);
+ *   init = 1 overwrites it with the partial, init = 0 merges into it.
+ *   O_out [rows, d] bf16 or NULL: also receives the merged O (last step).
+ *   rows >= 0 (any [B, H, L] flattened); d in {8, 16, 32, 64, 128, 256}.
+ *   All pointers 16-byte aligned, else ATTN_ERR_INVALID.  Rows whose two LSEs
+ *   are both -inf become O = 0, LSE = -inf.
+ */
+attn_status_t attn_merge_partial(const attn_bf16_t* O_part, const float* lse_part, float* O_acc,
+                                 float* lse_acc, attn_bf16_t* O_out, long long rows, int d,
+                                 int init, void* stream);
+
 /* ------------------------------------------------------------------ sliding window
  * Local causal (sliding-window) attention: the causal mask of attn_fwd /
  * attn_bwd plus a lower edge, so query row i sees only keys j with

@@ -1,0 +1,117 @@
+"""Ring attention host logic without a GPU: the step schedule (closed forms,
+and composed on the fp64 oracle it gives exact attention over the whole
+sequence) and the double-buffered K/V ring pass on 2 and 3 gloo ranks."""
+
+import os
+import socket
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from exact_io_aware_46_b200.ring import CAUSAL, FULL, SKIP, RingExchange, ring_steps
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 5])
+@pytest.mark.parametrize("causal", [False, True])
+def test_schedule_visits_every_chunk_once(world, causal):
+    for rank in range(world):
+        st = ring_steps(rank, world, causal)
+        assert [s for s, _, _ in st] == list(range(world))
+        assert sorted(src for _, src, _ in st) == list(range(world))
+        assert st[0][1] == rank  # a rank starts on its own chunk
+        for s, src, kind in st:
+            assert src == (rank - s) % world
+            if not causal:
+                assert kind == FULL
+            else:
+                assert kind == (CAUSAL if src == rank else FULL if src < rank else SKIP)
+
+
+def test_schedule_causal_closed_forms():
+    assert [k for _, _, k in ring_steps(0, 4, True)] == [CAUSAL, SKIP, SKIP, SKIP]
+    assert [k for _, _, k in ring_steps(3, 4, True)] == [CAUSAL, FULL, FULL, FULL]
+    assert [k for _, _, k in ring_steps(1, 4, True)] == [CAUSAL, FULL, SKIP, SKIP]
+    with pytest.raises(ValueError):
+        ring_steps(4, 4, True)
+
+
+@pytest.mark.parametrize("world,causal", [(3, True), (3, False), (4, True)])
+def test_schedule_composes_exact_attention_on_the_oracle(world, causal):
+    """Each rank's chunk partials (oracle forward per step kind), merged with
+    the oracle's normalised merge rule in step order, equal the oracle's
+    attention over the whole sequence for that rank's rows."""
+    Lc, d = 37, 8
+    L = world * Lc
+    Q = synth.bf16_bits_to_f64(synth.normal_bf16(611, (1, 2, L, d)))
+    K = synth.bf16_bits_to_f64(synth.normal_bf16(612, (1, 1, L, d)))
+    V = synth.bf16_bits_to_f64(synth.normal_bf16(613, (1, 1, L, d)))
+    Oref, Lref = oracle.fwd(Q, K, V, 0.3, causal=causal)
+    for rank in range(world):
+        q = Q[:, :, rank * Lc:(rank + 1) * Lc]
+        acc = None
+        for _, src, kind in ring_steps(rank, world, causal):
+            if kind == SKIP:
+                continue
+            kc = K[:, :, src * Lc:(src + 1) * Lc]
+            vc = V[:, :, src * Lc:(src + 1) * Lc]
+            Op, lp = oracle.fwd(q, kc, vc, 0.3, causal=(kind == CAUSAL))
+            if acc is None:
+                acc = [Op.copy(), lp.copy()]
+                continue
+            for h in range(2):
+                for i in range(Lc):
+                    m, l, o = oracle.merge(acc[1][0, h, i], 1.0, acc[0][0, h, i],
+                                           lp[0, h, i], 1.0, Op[0, h, i])
+                    acc[0][0, h, i] = o
+                    acc[1][0, h, i] = m + np.log(l)
+        rows = slice(rank * Lc, (rank + 1) * Lc)
+        assert np.max(np.abs(acc[0] - Oref[:, :, rows])) <= 1e-12
+        assert np.max(np.abs(acc[1] - Lref[:, :, rows])) <= 1e-12
+
+
+def _exchange_main(rank, world, port, out):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    k = torch.full((3, 5), float(rank))
+    v = torch.full((2, 7), 10.0 * rank)
+    ex = RingExchange((k, v))
+    seen = []
+    for s in range(world):
+        if s + 1 < world:
+            ex.start()
+        seen.append((float(ex.cur[0][0, 0]), float(ex.cur[1][1, 6])))
+        if s + 1 < world:
+            ex.finish()
+    dist.barrier()
+    dist.destroy_process_group()
+    with open(out + f".{rank}", "w") as f:
+        f.write(repr(seen))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_ring_exchange_on_gloo_ranks(tmp_path, world):
+    """At step s every rank holds the chunk of rank (rank - s) mod world."""
+    import torch.multiprocessing as mp
+
+    out = str(tmp_path / "x")
+    mp.start_processes(_exchange_main, args=(world, _free_port(), out), nprocs=world,
+                       join=True, start_method="spawn")
+    for rank in range(world):
+        seen = eval(open(out + f".{rank}").read())
+        assert seen == [(float((rank - s) % world), 10.0 * ((rank - s) % world))
+                        for s in range(world)]
