@@ -408,9 +408,10 @@ RING = dict(world=4, B=1, Hq=32, Hkv=8, L=16384, d=128)
 def ring_leg(steps, warmup, world, flush):
     """Ring attention's decomposition on one GPU: the long-context causal workload
     B1 Hq32 Hkv8 L16384 d128 split into 4 chunks of 4096; every emulated rank's
-    ring steps (attn_fwd on each visible chunk, attn_merge_partial into the fp32
-    accumulator) run back to back, without the exchange (one GPU).  Also times
-    attn_merge_partial alone on one chunk's rows (HBM-bound)."""
+    ring steps (attn_fwd_merge on each visible chunk: the forward with the fold
+    into the fp32 accumulator in its epilogue) run back to back, without the
+    exchange (one GPU).  Also times the stand-alone attn_merge_partial on one
+    chunk's rows (HBM-bound)."""
     import torch
 
     import exact_io_aware_46_b200 as attn
@@ -735,7 +736,7 @@ def main():
         line["ring"] = {
             "workload": f"ring attention's decomposition of the causal B1 Hq32 Hkv8 L16384 d128 "
                         f"forward into {RING['world']} chunks, every rank's steps run on this "
-                        f"GPU (attn_fwd per visible chunk + attn_merge_partial; no exchange: "
+                        f"GPU (one attn_fwd_merge per visible chunk; no exchange: "
                         f"one GPU)",
             "value": world * rflops / (t_r * 1e-3) / 1e12, "unit": "TFLOP/s",
             "ms_per_step": t_r, "flops_per_step": rflops, "chunk_folds_per_step": n_fold,
@@ -745,9 +746,9 @@ def main():
                       * (RING["L"] // RING["world"]), "ms": float(np.mean(mms)),
                       "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"],
                                    "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
-                                   "traffic": None}},
+                                   "traffic": traffic_per_launch("attn_merge_impl::merge_kernel")}},
         }
-        line["gpu_launches"] += 2 * n_fold * args.steps + 2 * args.steps
+        line["gpu_launches"] += n_fold * args.steps + 2 * args.steps
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:

@@ -54,6 +54,8 @@ SIGNATURES = {
                       _vp]),
     "attn_fwd_sliding": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _vp,
                               _sz, _vp]),
+    "attn_fwd_merge": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp,
+                            _vp, _sz, _vp]),
     "attn_merge_partial": (_i, [_vp, _vp, _vp, _vp, _vp, ctypes.c_longlong, _i, _i, _vp]),
     "attn_fwd_fp8": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i,
                           _vp, _vp, _sz, _vp]),
@@ -229,6 +231,34 @@ def attn_fwd_fp8(Q8, K8, V8, q_scale, k_scale, v_scale, scale=None, causal=False
                               _ptr(k_lens), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(code, "attn_fwd_fp8")
     return O, lse
+
+
+def attn_fwd_merge(Q, K, V, O_acc, lse_acc, init, O_out=None, scale=None, causal=False,
+                   k_lens=None, workspace=None, stream=None):
+    """attn_fwd over K/V (a subset of the keys), folded into the fp32 accumulator
+    (O_acc [B,Hq,Lq,d], lse_acc [B,Hq,Lq]) in place with the normalised merge
+    rule (``init``: overwrite it instead); ``O_out`` (bf16, optional) receives
+    the merged O."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _bf16(t, n)
+    for t, n in ((O_acc, "O_acc"), (lse_acc, "lse_acc")):
+        _f32(t, n)
+    B, Hq, Lq, d = Q.shape
+    Hkv, Lk = K.shape[1], K.shape[2]
+    if tuple(O_acc.shape) != (B, Hq, Lq, d) or tuple(lse_acc.shape) != (B, Hq, Lq) or \
+            (O_out is not None and tuple(O_out.shape) != (B, Hq, Lq, d)):
+        raise ValueError("accumulator shapes must match Q")
+    if O_out is not None:
+        _bf16(O_out, "O_out")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if workspace is None:
+        workspace = _workspace(attn_fwd_workspace_size(B, Hq, Hkv, Lq, Lk, d), Q.device, stream)
+    code = lib().attn_fwd_merge(_ptr(Q), _ptr(K), _ptr(V), _ptr(O_acc), _ptr(lse_acc),
+                                _ptr(O_out), 1 if init else 0, B, Hq, Hkv, Lq, Lk, d,
+                                float(scale), ATTN_MASK_CAUSAL if causal else ATTN_MASK_NONE,
+                                _ptr(k_lens), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(code, "attn_fwd_merge")
 
 
 def attn_merge_partial(O_part, lse_part, O_acc, lse_acc, init, O_out=None, stream=None):

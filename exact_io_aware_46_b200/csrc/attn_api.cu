@@ -143,6 +143,7 @@ static attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, co
   const int grid = n_items < sms ? n_items : sms;
   const int mode = p.cu_q      ? attn_fwd_impl::MODE_VARLEN
                    : p.q_scale ? attn_fwd_impl::MODE_FP8
+                   : p.o_acc   ? attn_fwd_impl::MODE_MERGE
                    : p.window > 0 ? attn_fwd_impl::MODE_WINDOW
                                   : attn_fwd_impl::MODE_PLAIN;
   cudaError_t e = cudaSuccess;
@@ -156,12 +157,14 @@ static attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, co
     if (mode == MODE_PLAIN) run(fwd_kernel<128, MODE_PLAIN>, smem);
     else if (mode == MODE_WINDOW) run(fwd_kernel<128, MODE_WINDOW>, smem);
     else if (mode == MODE_FP8) run(fwd_kernel<128, MODE_FP8>, Cfg<128, 1>::SMEM_BYTES);
+    else if (mode == MODE_MERGE) run(fwd_kernel<128, MODE_MERGE>, smem);
     else run(fwd_kernel<128, MODE_VARLEN>, smem);
   } else {
     if (mode == MODE_FP8) return ATTN_ERR_UNSUPPORTED;
     constexpr int smem = Cfg<64>::SMEM_BYTES;
     if (mode == MODE_PLAIN) run(fwd_kernel<64, MODE_PLAIN>, smem);
     else if (mode == MODE_WINDOW) run(fwd_kernel<64, MODE_WINDOW>, smem);
+    else if (mode == MODE_MERGE) run(fwd_kernel<64, MODE_MERGE>, smem);
     else run(fwd_kernel<64, MODE_VARLEN>, smem);
   }
   if (e != cudaSuccess) return ATTN_ERR_CUDA;
@@ -266,6 +269,38 @@ attn_status_t attn_fwd_fp8(const void* Q8, const void* K8, const void* V8, const
   p.n_qt = (Lq + attn_fwd_impl::BM - 1) / attn_fwd_impl::BM;
   p.n_kt = (Lk + attn_fwd_impl::BN - 1) / attn_fwd_impl::BN;
   return launch_fwd(tq, tk, tv, p, O, lse, B, Hq, Hkv, d, scale, mask_flags, workspace, stream);
+}
+
+attn_status_t attn_fwd_merge(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf16_t* V,
+                             float* O_acc, float* lse_acc, attn_bf16_t* O_out, int init, int B,
+                             int Hq, int Hkv, int Lq, int Lk, int d, float scale, int mask_flags,
+                             const int32_t* k_lens, void* workspace, size_t ws_bytes,
+                             void* stream) {
+  if (!shapes_ok(B, Hq, Hkv, Lq, Lk)) return ATTN_ERR_INVALID;
+  if (!Q || !K || !V || !O_acc || !lse_acc || !workspace) return ATTN_ERR_INVALID;
+  if (init != 0 && init != 1) return ATTN_ERR_INVALID;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O_acc) ||
+      !aligned16(lse_acc) || (O_out && !aligned16(O_out)) || (k_lens && !aligned16(k_lens)) ||
+      !aligned256(workspace))
+    return ATTN_ERR_INVALID;
+  if (!(std::isfinite(scale) && scale > 0.f)) return ATTN_ERR_INVALID;
+  if (mask_flags != ATTN_MASK_NONE && mask_flags != ATTN_MASK_CAUSAL) return ATTN_ERR_INVALID;
+  if (ws_bytes < attn_fwd_workspace_size(B, Hq, Hkv, Lq, Lk, d)) return ATTN_ERR_INVALID;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (Lq == 0) return ATTN_OK;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, Q, d, Lq, static_cast<long long>(B) * Hq, 128) ||
+      !make_tmap(&tk, K, d, Lk, static_cast<long long>(B) * Hkv, 128) ||
+      !make_tmap(&tv, V, d, Lk, static_cast<long long>(B) * Hkv, 128))
+    return ATTN_ERR_CUDA;
+  attn_fwd_impl::Params p{};
+  p.k_lens = k_lens;
+  p.Lq = Lq;
+  p.Lk = Lk;
+  p.o_acc = O_acc;
+  p.merge_init = init;
+  return launch_fwd(tq, tk, tv, p, O_out, lse_acc, B, Hq, Hkv, d, scale, mask_flags, workspace,
+                    stream);
 }
 
 size_t attn_fwd_varlen_workspace_size(int, int, int, int, int, int) { return kStatusBytes; }

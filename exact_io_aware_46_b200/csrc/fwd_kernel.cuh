@@ -96,6 +96,10 @@ struct Params {
   const float* k_scale;  // [B * Hkv][n_kt]
   const float* v_scale;  // [B * Hkv][n_kt]
   int n_qt, n_kt;
+  // folding into an accumulator (ring attention): o_acc [B, Hq, Lq, D] fp32 and
+  // lse [B, Hq, Lq] (in/out); O (bf16, may be nullptr) receives the merged O.
+  float* o_acc;
+  int merge_init;  // 1: the accumulator is overwritten instead of merged into
 };
 
 struct Item {
@@ -120,8 +124,9 @@ struct Item {
 //   MODE_PLAIN   [B, H, L, d] tensors, optional causal mask and key padding;
 //   MODE_WINDOW  the same with a sliding-window causal mask (p.window keys);
 //   MODE_VARLEN  packed sequences [T, H, d] with cu_seqlens offsets;
-//   MODE_FP8     the plain layout with E4M3 Q, K, V and per-tile scales.
-enum : int { MODE_PLAIN = 0, MODE_WINDOW = 1, MODE_VARLEN = 2, MODE_FP8 = 3 };
+//   MODE_FP8     the plain layout with E4M3 Q, K, V and per-tile scales;
+//   MODE_MERGE   the plain layout, the result folded into an fp32 accumulator.
+enum : int { MODE_PLAIN = 0, MODE_WINDOW = 1, MODE_VARLEN = 2, MODE_FP8 = 3, MODE_MERGE = 4 };
 
 constexpr int DEV_BAD_SCALE = 8;  // device status bit: a scale that is not finite and > 0
 
@@ -656,6 +661,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // ---------------- epilogue: O = o / l (bf16), LSE = ln(2) * (m + log2 l)
       if (!(ok = sm100::mbar_wait(&o_full[t], k & 1, abort_flag, p.status))) break;
       sm100::tc_fence_after();
+      const bool live = row < it.lq;
+      // folding: both warps of a row read the accumulator's LSE before the
+      // row-sum exchange below, which orders the write of the new LSE after it
+      float lse_a = -INFINITY;
+      const size_t rix = (static_cast<size_t>(it.b) * p.Hq + it.h) * p.Lq + (live ? row : 0);
+      if constexpr (MODE == MODE_MERGE)
+        if (live && !p.merge_init) lse_a = p.lse[rix];
       if (n_t > 0) {
         float* lx = lsum_x + ((e_cnt & 1) * 4 + t * 2) * BM;
         ++e_cnt;
@@ -663,8 +675,64 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         sm100::named_bar_sync(bar_id, 64);
         l += lx[(hf ^ 1) * BM + r];
       }
-      const bool live = row < it.lq;
       const float inv = (l > 0.f) ? v_ref / l : 0.f;  // v_ref: P of 8-bit inputs is relative to it
+      if constexpr (MODE == MODE_MERGE) {
+        // normalised merge rule in LSE form with (O_a, LSE_a) = the accumulator and
+        // (O_b, LSE_b) = this result: LSE = ln(e^LSE_a + e^LSE_b),
+        // O = e^(LSE_a - LSE) O_a + e^(LSE_b - LSE) O_b, with O_b = o / l
+        const float lse_b = (l > 0.f) ? (m_use + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        const float mx = fmaxf(lse_a, lse_b);
+        float wa = 0.f, wb = 0.f, lse_new = -INFINITY;
+        if (mx != -INFINITY) {
+          wa = (lse_a == -INFINITY) ? 0.f : expf(lse_a - mx);
+          wb = (lse_b == -INFINITY) ? 0.f : expf(lse_b - mx);
+          const float ws = wa + wb;
+          lse_new = mx + logf(ws);
+          wa /= ws;
+          wb = wb / ws * inv;
+        }
+        float* arow = p.o_acc + rix * D + DH * hf;
+        __nv_bfloat16* orow = p.O ? p.O + rix * D + DH * hf : nullptr;
+#pragma unroll 1
+        for (int c = 0; c < DH / 16; ++c) {
+          uint32_t o[16];
+          if (n_t > 0) {  // warp-uniform: the TMEM load is collective
+            sm100::tmem_ld16(o_addr + c * 16, o);
+            sm100::tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = 0u;
+          }
+          if (live) {
+            float4* a4 = reinterpret_cast<float4*>(arow + c * 16);
+            float res[16];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const float4 a = (wa != 0.f) ? a4[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+              res[4 * v] = wa * a.x + wb * __uint_as_float(o[4 * v]);
+              res[4 * v + 1] = wa * a.y + wb * __uint_as_float(o[4 * v + 1]);
+              res[4 * v + 2] = wa * a.z + wb * __uint_as_float(o[4 * v + 2]);
+              res[4 * v + 3] = wa * a.w + wb * __uint_as_float(o[4 * v + 3]);
+            }
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              a4[v] = make_float4(res[4 * v], res[4 * v + 1], res[4 * v + 2], res[4 * v + 3]);
+            if (orow) {
+              uint32_t pk[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) pk[e] = sm100::pack_bf16x2(res[2 * e], res[2 * e + 1]);
+              uint4* dst = reinterpret_cast<uint4*>(orow + c * 16);
+              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+          }
+        }
+        if (live && hf == 0) p.lse[rix] = lse_new;
+        sm100::tc_fence_before();
+        __syncwarp();
+        if (sm100::lane_id() == 0) sm100::mbar_arrive(&o_empty[t]);
+        continue;
+      }
       __nv_bfloat16* orow;
       if constexpr (MODE == MODE_VARLEN)
         orow = p.O + it.o_off + (live ? row : 0) * it.o_rstride + DH * hf;

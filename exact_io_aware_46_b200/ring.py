@@ -7,8 +7,9 @@ Rank r holds one contiguous chunk of the sequence: its query rows and its
 keys/values, all chunks of equal length.  In ``world`` steps every K/V chunk
 visits every rank: at step s rank r holds the chunk of rank (r - s) mod world,
 computes the partial attention of its queries against it with ``attn_fwd``
-(on the GPU kernels) and folds the partial into an fp32 accumulator with
-``attn_merge_partial`` (the normalised merge rule in LSE form).  While a step
+(on the GPU kernels) and folds the partial into an fp32 accumulator with the
+normalised merge rule in LSE form -- in the forward kernel's epilogue
+(``attn_fwd_merge``), so a step is one kernel launch.  While a step
 computes, the next chunk is already in flight: each rank sends the chunk it
 holds to rank r + 1 and receives the next from rank r - 1 with point-to-point
 operations of ``torch.distributed`` (NCCL between GPUs over NVLink; gloo on
@@ -84,14 +85,14 @@ class RingExchange:
 def fold_chunk(q, kc, vc, kind, O_acc, lse_acc, first, O_out=None, scale=None, workspace=None):
     """One ring step's compute: the partial attention of q against the K/V chunk
     (kc, vc) held at this step (kind FULL or CAUSAL), folded into the fp32
-    accumulator (O_acc, lse_acc); ``first`` initialises it, ``O_out`` (bf16)
-    receives the merged O at the last step."""
-    from . import attn_fwd, attn_merge_partial
+    accumulator (O_acc, lse_acc) by the forward kernel itself; ``first``
+    initialises it, ``O_out`` (bf16) receives the merged O at the last step."""
+    from . import attn_fwd_merge
 
     if kind == SKIP:
         return
-    Op, lp = attn_fwd(q, kc, vc, scale=scale, causal=(kind == CAUSAL), workspace=workspace)
-    attn_merge_partial(Op, lp, O_acc, lse_acc, init=first, O_out=O_out)
+    attn_fwd_merge(q, kc, vc, O_acc, lse_acc, init=first, O_out=O_out, scale=scale,
+                   causal=(kind == CAUSAL), workspace=workspace)
 
 
 def ring_attn_fwd(q, k, v, group=None, causal=True, scale=None):

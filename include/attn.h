@@ -145,6 +145,19 @@ attn_status_t attn_merge_partial(const attn_bf16_t* O_part, const float* lse_par
                                  float* lse_acc, attn_bf16_t* O_out, long long rows, int d,
                                  int init, void* stream);
 
+/* The same fold done by the forward kernel itself: attn_fwd of Q against K/V
+ * (one chunk of the keys), merged into the accumulator in the kernel's
+ * epilogue instead of being written out as a bf16 partial -- one launch per
+ * ring step.  Q, K, V, B, Hq, Hkv, Lq, Lk, d, scale, mask_flags, k_lens,
+ * workspace: as attn_fwd (d = 64 or 128).  O_acc [B,Hq,Lq,d] fp32 and lse_acc
+ * [B,Hq,Lq] fp32: the accumulator (in/out; init = 1 overwrites it); O_out
+ * [B,Hq,Lq,d] bf16 or NULL receives the merged O. */
+attn_status_t attn_fwd_merge(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf16_t* V,
+                             float* O_acc, float* lse_acc, attn_bf16_t* O_out, int init, int B,
+                             int Hq, int Hkv, int Lq, int Lk, int d, float scale, int mask_flags,
+                             const int32_t* k_lens, void* workspace, size_t ws_bytes,
+                             void* stream);
+
 /* ------------------------------------------------------------------ sliding window
  * Local causal (sliding-window) attention: the causal mask of attn_fwd /
  * attn_bwd plus a lower edge, so query row i sees only keys j with

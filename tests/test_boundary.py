@@ -137,6 +137,20 @@ def test_fp8_fwd_rejects_on_host(lib):
     assert call(Lq=0) == 0
 
 
+def test_fwd_merge_and_merge_partial_reject_on_host(lib):
+    def fm(acc=P, lse=P, init=1, d=128, mask=0, ws_bytes=256):
+        return lib.attn_fwd_merge(P, P, P, acc, lse, None, init, 1, 2, 1, 8, 8, d, 0.1, mask,
+                                  None, P, ws_bytes, None)
+    assert fm(acc=None) == 1 and fm(lse=None) == 1 and fm(init=2) == 1 and fm(mask=4) == 1
+    assert fm(ws_bytes=8) == 1 and fm(acc=ctypes.c_void_p(256 * 1024 + 4)) == 1
+    assert fm(d=96) == 2
+
+    def mp(d=128, rows=10, init=0, part=P):
+        return lib.attn_merge_partial(part, P, P, P, None, rows, d, init, None)
+    assert mp(d=96) == 1 and mp(d=512) == 1 and mp(rows=-1) == 1 and mp(init=3) == 1
+    assert mp(part=None) == 1 and mp(rows=0) == 0
+
+
 def test_product_path_does_not_touch_oracle():
     """The CUDA binding must neither import nor load anything from oracle/."""
     pkg = os.path.join(ROOT, "exact_io_aware_46_b200")

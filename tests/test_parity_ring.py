@@ -104,3 +104,39 @@ def test_ring_decomposition_matches_whole_sequence(world, causal, Hq, Hkv, Lc, d
         torch.cuda.synchronize()
         assert_out_close(to_f64(O), Oref[:, :, rows], f"O[rank {rank}]")
         assert_lse_close(to_f64(lse_acc), Lref[:, :, rows])
+
+
+def test_fwd_merge_rows_without_keys_keep_the_accumulator():
+    """attn_fwd_merge with a chunk whose keys are all padded away for one
+    sequence (k_lens = 0): that sequence's accumulator is unchanged; the other
+    sequence gets attention over both chunks.  Also init with no keys gives
+    O = 0, LSE = -inf."""
+    import torch
+
+    attn = _lib()
+    B, H, Lq, LA, LB, d = 2, 2, 150, 200, 180, 128
+    Q = synth.normal_bf16(9301, (B, H, Lq, d))
+    KA = synth.normal_bf16(9302, (B, H, LA, d))
+    VA = synth.normal_bf16(9303, (B, H, LA, d))
+    KB = synth.normal_bf16(9304, (B, H, LB, d))
+    VB = synth.normal_bf16(9305, (B, H, LB, d))
+    scale = 1.0 / math.sqrt(d)
+    acc = torch.empty((B, H, Lq, d), dtype=torch.float32, device="cuda")
+    lacc = torch.empty((B, H, Lq), dtype=torch.float32, device="cuda")
+    O = torch.empty((B, H, Lq, d), dtype=torch.bfloat16, device="cuda")
+    q = dev_bf16(Q)
+    attn.attn_fwd_merge(q, dev_bf16(KA), dev_bf16(VA), acc, lacc, init=True, scale=scale)
+    kl = torch.tensor([0, 150], dtype=torch.int32, device="cuda")
+    attn.attn_fwd_merge(q, dev_bf16(KB), dev_bf16(VB), acc, lacc, init=False, O_out=O,
+                        scale=scale, k_lens=kl)
+    torch.cuda.synchronize()
+    K = np.concatenate([KA, KB], axis=2)
+    V = np.concatenate([VA, VB], axis=2)
+    Oref, Lref = oracle.fwd(Q, K, V, scale, k_lens=[LA, LA + 150])
+    assert_out_close(to_f64(O), Oref)
+    assert_lse_close(to_f64(lacc), Lref)
+    # init from a chunk with no visible key at all
+    attn.attn_fwd_merge(q, dev_bf16(KB), dev_bf16(VB), acc, lacc, init=True, O_out=O,
+                        scale=scale, k_lens=torch.zeros(2, dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.all(acc == 0) and torch.all(O == 0) and torch.all(torch.isneginf(lacc))
