@@ -446,8 +446,22 @@ def ring_leg(steps, warmup, world, flush):
                 fold_chunk(qs[r], ks[src], vs[src], kind, acc[r][0], acc[r][1], first=(s == 0),
                            O_out=acc[r][2] if s == last else None, workspace=ws)
 
+    # one emulated step is ten launches with Python between them: capture it in a
+    # CUDA graph so that the timed region holds the kernels back to back (first
+    # run outside the capture, which also sets the kernels' attributes)
+    step()
+    torch.cuda.synchronize()
+    run, launch = step, "stream"
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        run, launch = graph.replay, "cuda graph"
+    except Exception as e:  # capture refused: time the plain launches instead
+        launch = f"stream (graph capture failed: {type(e).__name__})"
+        torch.cuda.synchronize()
     barrier(world)
-    ms = timed_loop(step, steps, warmup, torch.cuda.current_stream(), flush)
+    ms = timed_loop(run, steps, warmup, torch.cuda.current_stream(), flush)
     st = attn.attn_read_device_status(ws)
     if st[0] != attn.ATTN_OK:
         raise RuntimeError(f"device status {st}")
@@ -462,7 +476,7 @@ def ring_leg(steps, warmup, world, flush):
     mbytes = rows * (4 * c["d"] * 2 + 2 * c["d"] + 12)  # acc read + write, partial, LSEs
     del qs, ks, vs, acc
     torch.cuda.empty_cache()
-    return ms, flops, n_fold, mms, mbytes, wms
+    return ms, flops, n_fold, mms, mbytes, wms, launch
 
 
 def bwd_leg(steps, warmup, world, flush):
@@ -628,6 +642,7 @@ def main():
             rep["ring_ms"] = float(np.mean(ring[0]))
             rep["ring_TFLOPs"] = ring[1] / (float(np.mean(ring[0])) * 1e-3) / 1e12
             rep["merge_GBs"] = ring[4] / (float(np.mean(ring[3])) * 1e-3) / 1e9
+            rep["ring_launch"] = ring[6]
         if rank == 0:
             print(json.dumps(rep), flush=True)
         return
@@ -730,7 +745,7 @@ def main():
         }
         line["gpu_launches"] += 3 * max(3, args.steps // 2)
     if ring is not None:
-        rms, rflops, n_fold, mms, mbytes, wholems = ring
+        rms, rflops, n_fold, mms, mbytes, wholems, rlaunch = ring
         t_r = max_over_ranks(float(np.mean(rms)), world)
         gbs = mbytes / (float(np.mean(mms)) * 1e-3) / 1e9
         line["ring"] = {
@@ -740,6 +755,7 @@ def main():
                         f"one GPU)",
             "value": world * rflops / (t_r * 1e-3) / 1e12, "unit": "TFLOP/s",
             "ms_per_step": t_r, "flops_per_step": rflops, "chunk_folds_per_step": n_fold,
+            "launch": rlaunch,
             "undivided_ms": float(np.mean(wholems)),
             "undivided_TFLOPs": rflops / (float(np.mean(wholems)) * 1e-3) / 1e12,
             "merge": {"kernel": "attn_merge_impl::merge_kernel", "rows": RING["B"] * RING["Hq"]

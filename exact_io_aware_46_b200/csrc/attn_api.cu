@@ -9,6 +9,8 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <set>
+#include <tuple>
 
 #include "../../include/attn.h"
 #include "bwd_kernel.cuh"
@@ -107,9 +109,22 @@ bool shapes_ok(int B, int Hq, int Hkv, int Lq, int Lk) {
   return true;
 }
 
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device, size):
+// repeated launches then make no attribute call, which also keeps launches that
+// are being captured into a CUDA graph free of non-stream API calls.
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  static std::mutex mu;
+  static std::set<std::tuple<const void*, int, int>> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const auto key = std::make_tuple(reinterpret_cast<const void*>(kernel), dev, bytes);
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count(key)) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.insert(key);
+  return e;
 }
 
 }  // namespace
