@@ -415,7 +415,7 @@ def ring_leg(steps, warmup, world, flush):
     import torch
 
     import exact_io_aware_46_b200 as attn
-    from exact_io_aware_46_b200.ring import fold_chunk, ring_steps
+    from exact_io_aware_46_b200.ring import bwd_chunk, fold_chunk, ring_steps
 
     c = RING
     W, Lc = c["world"], c["L"] // c["world"]
@@ -429,10 +429,46 @@ def ring_leg(steps, warmup, world, flush):
     ws = torch.zeros(256, dtype=torch.uint8, device=dev)
     # the undivided sequence in one call, for comparison
     O1 = torch.empty_like(q)
-    whole = lambda: attn.attn_fwd(q, k, v, causal=True, O=O1, workspace=ws)
+    L1 = torch.empty((c["B"], c["Hq"], c["L"]), dtype=torch.float32, device=dev)
+    whole = lambda: attn.attn_fwd(q, k, v, causal=True, O=O1, lse=L1, workspace=ws)
     barrier(world)
     wms = timed_loop(whole, steps, warmup, torch.cuda.current_stream(), flush)
-    del q, k, v, O1
+    # the backward's decomposition: every rank's chunk pairs through attn_bwd, the
+    # partial gradients summed in fp32 (stream launches), next to the undivided call
+    dO = synth.normal_bf16_device(synth.workload_seed(3, "do"), tuple(q.shape), dev)
+    bws = torch.zeros(attn.attn_bwd_workspace_size(c["B"], c["Hq"], c["Hkv"], Lc, Lc, c["d"]),
+                      dtype=torch.uint8, device=dev)
+    bws_whole = torch.zeros(attn.attn_bwd_workspace_size(c["B"], c["Hq"], c["Hkv"], c["L"],
+                                                         c["L"], c["d"]),
+                            dtype=torch.uint8, device=dev)
+    os_ = [O1[:, :, r * Lc:(r + 1) * Lc].contiguous() for r in range(W)]
+    ls_ = [L1[:, :, r * Lc:(r + 1) * Lc].contiguous() for r in range(W)]
+    dos = [dO[:, :, r * Lc:(r + 1) * Lc].contiguous() for r in range(W)]
+    dq_acc = [torch.empty_like(qs[0], dtype=torch.float32) for _ in range(W)]
+    dk_acc = [torch.empty_like(ks[0], dtype=torch.float32) for _ in range(W)]
+    dv_acc = [torch.empty_like(vs[0], dtype=torch.float32) for _ in range(W)]
+    bplans = [ring_steps(r, W, True) for r in range(W)]
+
+    def bwd_step():
+        started = set()
+        for r in range(W):
+            first = True
+            for _, src, kind in bplans[r]:
+                part = bwd_chunk(qs[r], ks[src], vs[src], os_[r], dos[r], ls_[r], kind,
+                                 workspace=bws)
+                if part is None:
+                    continue
+                attn.attn_accumulate(part[0], dq_acc[r], init=first)
+                first = False
+                attn.attn_accumulate(part[1], dk_acc[src], init=src not in started)
+                attn.attn_accumulate(part[2], dv_acc[src], init=src not in started)
+                started.add(src)
+
+    barrier(world)
+    bms_ring = timed_loop(bwd_step, max(3, steps // 2), warmup, torch.cuda.current_stream(), flush)
+    whole_b = lambda: attn.attn_bwd(q, k, v, O1, dO, L1, causal=True, workspace=bws_whole)
+    bms_whole = timed_loop(whole_b, max(3, steps // 2), warmup, torch.cuda.current_stream(), flush)
+    del q, k, v, O1, L1, dO, os_, ls_, dos, dq_acc, dk_acc, dv_acc, bws, bws_whole
     acc = [(torch.empty((c["B"], c["Hq"], Lc, c["d"]), dtype=torch.float32, device=dev),
             torch.empty((c["B"], c["Hq"], Lc), dtype=torch.float32, device=dev),
             torch.empty((c["B"], c["Hq"], Lc, c["d"]), dtype=torch.bfloat16, device=dev))
@@ -476,7 +512,7 @@ def ring_leg(steps, warmup, world, flush):
     mbytes = rows * (4 * c["d"] * 2 + 2 * c["d"] + 12)  # acc read + write, partial, LSEs
     del qs, ks, vs, acc
     torch.cuda.empty_cache()
-    return ms, flops, n_fold, mms, mbytes, wms, launch
+    return ms, flops, n_fold, mms, mbytes, wms, launch, (bms_ring, bms_whole)
 
 
 def bwd_leg(steps, warmup, world, flush):
@@ -745,7 +781,7 @@ def main():
         }
         line["gpu_launches"] += 3 * max(3, args.steps // 2)
     if ring is not None:
-        rms, rflops, n_fold, mms, mbytes, wholems, rlaunch = ring
+        rms, rflops, n_fold, mms, mbytes, wholems, rlaunch, (rbms, wbms) = ring
         t_r = max_over_ranks(float(np.mean(rms)), world)
         gbs = mbytes / (float(np.mean(mms)) * 1e-3) / 1e9
         line["ring"] = {
@@ -756,6 +792,15 @@ def main():
             "value": world * rflops / (t_r * 1e-3) / 1e12, "unit": "TFLOP/s",
             "ms_per_step": t_r, "flops_per_step": rflops, "chunk_folds_per_step": n_fold,
             "launch": rlaunch,
+            "backward": {
+                "workload": "the same decomposition for the backward: attn_bwd per visible "
+                            "chunk pair from the whole-sequence O and LSE, partial gradients "
+                            "summed in fp32 with attn_accumulate (stream launches)",
+                "value": world * 2.5 * rflops / (max_over_ranks(float(np.mean(rbms)), world)
+                                                 * 1e-3) / 1e12,
+                "unit": "TFLOP/s", "ms_per_step": max_over_ranks(float(np.mean(rbms)), world),
+                "undivided_ms": float(np.mean(wbms)),
+                "undivided_TFLOPs": 2.5 * rflops / (float(np.mean(wbms)) * 1e-3) / 1e12},
             "undivided_ms": float(np.mean(wholems)),
             "undivided_TFLOPs": rflops / (float(np.mean(wholems)) * 1e-3) / 1e12,
             "merge": {"kernel": "attn_merge_impl::merge_kernel", "rows": RING["B"] * RING["Hq"]
@@ -764,7 +809,9 @@ def main():
                                    "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
                                    "traffic": traffic_per_launch("attn_merge_impl::merge_kernel")}},
         }
-        line["gpu_launches"] += n_fold * args.steps + 2 * args.steps
+        # backward: per visible chunk pair 3 bwd kernels + 3 sums; the undivided call 3
+        line["gpu_launches"] += (n_fold * args.steps + 2 * args.steps
+                                 + (6 * n_fold + 3) * max(3, args.steps // 2))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:

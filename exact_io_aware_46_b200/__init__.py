@@ -56,6 +56,7 @@ SIGNATURES = {
                               _sz, _vp]),
     "attn_fwd_merge": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp,
                             _vp, _sz, _vp]),
+    "attn_accumulate": (_i, [_vp, _vp, _vp, ctypes.c_longlong, _i, _vp]),
     "attn_merge_partial": (_i, [_vp, _vp, _vp, _vp, _vp, ctypes.c_longlong, _i, _i, _vp]),
     "attn_fwd_fp8": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i,
                           _vp, _vp, _sz, _vp]),
@@ -259,6 +260,23 @@ def attn_fwd_merge(Q, K, V, O_acc, lse_acc, init, O_out=None, scale=None, causal
                                 float(scale), ATTN_MASK_CAUSAL if causal else ATTN_MASK_NONE,
                                 _ptr(k_lens), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(code, "attn_fwd_merge")
+
+
+def attn_accumulate(part, acc, init, out=None, stream=None):
+    """acc (fp32) += part (bf16), or acc = part with ``init``; ``part`` None adds
+    nothing; ``out`` (bf16, optional) receives the sum."""
+    _f32(acc, "acc")
+    if part is not None:
+        _bf16(part, "part")
+        if part.shape != acc.shape:
+            raise ValueError("partial and accumulator shapes differ")
+    if out is not None:
+        _bf16(out, "out")
+        if out.shape != acc.shape:
+            raise ValueError("output and accumulator shapes differ")
+    code = lib().attn_accumulate(_ptr(part), _ptr(acc), _ptr(out), acc.numel(),
+                                 1 if init else 0, _stream(stream))
+    _check(code, "attn_accumulate")
 
 
 def attn_merge_partial(O_part, lse_part, O_acc, lse_acc, init, O_out=None, stream=None):

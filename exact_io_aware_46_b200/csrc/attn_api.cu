@@ -13,6 +13,7 @@
 #include <tuple>
 
 #include "../../include/attn.h"
+#include "accum_kernel.cuh"
 #include "bwd_kernel.cuh"
 #include "decode_kernel.cuh"
 #include "fwd_kernel.cuh"
@@ -385,6 +386,29 @@ attn_status_t attn_merge_partial(const attn_bf16_t* O_part, const float* lse_par
   const long long cap = static_cast<long long>(sms) * 8;  // 8 resident blocks per SM
   const int grid = static_cast<int>(need < cap ? need : cap);
   attn_merge_impl::merge_kernel<<<grid, attn_merge_impl::NTHREADS, 0,
+                                  reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_accumulate(const attn_bf16_t* part, float* acc, attn_bf16_t* out, long long n,
+                              int init, void* stream) {
+  if (n < 0 || n % 8 != 0 || (init != 0 && init != 1) || !acc) return ATTN_ERR_INVALID;
+  if (!part && init) return ATTN_ERR_INVALID;
+  if ((part && !aligned16(part)) || !aligned16(acc) || (out && !aligned16(out)))
+    return ATTN_ERR_INVALID;
+  if (n == 0) return ATTN_OK;
+  const int sms = device_sms();
+  if (sms <= 0) return ATTN_ERR_CUDA;
+  attn_accum_impl::Params p;
+  p.part = reinterpret_cast<const __nv_bfloat16*>(part);
+  p.acc = acc;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.n8 = n / 8;
+  p.init = init;
+  const long long need = (p.n8 + attn_accum_impl::NTHREADS - 1) / attn_accum_impl::NTHREADS;
+  const long long cap = static_cast<long long>(sms) * 8;
+  attn_accum_impl::accum_kernel<<<static_cast<int>(need < cap ? need : cap),
+                                  attn_accum_impl::NTHREADS, 0,
                                   reinterpret_cast<cudaStream_t>(stream)>>>(p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

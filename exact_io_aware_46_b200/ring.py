@@ -18,8 +18,17 @@ entirely masked and skipped (its exchange still runs, so every rank takes the
 same collective steps in the same order), the diagonal chunk is causal and the
 earlier chunks are fully visible.
 
-The exchange moves K/V between ranks and the kernels compute; there is no
-compute on the host and no fallback: ``ring_attn_fwd`` needs the CUDA library.
+The backward (``ring_attn_bwd``) runs the same ring with the forward's global O
+and LSE: the partial gradients of a (query chunk, key chunk) pair from
+``attn_bwd`` are exact pieces of the whole-sequence gradients, since P and
+D = rowsum(dO o O) only need the global LSE and O.  dQ sums locally; the running
+sums of a chunk's dK and dV travel with that chunk (each rank adds its share
+before passing them on) and one extra pass at the end brings them home.  The sums
+are kept in fp32 by ``attn_accumulate``.
+
+The exchange moves K/V (and gradient sums) between ranks and the kernels compute;
+there is no compute on the host and no fallback: ``ring_attn_fwd`` and
+``ring_attn_bwd`` need the CUDA library.
 """
 
 from __future__ import annotations
@@ -120,3 +129,76 @@ def ring_attn_fwd(q, k, v, group=None, causal=True, scale=None):
         if s + 1 < world:
             ex.finish()
     return O, lse_acc
+
+
+def bwd_chunk(q, kc, vc, o, do, lse, kind, scale=None, workspace=None):
+    """One ring step's backward: the partial (dQ, dK, dV) (bf16) of this rank's
+    query chunk against the K/V chunk held at this step, from the whole-sequence
+    O and LSE of this rank's rows; None for a SKIP step."""
+    from . import attn_bwd
+
+    if kind == SKIP:
+        return None
+    return attn_bwd(q, kc, vc, o, do, lse, scale=scale, causal=(kind == CAUSAL),
+                    workspace=workspace)
+
+
+def ring_bwd_pass(kv, grads, steps, compute, add, group=None):
+    """The backward's data movement.  ``kv``: this rank's K/V chunk tensors, sent
+    around the ring one step ahead as in the forward; ``grads``: zeroed running
+    sums of this chunk's gradients, which travel with their chunk.  At each step
+    ``compute(kind, src, kv_held)`` returns this rank's partial for the held
+    chunk (or None) while the previous step's sums are still in flight, then
+    ``add(partial, grads_held)`` adds it into the held chunk's sums, which are
+    passed on.  Returns this rank's own chunk's sums after the closing pass."""
+    world = len(steps)
+    kvx = RingExchange(kv, group)
+    gx = RingExchange(grads, group)
+    for s, src, kind in steps:
+        if s + 1 < world:
+            kvx.start()
+        part = compute(kind, src, kvx.cur)
+        if s > 0:
+            gx.finish()
+        if part is not None:
+            add(part, gx.cur)
+        gx.start()
+        if s + 1 < world:
+            kvx.finish()
+    gx.finish()
+    return gx.cur
+
+
+def ring_attn_bwd(q, k, v, o, do, lse, group=None, causal=True, scale=None):
+    """Ring-attention backward.  q, o, do [B, Hq, Lc, d] and lse [B, Hq, Lc] of
+    this rank's rows (o and lse from ``ring_attn_fwd``), k/v [B, Hkv, Lc, d] of
+    this rank's keys.  Returns this rank's (dQ, dK, dV) bf16 of the whole-sequence
+    loss."""
+    from . import attn_accumulate
+
+    if not q.is_cuda:
+        raise ValueError("ring_attn_bwd runs on the CUDA kernels")
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    steps = ring_steps(rank, world, causal)
+    dq_acc = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    first = [True]
+
+    def compute(kind, src, kv_held):
+        return bwd_chunk(q, kv_held[0], kv_held[1], o, do, lse, kind, scale=scale)
+
+    def add(part, g):
+        dqp, dkp, dvp = part
+        attn_accumulate(dqp, dq_acc, init=first[0])
+        first[0] = False
+        attn_accumulate(dkp, g[0], init=False)
+        attn_accumulate(dvp, g[1], init=False)
+
+    zeros = (torch.zeros(k.shape, dtype=torch.float32, device=k.device),
+             torch.zeros(v.shape, dtype=torch.float32, device=v.device))
+    gk, gv = ring_bwd_pass((k, v), zeros, steps, compute, add, group)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    attn_accumulate(None, dq_acc, init=False, out=dq)
+    attn_accumulate(None, gk, init=False, out=dk)
+    attn_accumulate(None, gv, init=False, out=dv)
+    return dq, dk, dv

@@ -158,6 +158,14 @@ attn_status_t attn_fwd_merge(const attn_bf16_t* Q, const attn_bf16_t* K, const a
                              const int32_t* k_lens, void* workspace, size_t ws_bytes,
                              void* stream);
 
+/* Adds a bf16 partial [n] into an fp32 accumulator [n] (init = 1: sets it to
+ * the partial; part = NULL with init = 0 adds nothing, to convert the sum);
+ * out [n] bf16 or NULL receives the running sum.  Used to sum ring attention's
+ * per-chunk partial gradients with one rounding at the end.  n >= 0 and a
+ * multiple of 8; pointers 16-byte aligned; else ATTN_ERR_INVALID. */
+attn_status_t attn_accumulate(const attn_bf16_t* part, float* acc, attn_bf16_t* out, long long n,
+                              int init, void* stream);
+
 /* ------------------------------------------------------------------ sliding window
  * Local causal (sliding-window) attention: the causal mask of attn_fwd /
  * attn_bwd plus a lower edge, so query row i sees only keys j with

@@ -149,6 +149,11 @@ def test_fwd_merge_and_merge_partial_reject_on_host(lib):
         return lib.attn_merge_partial(part, P, P, P, None, rows, d, init, None)
     assert mp(d=96) == 1 and mp(d=512) == 1 and mp(rows=-1) == 1 and mp(init=3) == 1
     assert mp(part=None) == 1 and mp(rows=0) == 0
+    # attn_accumulate: n a multiple of 8; no partial only when adding (convert)
+    assert lib.attn_accumulate(P, P, None, 12, 0, None) == 1
+    assert lib.attn_accumulate(None, P, None, 16, 1, None) == 1
+    assert lib.attn_accumulate(P, None, None, 16, 0, None) == 1
+    assert lib.attn_accumulate(P, P, None, 0, 0, None) == 0
 
 
 def test_product_path_does_not_touch_oracle():

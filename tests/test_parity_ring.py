@@ -140,3 +140,74 @@ def test_fwd_merge_rows_without_keys_keep_the_accumulator():
                         scale=scale, k_lens=torch.zeros(2, dtype=torch.int32, device="cuda"))
     torch.cuda.synchronize()
     assert torch.all(acc == 0) and torch.all(O == 0) and torch.all(torch.isneginf(lacc))
+
+
+def test_accumulate_kernel():
+    import torch
+
+    attn = _lib()
+    parts = [dev_bf16(synth.normal_bf16(9400 + i, (3, 5, 64))) for i in range(3)]
+    acc = torch.full((3, 5, 64), 7.0, device="cuda")
+    out = torch.empty((3, 5, 64), dtype=torch.bfloat16, device="cuda")
+    attn.attn_accumulate(parts[0], acc, init=True)
+    attn.attn_accumulate(parts[1], acc, init=False)
+    attn.attn_accumulate(parts[2], acc, init=False, out=out)
+    torch.cuda.synchronize()
+    ref = parts[0].float() + parts[1].float() + parts[2].float()
+    assert torch.equal(acc, ref) and torch.equal(out, ref.to(torch.bfloat16))
+    attn.attn_accumulate(None, acc, init=False, out=out)  # convert only
+    torch.cuda.synchronize()
+    assert torch.equal(acc, ref)
+
+
+@pytest.mark.parametrize("world,causal,Hq,Hkv,Lc,d", [
+    (2, True, 4, 2, 200, 128),
+    (3, True, 2, 2, 130, 128),
+    (3, False, 2, 1, 150, 128),   # the backward kernels take d = 128
+])
+def test_ring_backward_decomposition_matches_whole_sequence(world, causal, Hq, Hkv, Lc, d):
+    """Each rank's steps (bwd_chunk from the whole-sequence O and LSE, partials
+    summed in fp32 by attn_accumulate; each key chunk's dK/dV summed over every
+    rank) against the oracle's gradients of the whole sequence."""
+    import torch
+
+    from exact_io_aware_46_b200.ring import bwd_chunk
+
+    attn = _lib()
+    L = world * Lc
+    seed = 9500 + world * 10 + Lc
+    Q = synth.normal_bf16(seed * 8 + 1, (1, Hq, L, d))
+    K = synth.normal_bf16(seed * 8 + 2, (1, Hkv, L, d))
+    V = synth.normal_bf16(seed * 8 + 3, (1, Hkv, L, d))
+    dO = synth.normal_bf16(seed * 8 + 4, (1, Hq, L, d))
+    q, k, v, do = (dev_bf16(x) for x in (Q, K, V, dO))
+    scale = 1.0 / math.sqrt(d)
+    O, Lse = attn.attn_fwd(q, k, v, scale=scale, causal=causal)
+    rQ, rK, rV = oracle.bwd(Q, K, V, dO, scale, causal=causal)
+    sl = [slice(c * Lc, (c + 1) * Lc) for c in range(world)]
+    dk_acc = [torch.zeros((1, Hkv, Lc, d), device="cuda") for _ in range(world)]
+    dv_acc = [torch.zeros((1, Hkv, Lc, d), device="cuda") for _ in range(world)]
+    dq = torch.empty_like(q)
+    for rank in range(world):
+        qr, orr, dor = (t[:, :, sl[rank]].contiguous() for t in (q, O, do))
+        lr = Lse[:, :, sl[rank]].contiguous()
+        dq_acc = torch.empty((1, Hq, Lc, d), device="cuda")
+        first = True
+        for _, src, kind in ring_steps(rank, world, causal):
+            part = bwd_chunk(qr, k[:, :, sl[src]].contiguous(), v[:, :, sl[src]].contiguous(),
+                             orr, dor, lr, kind, scale=scale)
+            if part is None:
+                continue
+            attn.attn_accumulate(part[0], dq_acc, init=first)
+            first = False
+            attn.attn_accumulate(part[1], dk_acc[src], init=False)
+            attn.attn_accumulate(part[2], dv_acc[src], init=False)
+        out = torch.empty_like(qr)
+        attn.attn_accumulate(None, dq_acc, init=False, out=out)
+        dq[:, :, sl[rank]] = out
+    torch.cuda.synchronize()
+    dk = torch.cat(dk_acc, dim=2)
+    dv = torch.cat(dv_acc, dim=2)
+    from tests._util import GRAD_REL_L2, rel_l2
+    for got, ref, what in ((dq, rQ, "dQ"), (dk, rK, "dK"), (dv, rV, "dV")):
+        assert rel_l2(to_f64(got), ref) <= GRAD_REL_L2, f"{what}: {rel_l2(to_f64(got), ref):.3e}"

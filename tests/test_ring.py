@@ -115,3 +115,50 @@ def test_ring_exchange_on_gloo_ranks(tmp_path, world):
         seen = eval(open(out + f".{rank}").read())
         assert seen == [(float((rank - s) % world), 10.0 * ((rank - s) % world))
                         for s in range(world)]
+
+
+def _bwd_pass_main(rank, world, port, out, causal):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from exact_io_aware_46_b200.ring import ring_bwd_pass
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    steps = ring_steps(rank, world, causal)
+    seen = []
+
+    def compute(kind, src, kv_held):
+        seen.append(float(kv_held[0][0]))  # the K/V chunk held at this step
+        return None if kind == SKIP else float(rank + 1)
+
+    def add(part, g):
+        g[0] += part
+
+    kv = (torch.full((4,), float(rank)),)
+    sums = ring_bwd_pass(kv, (torch.zeros(4),), steps, compute, add)
+    dist.barrier()
+    dist.destroy_process_group()
+    with open(out + f".{rank}", "w") as f:
+        f.write(repr((seen, float(sums[0][0]))))
+
+
+@pytest.mark.parametrize("world,causal", [(2, True), (3, True), (3, False)])
+def test_ring_backward_gradient_sums_travel_home(tmp_path, world, causal):
+    """Every rank adds its share to the sums of the chunk it holds; after the
+    closing pass each rank holds its own chunk's total: the shares of every rank
+    whose step on that chunk was not skipped."""
+    import torch.multiprocessing as mp
+
+    out = str(tmp_path / "g")
+    mp.start_processes(_bwd_pass_main, args=(world, _free_port(), out, causal), nprocs=world,
+                       join=True, start_method="spawn")
+    for rank in range(world):
+        seen, total = eval(open(out + f".{rank}").read())
+        assert seen == [float((rank - s) % world) for s in range(world)]
+        contributors = [r for r in range(world) if not causal or r >= rank]
+        assert total == float(sum(r + 1 for r in contributors))
