@@ -153,6 +153,12 @@ def ring_bwd_pass(kv, grads, steps, compute, add, group=None):
     passed on.  Returns this rank's own chunk's sums after the closing pass."""
     world = len(steps)
     kvx = RingExchange(kv, group)
+    if world == 1:  # nothing travels: the rank's own chunk is the whole sequence
+        grads = [t.contiguous() for t in grads]
+        part = compute(steps[0][2], steps[0][1], kvx.cur)
+        if part is not None:
+            add(part, grads)
+        return grads
     gx = RingExchange(grads, group)
     for s, src, kind in steps:
         if s + 1 < world:

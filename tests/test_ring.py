@@ -103,7 +103,7 @@ def _exchange_main(rank, world, port, out):
         f.write(repr(seen))
 
 
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [1, 2, 3])
 def test_ring_exchange_on_gloo_ranks(tmp_path, world):
     """At step s every rank holds the chunk of rank (rank - s) mod world."""
     import torch.multiprocessing as mp
@@ -147,7 +147,7 @@ def _bwd_pass_main(rank, world, port, out, causal):
         f.write(repr((seen, float(sums[0][0]))))
 
 
-@pytest.mark.parametrize("world,causal", [(2, True), (3, True), (3, False)])
+@pytest.mark.parametrize("world,causal", [(1, True), (2, True), (3, True), (3, False)])
 def test_ring_backward_gradient_sums_travel_home(tmp_path, world, causal):
     """Every rank adds its share to the sums of the chunk it holds; after the
     closing pass each rank holds its own chunk's total: the shares of every rank
