@@ -48,6 +48,10 @@ def test_workspace_sizes_are_closed_forms(lib):
     assert attn.attn_bwd_workspace_size(2, 16, 16, 8192, 8192, 128) == 256 + ((rows * 128 * 4 + rows * 8 + 255) // 256) * 256
     rows = 1 * 2 * 128  # Lq = 100 pads to 128
     assert attn.attn_bwd_workspace_size(1, 2, 1, 100, 300, 128) == 256 + ((rows * 128 * 4 + rows * 8 + 255) // 256) * 256
+    # d = 64: the d = 128 scratch plus zero-padded 128-column copies of Q, O, dO, dQ
+    # (query rows) and K, V, dK, dV (key rows), bf16
+    pad = 4 * (1 * 2 * 100 + 1 * 1 * 300) * 128 * 2
+    assert attn.attn_bwd_workspace_size(1, 2, 1, 100, 300, 64) == 256 + ((rows * 128 * 4 + rows * 8 + 255) // 256) * 256 + pad
 
 
 def test_status_strings(lib):

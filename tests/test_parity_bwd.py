@@ -66,6 +66,39 @@ def test_bwd_matches_oracle(B, Hq, Hkv, Lq, Lk, causal, k_lens):
     _check(to_f64(dv), rV, "dV")
 
 
+D64_CASES = [
+    # B, Hq, Hkv, Lq, Lk, causal, k_lens
+    (1, 2, 2, 256, 256, False, None),          # the tiny workload's shape (B1 H2 L256 d64)
+    (1, 4, 2, 200, 300, True, None),           # causal, Lq < Lk, grouped heads
+    (2, 2, 1, 190, 190, True, [190, 77]),      # key padding, ragged tiles
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,causal,k_lens", D64_CASES)
+def test_bwd_d64_matches_oracle(B, Hq, Hkv, Lq, Lk, causal, k_lens):
+    """d = 64: the d = 128 kernels on zero-padded copies (the zero columns change
+    neither P nor dS); the gradients' first 64 columns against the oracle."""
+    import torch
+
+    attn = _lib()
+    d = 64
+    seed = 700 + Lq + 3 * Lk + Hq
+    Q = synth.normal_bf16(seed * 16 + 1, (B, Hq, Lq, d))
+    K = synth.normal_bf16(seed * 16 + 2, (B, Hkv, Lk, d))
+    V = synth.normal_bf16(seed * 16 + 3, (B, Hkv, Lk, d))
+    dO = synth.normal_bf16(seed * 16 + 4, (B, Hq, Lq, d))
+    scale = 1.0 / math.sqrt(d)
+    q, k, v, do = (dev_bf16(x) for x in (Q, K, V, dO))
+    kl = None if k_lens is None else torch.tensor(k_lens, dtype=torch.int32, device="cuda")
+    O, L = attn.attn_fwd(q, k, v, causal=causal, k_lens=kl)
+    dq, dk, dv = attn.attn_bwd(q, k, v, O, do, L, causal=causal, k_lens=kl)
+    torch.cuda.synchronize()
+    rQ, rK, rV = oracle.bwd(Q, K, V, dO, scale, causal=causal, k_lens=k_lens)
+    _check(to_f64(dq), rQ, "dQ")
+    _check(to_f64(dk), rK, "dK")
+    _check(to_f64(dv), rV, "dV")
+
+
 def test_bwd_full_size_sampled():
     """B=2, H=16, L=8192, d=128, causal: sampled rows of dQ and keys of dK, dV."""
     import torch
