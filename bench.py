@@ -436,7 +436,8 @@ def ring_leg(steps, warmup, world, flush):
     import torch
 
     import exact_io_aware_46_b200 as attn
-    from exact_io_aware_46_b200.ring import bwd_chunk, fold_chunk, ring_steps
+    from exact_io_aware_46_b200.ring import (bwd_chunk, fold_chunk, ring_steps, zigzag_chunks,
+                                             zigzag_folds)
 
     c = RING
     W, Lc = c["world"], c["L"] // c["world"]
@@ -447,6 +448,10 @@ def ring_leg(steps, warmup, world, flush):
     qs = [q[:, :, r * Lc:(r + 1) * Lc].contiguous() for r in range(W)]
     ks = [k[:, :, r * Lc:(r + 1) * Lc].contiguous() for r in range(W)]
     vs = [v[:, :, r * Lc:(r + 1) * Lc].contiguous() for r in range(W)]
+    Lz = c["L"] // (2 * W)  # zigzag: 2 * W chunks, rank r holds chunks r and 2W - 1 - r
+    zq = [q[:, :, i * Lz:(i + 1) * Lz].contiguous() for i in range(2 * W)]
+    zk = [k[:, :, i * Lz:(i + 1) * Lz].contiguous() for i in range(2 * W)]
+    zv = [v[:, :, i * Lz:(i + 1) * Lz].contiguous() for i in range(2 * W)]
     ws = torch.zeros(256, dtype=torch.uint8, device=dev)
     # the undivided sequence in one call, for comparison
     O1 = torch.empty_like(q)
@@ -524,6 +529,56 @@ def ring_leg(steps, warmup, world, flush):
         raise RuntimeError(f"device status {st}")
     flops = 4.0 * c["d"] * causal_pairs(c["L"], c["L"], True) * c["Hq"] * c["B"]
     n_fold = sum(1 for p in plans for _, _, kind in p if kind != "skip")
+
+    # one rank's own kernels (what each GPU of a 4-GPU ring computes, the exchange
+    # aside), contiguous chunks against the zigzag layout; the slowest rank sets
+    # the step time
+    def graphed(fn):
+        fn()
+        torch.cuda.synchronize()
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            return g.replay, g
+        except Exception:
+            torch.cuda.synchronize()
+            return fn, None
+
+    def contiguous_rank(r):
+        last = max(s for s, _, kind in plans[r] if kind != "skip")
+        for s, src, kind in plans[r]:
+            fold_chunk(qs[r], ks[src], vs[src], kind, acc[r][0], acc[r][1], first=(s == 0),
+                       O_out=acc[r][2] if s == last else None, workspace=ws)
+
+    zacc = [[(torch.empty_like(zq[0], dtype=torch.float32),
+              torch.empty(zq[0].shape[:-1], dtype=torch.float32, device=dev),
+              torch.empty_like(zq[0])) for _ in range(2)] for _ in range(W)]
+    zplans = [zigzag_folds(r, W) for r in range(W)]
+
+    def zigzag_rank(r):
+        mine = zigzag_chunks(r, W)
+        for _, src, qi, ki, kind, first, last in zplans[r]:
+            ch = zigzag_chunks(src, W)[ki]
+            a = zacc[r][qi]
+            fold_chunk(zq[mine[qi]], zk[ch], zv[ch], kind, a[0], a[1], first=first,
+                       O_out=a[2] if last else None, workspace=ws)
+
+    per_rank = {}
+    graphs = []
+    for name, fn in (("contiguous", contiguous_rank), ("zigzag", zigzag_rank)):
+        t = []
+        for r in range(W):
+            run_r, g = graphed(lambda r=r: fn(r))
+            graphs.append(g)
+            t.append(float(np.mean(timed_loop(run_r, steps, warmup, torch.cuda.current_stream(),
+                                              flush))))
+        per_rank[name] = t
+    n_zfold = sum(len(p) for p in zplans)
+    st = attn.attn_read_device_status(ws)
+    if st[0] != attn.ATTN_OK:
+        raise RuntimeError(f"device status {st}")
+    del graphs, zq, zk, zv, zacc
     # the merge kernel alone: one chunk's rows folded into an accumulator
     Op = acc[0][2]
     lp = torch.zeros_like(acc[0][1])
@@ -533,7 +588,7 @@ def ring_leg(steps, warmup, world, flush):
     mbytes = rows * (4 * c["d"] * 2 + 2 * c["d"] + 12)  # acc read + write, partial, LSEs
     del qs, ks, vs, acc
     torch.cuda.empty_cache()
-    return ms, flops, n_fold, mms, mbytes, wms, launch, (bms_ring, bms_whole)
+    return ms, flops, n_fold, mms, mbytes, wms, launch, (bms_ring, bms_whole), (per_rank, n_zfold)
 
 
 def bwd_leg(steps, warmup, world, flush):
@@ -805,7 +860,7 @@ def main():
         }
         line["gpu_launches"] += 3 * max(3, args.steps // 2)
     if ring is not None:
-        rms, rflops, n_fold, mms, mbytes, wholems, rlaunch, (rbms, wbms) = ring
+        rms, rflops, n_fold, mms, mbytes, wholems, rlaunch, (rbms, wbms), (prank, n_zfold) = ring
         t_r = max_over_ranks(float(np.mean(rms)), world)
         gbs = mbytes / (float(np.mean(mms)) * 1e-3) / 1e9
         line["ring"] = {
@@ -816,6 +871,14 @@ def main():
             "value": world * rflops / (t_r * 1e-3) / 1e12, "unit": "TFLOP/s",
             "ms_per_step": t_r, "flops_per_step": rflops, "chunk_folds_per_step": n_fold,
             "launch": rlaunch,
+            "per_rank": {
+                "what": "each rank's own folds timed alone on this GPU (CUDA graph): the "
+                        "compute of one step of a 4-GPU ring, exchange aside; the slowest "
+                        "rank sets the step time",
+                "contiguous_ms": prank["contiguous"], "contiguous_max_ms": max(prank["contiguous"]),
+                "zigzag_ms": prank["zigzag"], "zigzag_max_ms": max(prank["zigzag"]),
+                "zigzag_TFLOPs_per_gpu_modelled": rflops / RING["world"]
+                / (max(prank["zigzag"]) * 1e-3) / 1e12},
             "backward": {
                 "workload": "the same decomposition for the backward: attn_bwd per visible "
                             "chunk pair from the whole-sequence O and LSE, partial gradients "
@@ -835,7 +898,8 @@ def main():
         }
         # backward: per visible chunk pair 3 bwd kernels + 3 sums; the undivided call 3
         line["gpu_launches"] += (n_fold * args.steps + 2 * args.steps
-                                 + (6 * n_fold + 3) * max(3, args.steps // 2))
+                                 + (6 * n_fold + 3) * max(3, args.steps // 2)
+                                 + (n_fold + n_zfold) * args.steps)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:

@@ -208,3 +208,81 @@ def ring_attn_bwd(q, k, v, o, do, lse, group=None, causal=True, scale=None):
     attn_accumulate(None, gk, init=False, out=dk)
     attn_accumulate(None, gv, init=False, out=dv)
     return dq, dk, dv
+
+
+# ---------------------------------------------------------------- zigzag layout
+# Under the causal mask, contiguous chunks leave rank r with r + 1 chunk
+# computations and the last rank with world of them.  In the zigzag layout the
+# sequence is cut into 2 * world chunks and rank r holds chunks r and
+# 2 * world - 1 - r (an early and a late one); K/V chunk pairs travel the ring
+# as before.  Every rank then computes two full-chunk equivalents per step: at
+# step 0 its two diagonal chunks (causal) and late-on-early (full), at every
+# other step two full chunk pairs; the other two pairs of the step are masked.
+
+
+def zigzag_chunks(rank: int, world: int):
+    """The two global chunk indices (of 2 * world) that rank ``rank`` holds."""
+    if not 0 <= rank < world:
+        raise ValueError("rank out of range")
+    return rank, 2 * world - 1 - rank
+
+
+def ring_steps_zigzag(rank: int, world: int):
+    """The causal zigzag schedule of one rank: a list of (step, source rank,
+    [(q, kv, kind), ...]) where q and kv index this rank's query chunk and the
+    held K/V chunk (0 = the early one, 1 = the late one) and kind is FULL or
+    CAUSAL; masked pairs are left out."""
+    mine = zigzag_chunks(rank, world)
+    out = []
+    for s in range(world):
+        src = (rank - s) % world
+        held = zigzag_chunks(src, world)
+        pairs = []
+        for qi, a in enumerate(mine):
+            for ki, b in enumerate(held):
+                if a > b:
+                    pairs.append((qi, ki, FULL))
+                elif a == b:
+                    pairs.append((qi, ki, CAUSAL))
+        out.append((s, src, pairs))
+    return out
+
+
+def zigzag_folds(rank: int, world: int):
+    """The folds of one rank in order: (step, source rank, q, kv, kind, first,
+    last), with first / last marking the first and the last fold into query
+    chunk q (the first initialises its accumulator, the last writes O)."""
+    flat = [(s, src, qi, ki, kind) for s, src, pairs in ring_steps_zigzag(rank, world)
+            for qi, ki, kind in pairs]
+    out = []
+    for i, (s, src, qi, ki, kind) in enumerate(flat):
+        first = all(f[2] != qi for f in flat[:i])
+        last = all(f[2] != qi for f in flat[i + 1:])
+        out.append((s, src, qi, ki, kind, first, last))
+    return out
+
+
+def ring_attn_fwd_zigzag(q, k, v, group=None, scale=None):
+    """Causal ring-attention forward in the zigzag layout.  q, k, v: pairs of
+    bf16 CUDA tensors, this rank's early and late chunk (global chunks r and
+    2 * world - 1 - r of equal length): q [B, Hq, Lc, d], k/v [B, Hkv, Lc, d].
+    Returns (O pair, LSE pair) for the two query chunks."""
+    if not q[0].is_cuda:
+        raise ValueError("ring_attn_fwd_zigzag runs on the CUDA kernels")
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    folds = zigzag_folds(rank, world)
+    O_acc = [torch.empty(t.shape, dtype=torch.float32, device=t.device) for t in q]
+    lse_acc = [torch.empty(t.shape[:-1], dtype=torch.float32, device=t.device) for t in q]
+    O = [torch.empty_like(t) for t in q]
+    ex = RingExchange((k[0], k[1], v[0], v[1]), group)
+    for s in range(world):
+        if s + 1 < world:
+            ex.start()
+        k0, k1, v0, v1 = ex.cur
+        for _, _, qi, ki, kind, first, last in (f for f in folds if f[0] == s):
+            fold_chunk(q[qi], (k0, k1)[ki], (v0, v1)[ki], kind, O_acc[qi], lse_acc[qi],
+                       first=first, O_out=O[qi] if last else None, scale=scale)
+        if s + 1 < world:
+            ex.finish()
+    return tuple(O), tuple(lse_acc)

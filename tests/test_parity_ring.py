@@ -211,3 +211,39 @@ def test_ring_backward_decomposition_matches_whole_sequence(world, causal, Hq, H
     from tests._util import GRAD_REL_L2, rel_l2
     for got, ref, what in ((dq, rQ, "dQ"), (dk, rK, "dK"), (dv, rV, "dV")):
         assert rel_l2(to_f64(got), ref) <= GRAD_REL_L2, f"{what}: {rel_l2(to_f64(got), ref):.3e}"
+
+
+@pytest.mark.parametrize("world,Hq,Hkv,Lc", [(2, 4, 2, 150), (3, 2, 2, 130)])
+def test_ring_zigzag_decomposition_matches_whole_sequence(world, Hq, Hkv, Lc):
+    """The causal zigzag layout (rank r holds chunks r and 2*world-1-r): every
+    rank's folds from zigzag_folds on the CUDA kernels, chunks taken from one
+    tensor, against the oracle's whole-sequence attention."""
+    import torch
+
+    from exact_io_aware_46_b200.ring import zigzag_chunks, zigzag_folds
+
+    d = 128
+    L = 2 * world * Lc
+    seed = 9700 + world * 10 + Lc
+    Q = synth.normal_bf16(seed * 4 + 1, (1, Hq, L, d))
+    K = synth.normal_bf16(seed * 4 + 2, (1, Hkv, L, d))
+    V = synth.normal_bf16(seed * 4 + 3, (1, Hkv, L, d))
+    q_all, k_all, v_all = dev_bf16(Q), dev_bf16(K), dev_bf16(V)
+    scale = 1.0 / math.sqrt(d)
+    Oref, Lref = oracle.fwd(Q, K, V, scale, causal=True)
+    ch = lambda t, c: t[:, :, c * Lc:(c + 1) * Lc]
+    for rank in range(world):
+        mine = zigzag_chunks(rank, world)
+        qs = [ch(q_all, c).contiguous() for c in mine]
+        acc = [torch.empty((1, Hq, Lc, d), device="cuda") for _ in range(2)]
+        lacc = [torch.empty((1, Hq, Lc), device="cuda") for _ in range(2)]
+        O = [torch.empty((1, Hq, Lc, d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+        for _, src, qi, ki, kind, first, last in zigzag_folds(rank, world):
+            c = zigzag_chunks(src, world)[ki]
+            fold_chunk(qs[qi], ch(k_all, c).contiguous(), ch(v_all, c).contiguous(), kind,
+                       acc[qi], lacc[qi], first=first, O_out=O[qi] if last else None,
+                       scale=scale)
+        torch.cuda.synchronize()
+        for qi in (0, 1):
+            assert_out_close(to_f64(O[qi]), ch(Oref, mine[qi]), f"O[rank {rank}, chunk {qi}]")
+            assert_lse_close(to_f64(lacc[qi]), ch(Lref, mine[qi]))

@@ -162,3 +162,79 @@ def test_ring_backward_gradient_sums_travel_home(tmp_path, world, causal):
         assert seen == [float((rank - s) % world) for s in range(world)]
         contributors = [r for r in range(world) if not causal or r >= rank]
         assert total == float(sum(r + 1 for r in contributors))
+
+
+# ---------------------------------------------------------------- zigzag layout
+
+from exact_io_aware_46_b200.ring import ring_steps_zigzag, zigzag_chunks  # noqa: E402
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
+def test_zigzag_schedule_is_balanced_and_complete(world):
+    """Every visible (query chunk, key chunk) pair of the causal 2*world-chunk
+    sequence is computed exactly once, by the rank holding the query chunk, and
+    every rank computes two full-chunk equivalents per step (a causal diagonal
+    pair counts one half)."""
+    seen = set()
+    for rank in range(world):
+        mine = zigzag_chunks(rank, world)
+        for s, src, pairs in ring_steps_zigzag(rank, world):
+            held = zigzag_chunks(src, world)
+            assert src == (rank - s) % world
+            work = 0.0
+            for qi, ki, kind in pairs:
+                a, b = mine[qi], held[ki]
+                assert (kind == CAUSAL) == (a == b) and a >= b
+                assert (a, b) not in seen
+                seen.add((a, b))
+                work += 0.5 if kind == CAUSAL else 1.0
+            assert work == 2.0
+    n = 2 * world
+    assert seen == {(a, b) for a in range(n) for b in range(a + 1)}
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_zigzag_schedule_composes_exact_attention_on_the_oracle(world):
+    """Each rank's zigzag partials (oracle forward per pair), merged in fold
+    order with the oracle's merge rule, equal the oracle's causal attention over
+    the whole sequence for the rank's two chunks."""
+    Lc, d = 23, 8
+    L = 2 * world * Lc
+    Q = synth.bf16_bits_to_f64(synth.normal_bf16(631, (1, 2, L, d)))
+    K = synth.bf16_bits_to_f64(synth.normal_bf16(632, (1, 1, L, d)))
+    V = synth.bf16_bits_to_f64(synth.normal_bf16(633, (1, 1, L, d)))
+    Oref, Lref = oracle.fwd(Q, K, V, 0.4, causal=True)
+    ch = lambda t, c: t[:, :, c * Lc:(c + 1) * Lc]
+    for rank in range(world):
+        mine = zigzag_chunks(rank, world)
+        acc = [None, None]
+        for _, src, pairs in ring_steps_zigzag(rank, world):
+            held = zigzag_chunks(src, world)
+            for qi, ki, kind in pairs:
+                Op, lp = oracle.fwd(ch(Q, mine[qi]), ch(K, held[ki]), ch(V, held[ki]), 0.4,
+                                    causal=(kind == CAUSAL))
+                if acc[qi] is None:
+                    acc[qi] = [Op.copy(), lp.copy()]
+                    continue
+                for h in range(2):
+                    for i in range(Lc):
+                        m, l, o = oracle.merge(acc[qi][1][0, h, i], 1.0, acc[qi][0][0, h, i],
+                                               lp[0, h, i], 1.0, Op[0, h, i])
+                        acc[qi][0][0, h, i] = o
+                        acc[qi][1][0, h, i] = m + np.log(l)
+        for qi in (0, 1):
+            assert np.max(np.abs(acc[qi][0] - ch(Oref, mine[qi]))) <= 1e-12
+            assert np.max(np.abs(acc[qi][1] - ch(Lref, mine[qi]))) <= 1e-12
+
+
+def test_zigzag_folds_mark_first_and_last():
+    from exact_io_aware_46_b200.ring import zigzag_folds
+
+    for world in (1, 2, 4):
+        for rank in range(world):
+            folds = zigzag_folds(rank, world)
+            for qi in (0, 1):
+                mine = [f for f in folds if f[2] == qi]
+                assert mine[0][5] and not any(f[5] for f in mine[1:])
+                assert mine[-1][6] and not any(f[6] for f in mine[:-1])
+            assert [f[0] for f in folds] == sorted(f[0] for f in folds)  # step order
