@@ -26,6 +26,11 @@ sums of a chunk's dK and dV travel with that chunk (each rank adds its share
 before passing them on) and one extra pass at the end brings them home.  The sums
 are kept in fp32 by ``attn_accumulate``.
 
+For the causal mask there is also a zigzag layout (``ring_attn_fwd_zigzag``,
+``ring_attn_bwd_zigzag``): the sequence is cut into 2 * world chunks and rank r
+holds chunks r and 2 * world - 1 - r, which gives every rank the same work at
+every step.
+
 The exchange moves K/V (and gradient sums) between ranks and the kernels compute;
 there is no compute on the host and no fallback: ``ring_attn_fwd`` and
 ``ring_attn_bwd`` need the CUDA library.
@@ -286,3 +291,43 @@ def ring_attn_fwd_zigzag(q, k, v, group=None, scale=None):
         if s + 1 < world:
             ex.finish()
     return tuple(O), tuple(lse_acc)
+
+
+def ring_attn_bwd_zigzag(q, k, v, o, do, lse, group=None, scale=None):
+    """Causal ring-attention backward in the zigzag layout.  q, o, do, lse, k,
+    v: pairs (this rank's early and late chunk) shaped as in ``ring_attn_bwd``,
+    o and lse from ``ring_attn_fwd_zigzag``.  Returns (dQ pair, dK pair, dV pair)
+    bf16.  The running sums of the held chunks' dK and dV (four fp32 tensors)
+    travel with the K/V pair."""
+    from . import attn_accumulate
+
+    if not q[0].is_cuda:
+        raise ValueError("ring_attn_bwd_zigzag runs on the CUDA kernels")
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    steps = ring_steps_zigzag(rank, world)  # the pair list rides in the "kind" slot
+    dq_acc = [torch.empty(t.shape, dtype=torch.float32, device=t.device) for t in q]
+    first = [True, True]
+
+    def compute(pairs, src, kv_held):
+        k0, k1, v0, v1 = kv_held
+        return [(qi, ki, bwd_chunk(q[qi], (k0, k1)[ki], (v0, v1)[ki], o[qi], do[qi], lse[qi],
+                                   kind, scale=scale)) for qi, ki, kind in pairs]
+
+    def add(parts, g):
+        for qi, ki, (dqp, dkp, dvp) in parts:
+            attn_accumulate(dqp, dq_acc[qi], init=first[qi])
+            first[qi] = False
+            attn_accumulate(dkp, g[ki], init=False)
+            attn_accumulate(dvp, g[2 + ki], init=False)
+
+    zeros = tuple(torch.zeros(t.shape, dtype=torch.float32, device=t.device)
+                  for t in (k[0], k[1], v[0], v[1]))
+    g = ring_bwd_pass((k[0], k[1], v[0], v[1]), zeros, steps, compute, add, group)
+    dq = tuple(torch.empty_like(t) for t in q)
+    dk = tuple(torch.empty_like(t) for t in k)
+    dv = tuple(torch.empty_like(t) for t in v)
+    for acc, out in zip((dq_acc[0], dq_acc[1], g[0], g[1], g[2], g[3]),
+                        (dq[0], dq[1], dk[0], dk[1], dv[0], dv[1])):
+        attn_accumulate(None, acc, init=False, out=out)
+    return dq, dk, dv

@@ -247,3 +247,49 @@ def test_ring_zigzag_decomposition_matches_whole_sequence(world, Hq, Hkv, Lc):
         for qi in (0, 1):
             assert_out_close(to_f64(O[qi]), ch(Oref, mine[qi]), f"O[rank {rank}, chunk {qi}]")
             assert_lse_close(to_f64(lacc[qi]), ch(Lref, mine[qi]))
+
+
+@pytest.mark.parametrize("world,Hq,Hkv,Lc", [(2, 4, 2, 140), (3, 2, 2, 100)])
+def test_ring_zigzag_backward_matches_whole_sequence(world, Hq, Hkv, Lc):
+    """Zigzag backward decomposition: every rank's pairs (bwd_chunk from the
+    whole-sequence O and LSE) summed in fp32, each key chunk's dK/dV over every
+    rank, against the oracle's whole-sequence gradients."""
+    import torch
+
+    from exact_io_aware_46_b200.ring import bwd_chunk, ring_steps_zigzag, zigzag_chunks
+
+    attn = _lib()
+    d = 128
+    L = 2 * world * Lc
+    seed = 9900 + world * 10 + Lc
+    Q = synth.normal_bf16(seed * 8 + 1, (1, Hq, L, d))
+    K = synth.normal_bf16(seed * 8 + 2, (1, Hkv, L, d))
+    V = synth.normal_bf16(seed * 8 + 3, (1, Hkv, L, d))
+    dO = synth.normal_bf16(seed * 8 + 4, (1, Hq, L, d))
+    q, k, v, do = (dev_bf16(x) for x in (Q, K, V, dO))
+    scale = 1.0 / math.sqrt(d)
+    O, Lse = attn.attn_fwd(q, k, v, scale=scale, causal=True)
+    rQ, rK, rV = oracle.bwd(Q, K, V, dO, scale, causal=True)
+    ch = lambda t, c: t[:, :, c * Lc:(c + 1) * Lc].contiguous()
+    n = 2 * world
+    dq_acc = [torch.empty((1, Hq, Lc, d), device="cuda") for _ in range(n)]
+    dk_acc = [torch.zeros((1, Hkv, Lc, d), device="cuda") for _ in range(n)]
+    dv_acc = [torch.zeros((1, Hkv, Lc, d), device="cuda") for _ in range(n)]
+    started = set()
+    for rank in range(world):
+        mine = zigzag_chunks(rank, world)
+        for _, src, pairs in ring_steps_zigzag(rank, world):
+            held = zigzag_chunks(src, world)
+            for qi, ki, kind in pairs:
+                a, b = mine[qi], held[ki]
+                dqp, dkp, dvp = bwd_chunk(ch(q, a), ch(k, b), ch(v, b), ch(O, a), ch(do, a),
+                                          ch(Lse, a), kind, scale=scale)
+                attn.attn_accumulate(dqp, dq_acc[a], init=a not in started)
+                started.add(a)
+                attn.attn_accumulate(dkp, dk_acc[b], init=False)
+                attn.attn_accumulate(dvp, dv_acc[b], init=False)
+    torch.cuda.synchronize()
+    from tests._util import GRAD_REL_L2, rel_l2
+    for got, ref, what in ((torch.cat(dq_acc, 2), rQ, "dQ"), (torch.cat(dk_acc, 2), rK, "dK"),
+                           (torch.cat(dv_acc, 2), rV, "dV")):
+        assert rel_l2(to_f64(got), ref) <= GRAD_REL_L2, f"{what}: {rel_l2(to_f64(got), ref):.3e}"

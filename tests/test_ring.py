@@ -238,3 +238,51 @@ def test_zigzag_folds_mark_first_and_last():
                 assert mine[0][5] and not any(f[5] for f in mine[1:])
                 assert mine[-1][6] and not any(f[6] for f in mine[:-1])
             assert [f[0] for f in folds] == sorted(f[0] for f in folds)  # step order
+
+
+def _zigzag_bwd_main(rank, world, port, out):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from exact_io_aware_46_b200.ring import ring_bwd_pass
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    mine = zigzag_chunks(rank, world)
+    steps = ring_steps_zigzag(rank, world)
+
+    def compute(pairs, src, kv_held):
+        held = zigzag_chunks(src, world)
+        assert [float(kv_held[i][0]) for i in (0, 1)] == [float(c) for c in held]
+        return [(ki, float(mine[qi] + 1)) for qi, ki, _ in pairs]
+
+    def add(parts, g):
+        for ki, val in parts:
+            g[ki] += val
+
+    kv = tuple(torch.full((4,), float(c)) for c in mine)
+    sums = ring_bwd_pass(kv, (torch.zeros(4), torch.zeros(4)), steps, compute, add)
+    dist.barrier()
+    dist.destroy_process_group()
+    with open(out + f".{rank}", "w") as f:
+        f.write(repr([float(t[0]) for t in sums]))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_zigzag_backward_sums_travel_home(tmp_path, world):
+    """Zigzag backward routing: every query chunk a adds a + 1 to the sums of each
+    key chunk b <= a it meets; after the closing pass a rank holds, for each of
+    its two chunks b, the total over a >= b."""
+    import torch.multiprocessing as mp
+
+    out = str(tmp_path / "z")
+    mp.start_processes(_zigzag_bwd_main, args=(world, _free_port(), out), nprocs=world,
+                       join=True, start_method="spawn")
+    for rank in range(world):
+        got = eval(open(out + f".{rank}").read())
+        want = [float(sum(a + 1 for a in range(b, 2 * world))) for b in zigzag_chunks(rank, world)]
+        assert got == want
