@@ -169,3 +169,34 @@ def test_product_path_does_not_touch_oracle():
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
                 assert "attn_oracle" not in txt, f
+
+
+def test_binding_refuses_host_tensors():
+    """No CPU fallback: every entry point of the binding (and the ring drivers)
+    rejects host tensors before anything runs."""
+    import torch
+
+    import exact_io_aware_46_b200 as attn
+    from exact_io_aware_46_b200 import ring
+
+    b = torch.zeros((1, 2, 8, 128), dtype=torch.bfloat16)
+    f = torch.zeros((1, 2, 8, 128), dtype=torch.float32)
+    l = torch.zeros((1, 2, 8), dtype=torch.float32)
+    u8 = torch.zeros((1, 2, 8, 128), dtype=torch.uint8)
+    s = torch.ones((1, 2, 1), dtype=torch.float32)
+    calls = [
+        lambda: attn.attn_fwd(b, b, b),
+        lambda: attn.attn_fwd_sliding(b, b, b, 4),
+        lambda: attn.attn_bwd(b, b, b, b, b, l),
+        lambda: attn.attn_fwd_fp8(u8, u8, u8, s, s, s),
+        lambda: attn.attn_fwd_merge(b, b, b, f, l, init=True),
+        lambda: attn.attn_merge_partial(b, l, f, l, init=True),
+        lambda: attn.attn_accumulate(b, f, init=True),
+        lambda: ring.ring_attn_fwd(b, b, b),
+        lambda: ring.ring_attn_bwd(b, b, b, b, b, l),
+        lambda: ring.ring_attn_fwd_zigzag((b, b), (b, b), (b, b)),
+        lambda: ring.ring_attn_bwd_zigzag((b, b), (b, b), (b, b), (b, b), (b, b), (l, l)),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError):
+            call()
