@@ -19,8 +19,8 @@
  *   Q, O, dO, dQ: [B, Hq, Lq, d]; K, V, dK, dV: [B, Hkv, Lk, d];
  *   LSE: [B, Hq, Lq] fp32.  Query head h reads key/value head h / (Hq / Hkv)
  *   (grouped-query attention; Hq must be a multiple of Hkv).
- * - d (head dimension) must be 64 or 128; anything else returns
- *   ATTN_ERR_UNSUPPORTED.  There is no fallback path of any kind.
+ * - d (head dimension) must be 64 or 128 (the 8-bit forward: 128); anything
+ *   else returns ATTN_ERR_UNSUPPORTED.  There is no fallback path of any kind.
  * - All device pointers must be 16-byte aligned (the tensor-memory-accelerator
  *   copies require it) and must not alias one another (except where stated).
  * - Masks: `mask_flags` = ATTN_MASK_NONE or ATTN_MASK_CAUSAL.  Causal is
@@ -40,10 +40,11 @@
  * - Errors: argument errors are detected on the host before anything is
  *   launched and return ATTN_ERR_INVALID or ATTN_ERR_UNSUPPORTED.  A failed
  *   launch returns ATTN_ERR_CUDA.  Errors found on the device (a k_lens entry
- *   outside [0, Lk], a paged-cache block-table entry outside [0, n_pages), an
- *   internal wait that timed out) set bits of a status
- *   word kept in the first 16 bytes of the workspace; the affected work units
- *   write zeros.  The word is sticky: read it with attn_read_device_status and
+ *   outside [0, Lk], a paged-cache block-table entry outside [0, n_pages), a
+ *   malformed packed-sequence offset, an 8-bit scale that is not finite and
+ *   positive, an internal wait that timed out) set bits of a status word kept
+ *   in the first 16 bytes of the workspace; the affected work units write
+ *   zeros (a bad 8-bit scale leaves its results undefined instead).  The word is sticky: read it with attn_read_device_status and
  *   clear it with attn_clear_device_status (a fresh workspace must be cleared
  *   once before first use).
  * - Workspace: each call has an *_workspace_size query; pass at least that
