@@ -569,3 +569,4 @@ def test_fp8_brute_force_against_torch():
     O, L = oracle.fwd_fp8(Q8, K8, V8, qs, ks, vs, 0.3, causal=True)
     assert np.max(np.abs(O - (torch.softmax(s, -1) @ v).numpy())) <= 1e-12
     assert np.max(np.abs(L - torch.logsumexp(s, -1).numpy())) <= 1e-12
+

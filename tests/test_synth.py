@@ -1,7 +1,9 @@
-"""The seeded input generator: determinism, distribution and bf16 rounding."""
+"""The seeded input generator: determinism, distribution, bf16 rounding and the
+8-bit (E4M3) input recipe."""
 
 import numpy as np
 
+import oracle
 import synth
 
 
@@ -35,3 +37,29 @@ def test_uniform_int_range():
     k = synth.uniform_int(9, 10000, 1024, 32768)
     assert k.min() >= 1024 and k.max() <= 32768
     assert abs(k.mean() - (1024 + 32768) / 2) < 400
+
+
+def test_e4m3_quantised_inputs_follow_the_recipe():
+    """The 8-bit input recipe: per 128-row tile, scale = the tile's largest
+    magnitude / 448 (its largest element becomes +-448 exactly) and every code
+    is within half an E4M3 step of x / scale (relative 2^-4 for normal values,
+    absolute 2^-10 in the subnormal range)."""
+    import torch
+
+    x = synth.bf16_bits_to_f64(synth.normal_bf16(951, (2, 3, 300, 64)))
+    codes, scales = synth.normal_e4m3(951, (2, 3, 300, 64))
+    assert codes.dtype == np.uint8 and scales.shape == (2, 3, 3)
+    deq = oracle.e4m3_to_f64(codes)
+    for t in range(3):
+        rows = slice(128 * t, min(128 * (t + 1), 300))
+        xt = x[:, :, rows]
+        amax = np.max(np.abs(xt), axis=(2, 3))
+        assert np.allclose(scales[:, :, t], (amax / 448.0).astype(np.float32), rtol=1e-7)
+        assert np.max(np.abs(deq[:, :, rows]), axis=(2, 3)).tolist() == [[448.0] * 3] * 2
+        y = xt / scales[:, :, t][..., None, None].astype(np.float64)
+        err = np.abs(deq[:, :, rows] - y)
+        bound = np.maximum(np.abs(y) * 2.0 ** -4, 2.0 ** -10) * (1 + 1e-6)
+        assert np.all(err <= bound)
+    # the device twin quantises the same values the same way
+    c2, s2 = synth.quantize_e4m3_tiles(torch.from_numpy(x.astype(np.float32)))
+    assert np.array_equal(c2.numpy(), codes) and np.array_equal(s2.numpy(), scales)
