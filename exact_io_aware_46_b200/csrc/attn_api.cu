@@ -9,14 +9,13 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
-#include <set>
-#include <tuple>
 
 #include "../../include/attn.h"
 #include "accum_kernel.cuh"
 #include "bwd_kernel.cuh"
 #include "decode_kernel.cuh"
 #include "fwd_kernel.cuh"
+#include "launch_cache.cuh"
 #include "merge_kernel.cuh"
 #include "pad_kernel.cuh"
 
@@ -111,23 +110,7 @@ bool shapes_ok(int B, int Hq, int Hkv, int Lq, int Lk) {
   return true;
 }
 
-// Raises a kernel's dynamic shared-memory limit once per (kernel, device, size):
-// repeated launches then make no attribute call, which also keeps launches that
-// are being captured into a CUDA graph free of non-stream API calls.
-template <typename K>
-cudaError_t set_smem(K kernel, int bytes) {
-  static std::mutex mu;
-  static std::set<std::tuple<const void*, int, int>> done;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-  const auto key = std::make_tuple(reinterpret_cast<const void*>(kernel), dev, bytes);
-  std::lock_guard<std::mutex> lock(mu);
-  if (done.count(key)) return cudaSuccess;
-  const cudaError_t e =
-      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) done.insert(key);
-  return e;
-}
+using attn_host::set_smem;
 
 }  // namespace
 

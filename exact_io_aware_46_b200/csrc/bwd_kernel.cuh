@@ -29,6 +29,7 @@
 //  3. convert: dQ = bf16(scale * accumulator).
 #pragma once
 
+#include "launch_cache.cuh"
 #include "sm100.cuh"
 
 namespace attn_bwd_impl {
@@ -693,8 +694,7 @@ inline attn_status_t launch(const Args& a, cudaStream_t s) {
         !make_tmap_rows(&tk, a.K, a.Lk, static_cast<long long>(a.B) * a.Hkv, BN) ||
         !make_tmap_rows(&tv, a.V, a.Lk, static_cast<long long>(a.B) * a.Hkv, BN))
       return ATTN_ERR_CUDA;
-    if (cudaFuncSetAttribute(bwd_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
+    if (attn_host::set_smem(bwd_main_kernel, SMEM_BYTES) != cudaSuccess)
       return ATTN_ERR_CUDA;
     const int grid = p.n_items < a.sms ? p.n_items : a.sms;
     bwd_main_kernel<<<grid, NTHREADS, SMEM_BYTES, s>>>(tq, tdo, tk, tv, p);

@@ -23,6 +23,7 @@
 //    weights: O = sum_c e^{LSE_c - M} O_c / sum_c e^{LSE_c - M}.
 #pragma once
 
+#include "launch_cache.cuh"
 #include "sm100.cuh"
 
 namespace attn_decode_impl {
@@ -184,9 +185,11 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) decode_split_kernel(con
       const uint8_t* gV = reinterpret_cast<const uint8_t*>(p.V);
       const size_t head_row0 = (static_cast<size_t>(b) * p.Hkv + hkv) * p.Lmax + k0;
       const int page = 1 << p.page_log2;
+      int issued = 0;  // stages whose copies were issued
       for (int s = 0; s < nstages; ++s) {
         const int slot = s % NST;
         if (!sm100::mbar_wait(&empty[slot], ((s / NST) & 1) ^ 1, abort_flag, p.status)) break;
+        ++issued;
         const int n = min(SR, rows - s * SR);
         const uint32_t bytes = static_cast<uint32_t>(n * ROWB);
         sm100::mbar_arrive_expect_tx(&full[slot], 2 * bytes);
@@ -213,6 +216,12 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) decode_split_kernel(con
           }
         }
       }
+      // the CTA must not exit while bulk copies still write into its shared
+      // memory, which can happen once a wait has expired (the compute warps
+      // then stop reading the ring): wait, bounded, for the last issued stage
+      // of every slot (in normal operation these have long landed)
+      for (int s = issued - 1; s >= 0 && s >= issued - NST; --s)
+        sm100::mbar_wait_drain(&full[s % NST], (s / NST) & 1);
     }
     return;  // the producer takes no part in the merge below
   }
@@ -356,8 +365,19 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) decode_split_kernel(con
       o2[g][c].x += __shfl_xor_sync(0xffffffffu, o2[g][c].x, 16);
       o2[g][c].y += __shfl_xor_sync(0xffffffffu, o2[g][c].y, 16);
     }
-  // all stages are consumed: reuse the K ring for the per-warp partials
+  // all stages are consumed: reuse the K ring for the per-warp partials --
+  // unless a wait expired (every compute warp that stopped early set the
+  // abort flag before this barrier): bulk copies may then still be landing in
+  // the ring, so the chunk contributes an empty partial written directly
   sm100::named_bar_sync(1, NCW * 32);
+  if (*abort_flag) {
+    for (int e = threadIdx.x; e < p.G * D; e += NCW * 32) {
+      const size_t ph = (static_cast<size_t>(b) * p.Hq + hkv * p.G + e / D) * p.nsm + chunk;
+      p.part_o[ph * D + e % D] = 0.f;
+      if (e % D == 0) p.part_lse[ph] = -INFINITY;
+    }
+    return;
+  }
   float* wm = reinterpret_cast<float*>(sK);        // [NCW][GP]
   float* wl = wm + NCW * GP;                       // [NCW][GP]
   float* wo = wl + NCW * GP;                       // [NCW][GP][D]
@@ -432,8 +452,7 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const CombineParams p
 template <int D, int GP>
 cudaError_t launch_t(const SplitParams& sp, const CombineParams& cp, cudaStream_t s) {
   constexpr int smem = smem_bytes<D>();
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, GP>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = attn_host::set_smem(decode_split_kernel<D, GP>, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(sp.nsm, sp.Hkv, sp.B);
   decode_split_kernel<D, GP><<<grid, NTHREADS, smem, s>>>(sp);
