@@ -2,20 +2,21 @@
 // memory.
 //
 // attn_fwd_splitkv_decode needs a caller-provided workspace for its fp32
-// per-chunk partials.  Some callers have no way to provide one: code that runs
-// while a stream is being captured into a CUDA graph (where a cudaMalloc would
-// break the capture), runtimes that hand the library only the tensors they
-// already own (a fixed memory plan with no scratch pool to draw from), and
-// latency-critical loops where an allocation's implicit synchronisation is not
-// acceptable.  attn_fwd_splitkv_decode_noalloc serves them: the same two
-// kernels, with the partials in a fixed, file-scope device array instead of a
-// workspace.
+// per-chunk partials.  Some callers have no way to provide one: runtimes that
+// hand the library only the tensors they already own (a memory plan fixed up
+// front, with no scratch pool to draw from), host frameworks whose operator
+// interface passes tensors but no allocator, and latency-critical loops where
+// a cudaMalloc's implicit device synchronisation is not acceptable.
+// attn_fwd_splitkv_decode_noalloc serves them: the same two kernels, with the
+// partials in a fixed, file-scope device array instead of a workspace.
 //
 // The array is static device memory: every GPU that loads the library holds
 // ATTN_NOALLOC_SCRATCH_BYTES of it until the process exits.  In host code the
 // array's name is only a host-side stand-in for the symbol, not a device
-// address, so the real address is obtained once per device with
-// cudaGetSymbolAddress (with that device current) and passed to the kernels.
+// address, so the real address is looked up with cudaGetSymbolAddress (with
+// the device current) and passed to the kernels.  The lookup is done once per
+// device and CUDA context and repeated when the context changes (after a
+// cudaDeviceReset the old address is no longer valid).
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -34,21 +35,30 @@ namespace {
 constexpr size_t kHeader = 256;
 constexpr int kMaxDevices = 64;
 
-std::mutex g_mutex;
-uint8_t* g_addr[kMaxDevices] = {};
+struct ScratchSlot {
+  uint8_t* addr = nullptr;
+  unsigned long long ctx = 0;  // context the address was looked up in
+};
 
-// Device address of the scratch array on the current device, resolved on the
-// first call for that device; nullptr if the lookup fails.
+std::mutex g_mutex;
+ScratchSlot g_slot[kMaxDevices];
+
+// Device address of the scratch array in the current device's current
+// context; looked up on the first call there and again whenever the context
+// has changed (or cannot be identified); nullptr if the lookup fails.
 uint8_t* scratch_for_current_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (!g_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
-    g_addr[dev] = static_cast<uint8_t*>(p);
-  }
-  return g_addr[dev];
+  ScratchSlot& slot = g_slot[dev];
+  const unsigned long long ctx = attn_host::current_context_id();
+  if (slot.addr && ctx != 0 && ctx == slot.ctx) return slot.addr;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+  slot.addr = static_cast<uint8_t*>(p);
+  // the lookup creates the primary context if there was none yet
+  slot.ctx = attn_host::current_context_id();
+  return slot.addr;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -290,28 +290,32 @@ attn_status_t attn_bwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf
 /* ------------------------------------------------------------------ decode without allocation
  * No counterpart in the pages: an interface addition for callers that cannot
  * allocate device memory.  attn_fwd_splitkv_decode needs a workspace for its
- * fp32 per-chunk partials; callers that cannot hand one over (code running
- * while a stream is being captured into a CUDA graph, where an allocation would
- * break the capture; runtimes with a fixed memory plan that only pass the
- * tensors they own; latency-critical loops that must not pay an allocation's
- * implicit synchronisation) use this variant instead.  It computes exactly what
- * attn_fwd_splitkv_decode computes, with the same kernels and arguments minus
- * the workspace.
+ * fp32 per-chunk partials; some callers cannot hand one over: runtimes whose
+ * memory plan is fixed up front and that pass only the tensors they own (no
+ * scratch pool to draw from), host frameworks whose operator interface gives
+ * tensors but no allocator, and latency-critical loops that must not pay a
+ * cudaMalloc's implicit device synchronisation.  They use this variant
+ * instead.  It computes exactly what attn_fwd_splitkv_decode computes, with
+ * the same kernels and arguments minus the workspace.
  *
  * Scratch: a file-scope device array of ATTN_NOALLOC_SCRATCH_BYTES that every
  * GPU loading the library holds until the process exits.  A request whose
  * partials need more (256 + B*Hq*ceil(Lmax/2048)*(4*d + 4) bytes, rounded up to
  * 256) returns ATTN_ERR_CAPACITY before anything is launched.  The first call
  * on a device looks up the array's device address (cudaGetSymbolAddress, with
- * that device current); make that first call before any stream capture.  The
- * call allocates and frees nothing.
+ * that device current) and raises the kernels' shared-memory limit; make that
+ * first call before any stream capture.  The set-up is repeated when the
+ * device's CUDA context changes (after cudaDeviceReset, the next call is a
+ * first call again).  The call allocates and frees nothing.
  *
  * All calls share the one array: calls that may overlap on the GPU (different
  * streams, or different host threads on one device) race and corrupt each
  * other's results; serialise them.  Each call clears the status word it keeps
- * at the head of the array; the partials need no clearing.  Device-side errors
- * (a k_lens entry outside [0, Lmax]) zero the affected outputs but are not
- * reported (there is no workspace to read them from).
+ * at the head of the array; the partials need no clearing.  Device-side
+ * errors are not reported (there is no workspace to read a status from):
+ * a k_lens entry outside [0, Lmax] zeroes that sequence's outputs, and a wait
+ * that expired makes its chunk contribute nothing, so O and LSE are then
+ * partial results although the call returned ATTN_OK.
  */
 #define ATTN_NOALLOC_SCRATCH_BYTES (16u << 20)
 attn_status_t attn_fwd_splitkv_decode_noalloc(const attn_bf16_t* Q, const attn_bf16_t* Kcache,

@@ -1,8 +1,9 @@
 """attn_fwd_splitkv_decode_noalloc: decode for callers that cannot allocate.
 
-Callers that run while a stream is captured into a CUDA graph, or inside a
-runtime with a fixed memory plan, cannot hand the library a workspace.  The
-no-alloc entry point keeps its partials in a fixed device array instead.  It
+Callers inside a runtime whose device memory plan is fixed up front, or
+behind an operator interface that passes tensors but no allocator, cannot hand
+the library a workspace.  The no-alloc entry point keeps its partials in a
+fixed device array instead.  It
 must give the same output as the workspace entry point, call after call (the
 array keeps the previous call's contents, which must not leak into the next
 result).
