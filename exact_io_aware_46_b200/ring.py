@@ -67,7 +67,16 @@ class RingExchange:
     """Double-buffered ring pass of a tuple of tensors: ``start()`` posts the
     send of the held tensors to rank + 1 and the receive of the next ones from
     rank - 1; ``finish()`` waits for both and makes the received tensors the
-    held ones.  Works on any backend with point-to-point operations."""
+    held ones.  Works on any backend with point-to-point operations.
+
+    NCCL moves CUDA tensors device to device (over NVLink between GPUs).  A
+    gloo group cannot send CUDA tensors, so there the pass is staged through
+    pinned host buffers: ``start()`` copies the held tensors to the host (after
+    the work already queued on the current stream, which wrote them) and sends
+    the bytes; ``finish()`` copies what arrived back into the device buffer.
+    The staged path exists for process groups without a device transport (and
+    for testing the drivers with several processes on one GPU); its host copies
+    are not overlapped with the compute."""
 
     def __init__(self, tensors, group=None):
         self.group = group
@@ -76,6 +85,12 @@ class RingExchange:
         self.cur = [t.contiguous() for t in tensors]
         self.nxt = [torch.empty_like(t) for t in self.cur]
         self.reqs = None
+        self.staged = (any(t.is_cuda for t in self.cur)
+                       and dist.get_backend(group) == dist.Backend.GLOO)
+        if self.staged:
+            pin = torch.cuda.is_available()
+            self.h_send = [torch.empty(t.shape, dtype=t.dtype, pin_memory=pin) for t in self.cur]
+            self.h_recv = [torch.empty(t.shape, dtype=t.dtype, pin_memory=pin) for t in self.cur]
 
     def _peer(self, r):
         return dist.get_global_rank(self.group, r) if self.group is not None else r
@@ -85,14 +100,24 @@ class RingExchange:
             raise RuntimeError("a ring step is already in flight")
         to = self._peer((self.rank + 1) % self.world)
         frm = self._peer((self.rank - 1) % self.world)
-        ops = [dist.P2POp(dist.isend, t, to, self.group) for t in self.cur]
-        ops += [dist.P2POp(dist.irecv, t, frm, self.group) for t in self.nxt]
+        send, recv = self.cur, self.nxt
+        if self.staged:
+            for h, t in zip(self.h_send, self.cur):
+                h.copy_(t)  # waits for the stream's writes of t
+            # bytes on the wire: the transport need not know the element type
+            send = [h.view(torch.uint8) for h in self.h_send]
+            recv = [h.view(torch.uint8) for h in self.h_recv]
+        ops = [dist.P2POp(dist.isend, t, to, self.group) for t in send]
+        ops += [dist.P2POp(dist.irecv, t, frm, self.group) for t in recv]
         self.reqs = dist.batch_isend_irecv(ops)
 
     def finish(self):
         for r in self.reqs:
             r.wait()
         self.reqs = None
+        if self.staged:
+            for t, h in zip(self.nxt, self.h_recv):
+                t.copy_(h)
         self.cur, self.nxt = self.nxt, self.cur
 
 
