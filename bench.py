@@ -423,6 +423,49 @@ def decode_leg(steps, warmup, world, flush):
     return ms, kv_bytes, k_lens, (page, pms)
 
 
+LONG = dict(B=1, Hq=32, Hkv=8, L=16384, d=128, klo=8192)
+
+
+def long_klen():
+    """The padding variant's valid key length, uniform in [8192, 16384] (seeded)."""
+    c = LONG
+    return int(synth.uniform_int(synth.workload_seed(3, "klen"), c["B"], c["klo"], c["L"])[0])
+
+
+def long_leg(steps, warmup, world, flush):
+    """Long-context causal forward B1 Hq32 Hkv8 (GQA) L16384 d128, and the same
+    with key padding (k_len ~ U[8192, 16384], seeded); FLOPs over visible pairs."""
+    import torch
+
+    import exact_io_aware_46_b200 as attn
+
+    c = LONG
+    dev = torch.device("cuda")
+    q = synth.normal_bf16_device(synth.workload_seed(3, "q"), (c["B"], c["Hq"], c["L"], c["d"]), dev)
+    k = synth.normal_bf16_device(synth.workload_seed(3, "k"), (c["B"], c["Hkv"], c["L"], c["d"]), dev)
+    v = synth.normal_bf16_device(synth.workload_seed(3, "v"), (c["B"], c["Hkv"], c["L"], c["d"]), dev)
+    O = torch.empty_like(q)
+    lse = torch.empty((c["B"], c["Hq"], c["L"]), dtype=torch.float32, device=dev)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    kl = long_klen()
+    k_lens = torch.full((c["B"],), kl, dtype=torch.int32, device=dev)
+    out = {}
+    for name, kls in (("causal", None), ("padded", k_lens)):
+        call = lambda kls=kls: attn.attn_fwd(q, k, v, causal=True, k_lens=kls, O=O, lse=lse,
+                                             workspace=ws, stream=stream)
+        barrier(world)
+        out[name] = timed_loop(call, steps, warmup, stream, flush)
+        st = attn.attn_read_device_status(ws)
+        if st[0] != attn.ATTN_OK:
+            raise RuntimeError(f"device status {st}")
+    flops = {"causal": 4.0 * c["d"] * causal_pairs(c["L"], c["L"], True) * c["B"] * c["Hq"],
+             "padded": 4.0 * c["d"] * causal_pairs(c["L"], c["L"], True, kl) * c["B"] * c["Hq"]}
+    del q, k, v, O, lse
+    torch.cuda.empty_cache()
+    return out, flops, kl
+
+
 RING = dict(world=4, B=1, Hq=32, Hkv=8, L=16384, d=128)
 
 
@@ -626,59 +669,154 @@ def bwd_leg(steps, warmup, world, flush):
 
 
 # ------------------------------------------------------------------ CPU baseline (oracle)
+# The fp64 oracle, as it stands, on the host cores, on the workloads' own input
+# values (each sampled head drawn at its counters in the same seeded streams the
+# GPU legs use).  One sampling unit per workload, shared by the cpu_baseline
+# entries and by the reference arm:
+#   forward (B4 H16 L4096 d128, causal): unit u = query rows i = u mod 16,
+#     u mod 16 + 16, ... (256 rows) of head u // 16 (a (b, h) index): 256 rows
+#     per call keep every host core busy (the oracle runs its rows in parallel);
+#   long context (B1 Hq32 Hkv8 L16384 d128, causal, with and without padding):
+#     whole query heads, taken in order; the rate is FLOPs of the visible pairs
+#     computed over time, so the heads not run are "scaled" by the per-head rate;
+#   decode (B64 Hq32 Hkv8 d128, k_len ~ U[1024, 32768]): whole sequences (all 32
+#     query heads over the sequence's k_len keys), bytes = its K and V rows;
+#   backward (B2 H16 L8192 d128, causal): whole heads through oracle.bwd.
 
 
-def cpu_baseline(budget_s=12.0):
-    """The fp64 oracle on the host cores, on a bounded sample of the forward
-    workload: every 16th query row of head (0, 0), scaled by visible pairs."""
+def _head(workload, tensor, shape, bh):
+    return synth.normal_bf16_block(synth.workload_seed(workload, tensor), shape, bh)
+
+
+_FWD_HEAD = {}
+
+
+def oracle_fwd_unit(u):
+    """Runs forward sampling unit ``u`` on the oracle; returns (seconds, FLOPs)."""
     import oracle
 
     c = FWD
+    L, d, H = c["L"], c["d"], c["Hq"]
+    shp = (c["B"], c["Hq"], L, d)
+    h = (u // 16) % (c["B"] * H)
+    if h not in _FWD_HEAD:  # the 16 units of a head share its inputs (drawn untimed)
+        _FWD_HEAD.clear()
+        bh = (h // H, h % H)
+        _FWD_HEAD[h] = tuple(_head(2, x, shp, bh)[None, None] for x in ("q", "k", "v"))
+    Q, K, V = _FWD_HEAD[h]
+    rows = np.arange(u % 16, L, 16, dtype=np.int32)
+    t0 = time.perf_counter()
+    oracle.fwd(Q, K, V, 1 / math.sqrt(d), causal=True, rows=rows)
+    dt = time.perf_counter() - t0
+    return dt, 4.0 * d * float(np.sum(rows + 1))
+
+
+def cpu_baseline_fwd(budget_s=10.0):
+    import oracle
+
+    t, fl, u = 0.0, 0.0, 0
+    while t < budget_s and u < 4096:
+        dt, f = oracle_fwd_unit(u)
+        t += dt
+        fl += f
+        u += 1
+    return {"value": fl / t / 1e12, "unit": "TFLOP/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{u} units of 256 query rows (rows = u mod 16 + 16 k of one (b, h) head, "
+                      f"heads in order) of the causal B4 H16 L4096 d128 forward, fp64, "
+                      f"{t:.1f} s of oracle time; the reference arm times the same units"}
+
+
+def cpu_baseline_long(budget_s=8.0, padded=False):
+    import oracle
+
+    c = LONG
     L, d = c["L"], c["d"]
-    Q = synth.normal_bf16(synth.workload_seed(2, "q") ^ 0x55, (1, 1, L, d))
-    K = synth.normal_bf16(synth.workload_seed(2, "k") ^ 0x55, (1, 1, L, d))
-    V = synth.normal_bf16(synth.workload_seed(2, "v") ^ 0x55, (1, 1, L, d))
-    stride = 16
-    done_flops, t_used, reps = 0.0, 0.0, 0
-    while t_used < budget_s and reps < 4096:
-        rows = np.arange(reps % stride, L, stride, dtype=np.int32)
+    G = c["Hq"] // c["Hkv"]
+    kl = int(long_klen()) if padded else L
+    t, fl, n = 0.0, 0.0, 0
+    while t < budget_s and n < c["Hq"]:
+        Q = _head(3, "q", (1, c["Hq"], L, d), (0, n))[None, None]
+        K = _head(3, "k", (1, c["Hkv"], L, d), (0, n // G))[None, None]
+        V = _head(3, "v", (1, c["Hkv"], L, d), (0, n // G))[None, None]
         t0 = time.perf_counter()
-        oracle.fwd(Q, K, V, 1 / math.sqrt(d), causal=True, rows=rows)
-        t_used += time.perf_counter() - t0
-        done_flops += 4.0 * d * float(np.sum(rows + 1))
-        reps += 1
-    return {"value": done_flops / t_used / 1e12, "unit": "TFLOP/s", "cores": oracle.threads(),
-            "kind": "oracle",
-            "sample": f"{reps} x {L // stride} query rows (every {stride}th) of one "
-                      f"(b,h) head of the causal B4 H16 L4096 d128 forward, fp64, "
-                      f"{t_used:.1f} s of CPU time"}
+        oracle.fwd(Q, K, V, 1 / math.sqrt(d), causal=True,
+                   k_lens=np.array([kl], dtype=np.int32) if padded else None)
+        t += time.perf_counter() - t0
+        fl += 4.0 * d * causal_pairs(L, L, True, kl)
+        n += 1
+    what = f", key padding k_len = {kl}" if padded else ""
+    return {"value": fl / t / 1e12, "unit": "TFLOP/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{n} of {c['Hq']} query heads (whole heads, all {L} rows) of the causal "
+                      f"B1 Hq32 Hkv8 L16384 d128 forward{what}, fp64, {t:.1f} s; scaled: the "
+                      f"rate of these heads stands for all {c['Hq']}"}
+
+
+def cpu_baseline_decode(k_lens, budget_s=3.0):
+    import oracle
+
+    c = DEC
+    d, Hq, Hkv = c["d"], c["Hq"], c["Hkv"]
+    t, nbytes, n = 0.0, 0.0, 0
+    while t < budget_s and n < c["B"]:
+        kl = int(k_lens[n])
+        Q = _head(4, "q", (c["B"], Hq, 1, d), (n,))[None]
+        # the sequence's cache rows [0, k_len) of every kv head
+        shp = (c["B"], Hkv, c["Lmax"], d)
+        K = np.stack([synth.normal_bf16_block(synth.workload_seed(4, "k"), shp, (n, h), first=kl)
+                      for h in range(Hkv)])
+        V = np.stack([synth.normal_bf16_block(synth.workload_seed(4, "v"), shp, (n, h), first=kl)
+                      for h in range(Hkv)])
+        t0 = time.perf_counter()
+        oracle.fwd(Q, K[None], V[None], 1 / math.sqrt(d))
+        t += time.perf_counter() - t0
+        nbytes += 2.0 * Hkv * kl * d * 2
+        n += 1
+    return {"value": nbytes / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} of {c['B']} sequences (all {Hq} query heads over the sequence's "
+                      f"k_len cache rows; {nbytes / 1e9:.3f} GB of K and V) of the split-KV decode "
+                      f"B64 Hq32 Hkv8 d128, fp64, {t:.1f} s; the oracle computes one query row "
+                      f"per head, so one host thread works"}
+
+
+def cpu_baseline_bwd(budget_s=8.0):
+    import oracle
+
+    c = BWD
+    L, d = c["L"], c["d"]
+    shp = (c["B"], c["Hq"], L, d)
+    t, fl, n = 0.0, 0.0, 0
+    while t < budget_s and n < c["B"] * c["Hq"]:
+        bh = (n // c["Hq"], n % c["Hq"])
+        Q, K, V, dO = (_head(5, x, shp, bh)[None, None] for x in ("q", "k", "v", "do"))
+        t0 = time.perf_counter()
+        oracle.bwd(Q, K, V, dO, 1 / math.sqrt(d), causal=True)
+        t += time.perf_counter() - t0
+        fl += 10.0 * d * causal_pairs(L, L, True)
+        n += 1
+    return {"value": fl / t / 1e12, "unit": "TFLOP/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{n} of {c['B'] * c['Hq']} (b, h) heads (whole heads, all {L} rows: dQ, dK, "
+                      f"dV) of the causal backward B2 H16 L8192 d128, fp64, {t:.1f} s; scaled: "
+                      f"the rate of these heads stands for all"}
 
 
 def reference_arm(args, rank, world):
-    """--impl reference: the oracle, as it stands, on this machine's host cores."""
+    """--impl reference: the oracle, as it stands, on this machine's host cores: each
+    step is the next forward sampling unit (the units of cpu_baseline_fwd)."""
     if rank != 0:
         return
     steps, warmup = args.steps, args.warmup
     import oracle
 
-    c = FWD
-    L, d = c["L"], c["d"]
-    Q = synth.normal_bf16(synth.workload_seed(2, "q") ^ 0x55, (1, 1, L, d))
-    K = synth.normal_bf16(synth.workload_seed(2, "k") ^ 0x55, (1, 1, L, d))
-    V = synth.normal_bf16(synth.workload_seed(2, "v") ^ 0x55, (1, 1, L, d))
-    stride = 64
     times, flops = [], []
     for it in range(warmup + steps):
-        rows = np.arange(it % stride, L, stride, dtype=np.int32)
-        t0 = time.perf_counter()
-        oracle.fwd(Q, K, V, 1 / math.sqrt(d), causal=True, rows=rows)
-        dt = time.perf_counter() - t0
+        dt, f = oracle_fwd_unit(it)
         if it >= warmup:
             times.append(dt)
-            flops.append(4.0 * d * float(np.sum(rows + 1)))
+            flops.append(f)
     val = sum(flops) / sum(times) / 1e12
-    sample = (f"each step: {L // stride} query rows (every {stride}th) of one head of the causal "
-              f"B4 H16 L4096 d128 forward, fp64 oracle")
+    sample = ("each step: one unit of 256 query rows (rows = u mod 16 + 16 k of one (b, h) head) "
+              "of the causal B4 H16 L4096 d128 forward, fp64 oracle (the units of the "
+              "cpu_baseline entry)")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": steps, "warmup": warmup,
@@ -702,8 +840,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--legs", default="fwd,decode,bwd,ring",
-                    help="comma list of fwd, decode, bwd (subsets are for profiling runs)")
+    ap.add_argument("--legs", default="fwd,decode,bwd,long,ring",
+                    help="comma list of fwd, decode, bwd, long, ring (subsets are for profiling "
+                         "runs)")
     ap.add_argument("--decode-lmax", type=int, default=DEC["Lmax"],
                     help="smaller KV cache for profiling captures (k_len ~ U[1024, Lmax])")
     args = ap.parse_args()
@@ -734,11 +873,13 @@ def main():
             (ms, ms_e2e, h2d, d2h, (vms, vflops, vtotal),
              (W, wms, wflops), fms) = fwd_leg(args.steps, args.warmup, world, flush)
         if "decode" in legs:
-            dms, kv_bytes, _, (page, pms) = decode_leg(args.steps, args.warmup, world, flush)
+            dms, kv_bytes, dec_klens, (page, pms) = decode_leg(args.steps, args.warmup, world,
+                                                               flush)
         if "bwd" in legs:
             bms = bwd_leg(max(3, args.steps // 2), args.warmup, world, flush)
         else:
             bms = None
+        lng = long_leg(args.steps, args.warmup, world, flush) if "long" in legs else None
         ring = ring_leg(args.steps, args.warmup, world, flush) if "ring" in legs else None
     clocks = clk.summary()
     if "fwd" not in legs:  # profiling runs of single legs: report what ran
@@ -750,6 +891,10 @@ def main():
         if bms is not None:
             rep["bwd_ms"] = float(np.mean(bms))
             rep["bwd_TFLOPs"] = bwd_flops(BWD) / (float(np.mean(bms)) * 1e-3) / 1e12
+        if lng is not None:
+            for name in ("causal", "padded"):
+                rep[f"long_{name}_ms"] = float(np.mean(lng[0][name]))
+                rep[f"long_{name}_TFLOPs"] = lng[1][name] / (float(np.mean(lng[0][name])) * 1e-3) / 1e12
         if ring is not None:
             rep["ring_ms"] = float(np.mean(ring[0]))
             rep["ring_TFLOPs"] = ring[1] / (float(np.mean(ring[0])) * 1e-3) / 1e12
@@ -859,6 +1004,25 @@ def main():
                          "traffic": traffic_per_launch("attn_bwd_impl::bwd_main_kernel")},
         }
         line["gpu_launches"] += 3 * max(3, args.steps // 2)
+    if lng is not None:
+        lms, lflops, kl = lng
+        entry = {}
+        for name, what in (("causal", "causal"),
+                           ("padded", f"causal with key padding: k_len = {kl} (drawn from "
+                                      f"U[{LONG['klo']}, {LONG['L']}])")):
+            t_l = max_over_ranks(float(np.mean(lms[name])), world)
+            ach = lflops[name] / (float(np.mean(lms[name])) * 1e-3) / 1e12
+            entry[name] = {
+                "workload": f"long-context forward B1 Hq32 Hkv8 (GQA) L16384 d128, {what}; "
+                            f"FLOPs = 4 d x visible pairs",
+                "value": world * lflops[name] / (t_l * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": t_l, "flops_per_step": lflops[name],
+                "roofline": {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
+                             "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"],
+                             "traffic": traffic_per_launch("attn_fwd_impl::fwd_kernel<128>:long"),
+                             "kernel": "attn_fwd_impl::fwd_kernel<128>"}}
+        line["long_context"] = entry
+        line["gpu_launches"] += 2 * args.steps
     if ring is not None:
         rms, rflops, n_fold, mms, mbytes, wholems, rlaunch, (rbms, wbms), (prank, n_zfold) = ring
         t_r = max_over_ranks(float(np.mean(rms)), world)
@@ -901,7 +1065,14 @@ def main():
                                  + (6 * n_fold + 3) * max(3, args.steps // 2)
                                  + (n_fold + n_zfold) * args.steps)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline()
+        line["cpu_baseline"] = cpu_baseline_fwd()
+        if lng is not None:
+            line["long_context"]["causal"]["cpu_baseline"] = cpu_baseline_long()
+            line["long_context"]["padded"]["cpu_baseline"] = cpu_baseline_long(padded=True)
+        if "decode" in legs:
+            line["decode"]["cpu_baseline"] = cpu_baseline_decode(dec_klens)
+        if bms is not None:
+            line["bwd"]["cpu_baseline"] = cpu_baseline_bwd()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -81,6 +81,32 @@ def normal_bf16(seed: int, shape) -> np.ndarray:
     return f64_to_bf16_bits(normal_f64(seed, n)).reshape(shape)
 
 
+def normal_bf16_block(seed: int, shape, index, first: int = None) -> np.ndarray:
+    """``normal_bf16(seed, shape)[index]`` for a tuple ``index`` of leading
+    indices (e.g. (b, h) of a [B, H, L, d] tensor), drawn directly at its
+    counters: element i of the full tensor uses the stream's draws 2 i and
+    2 i + 1, so a block needs no more than its own draws.  ``first``: only the
+    block's first ``first`` entries along its leading axis (e.g. rows [0, first))."""
+    shape = tuple(int(x) for x in shape)
+    index = tuple(int(x) for x in index)
+    inner = shape[len(index):]
+    n = int(np.prod(inner)) if inner else 1
+    if first is not None:
+        if not inner or not 0 <= first <= inner[0]:
+            raise IndexError("first out of range")
+        n_full, inner = n, (int(first),) + inner[1:]
+        n = int(np.prod(inner))
+    start = 0
+    for i, (ix, ext) in enumerate(zip(index, shape)):
+        if not 0 <= ix < ext:
+            raise IndexError("block index out of range")
+        start = start * ext + ix
+    start *= n if first is None else n_full
+    raw = uniform_u64(seed, 2 * n, offset=2 * start)
+    x = np.sqrt(-2.0 * np.log(_unit(raw[0::2]))) * np.cos(2.0 * np.pi * _unit(raw[1::2]))
+    return f64_to_bf16_bits(x).reshape(inner)
+
+
 def uniform_int(seed: int, n: int, lo: int, hi: int) -> np.ndarray:
     """``n`` integers uniform in ``[lo, hi]`` (int32)."""
     raw = uniform_u64(seed, n)
@@ -133,6 +159,7 @@ def workload_seed(workload: int, tensor: str) -> int:
 
 
 __all__ = [
+    "normal_bf16_block",
     "uniform_u64",
     "normal_f64",
     "f64_to_bf16_bits",

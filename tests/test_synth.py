@@ -2,6 +2,7 @@
 8-bit (E4M3) input recipe."""
 
 import numpy as np
+import pytest
 
 import oracle
 import synth
@@ -63,3 +64,17 @@ def test_e4m3_quantised_inputs_follow_the_recipe():
     # the device twin quantises the same values the same way
     c2, s2 = synth.quantize_e4m3_tiles(torch.from_numpy(x.astype(np.float32)))
     assert np.array_equal(c2.numpy(), codes) and np.array_equal(s2.numpy(), scales)
+
+
+def test_block_draws_equal_the_full_tensor_slice():
+    """A head drawn at its own counters equals that head of the full tensor."""
+    full = synth.normal_bf16(4321, (2, 3, 5, 8))
+    for b in range(2):
+        for h in range(3):
+            assert np.array_equal(synth.normal_bf16_block(4321, (2, 3, 5, 8), (b, h)), full[b, h])
+    assert np.array_equal(synth.normal_bf16_block(4321, (2, 3, 5, 8), (1,)), full[1])
+    assert np.array_equal(synth.normal_bf16_block(4321, (2, 3, 5, 8), (1, 2, 4)), full[1, 2, 4])
+    assert np.array_equal(synth.normal_bf16_block(4321, (2, 3, 5, 8), (1, 1), first=3),
+                          full[1, 1, :3])
+    with pytest.raises(IndexError):
+        synth.normal_bf16_block(4321, (2, 3, 5, 8), (2, 0))
