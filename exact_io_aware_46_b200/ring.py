@@ -82,7 +82,10 @@ class RingExchange:
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
+        # the first held tensors are the caller's: they are sent but never
+        # received into (the caller still owns them after the pass)
         self.cur = [t.contiguous() for t in tensors]
+        self.borrowed = True
         self.nxt = [torch.empty_like(t) for t in self.cur]
         self.reqs = None
         self.staged = (any(t.is_cuda for t in self.cur)
@@ -118,7 +121,13 @@ class RingExchange:
         if self.staged:
             for t, h in zip(self.nxt, self.h_recv):
                 t.copy_(h)
-        self.cur, self.nxt = self.nxt, self.cur
+        old = self.cur
+        self.cur = self.nxt
+        if self.borrowed:
+            self.nxt = [torch.empty_like(t) for t in old]
+            self.borrowed = False
+        else:
+            self.nxt = old
 
 
 def fold_chunk(q, kc, vc, kind, O_acc, lse_acc, first, O_out=None, scale=None, workspace=None):

@@ -103,6 +103,53 @@ def _exchange_main(rank, world, port, out):
         f.write(repr(seen))
 
 
+def _caller_tensors_main(rank, world, port, out):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from exact_io_aware_46_b200.ring import ring_bwd_pass
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    k = torch.full((3, 5), float(rank))
+    v = torch.full((2, 7), 10.0 * rank)
+    ex = RingExchange((k, v))
+    for s in range(world):
+        if s + 1 < world:
+            ex.start()
+            ex.finish()
+    g = torch.zeros(4)
+    ring_bwd_pass((k, v), (g,), ring_steps(rank, world, False), lambda *a: None,
+                  lambda part, gs: None)
+    dist.barrier()
+    dist.destroy_process_group()
+    with open(out + f".{rank}", "w") as f:
+        f.write(repr((float(k.min()), float(k.max()), float(v.min()), float(v.max()),
+                      float(g.abs().max()))))
+
+
+@pytest.mark.parametrize("world", [2, 3, 4])
+def test_ring_pass_leaves_the_callers_tensors_alone(tmp_path, world):
+    """A full ring pass (forward exchange, then the backward's two exchanges)
+    sends the caller's K/V but never receives into them: a driver's caller can
+    run the backward on the same K/V tensors after the forward.  (Receiving into
+    the first held tensors broke this from the second swap on, i.e. from three
+    ranks.)"""
+    import torch.multiprocessing as mp
+
+    out = str(tmp_path / "c")
+    mp.start_processes(_caller_tensors_main, args=(world, _free_port(), out), nprocs=world,
+                       join=True, start_method="spawn")
+    for rank in range(world):
+        kmin, kmax, vmin, vmax, g = eval(open(out + f".{rank}").read())
+        assert (kmin, kmax, vmin, vmax) == (rank, rank, 10.0 * rank, 10.0 * rank)
+        assert g == 0.0
+
+
 @pytest.mark.parametrize("world", [1, 2, 3])
 def test_ring_exchange_on_gloo_ranks(tmp_path, world):
     """At step s every rank holds the chunk of rank (rank - s) mod world."""
