@@ -12,20 +12,25 @@
 // B200 design.  Three launches:
 //  1. prep: D per query row, LSE in log2 units (+inf for rows without a
 //     visible key or past Lq, so their P is exactly 0), and a zeroed fp32 dQ
-//     accumulator; rows are padded to a multiple of 64 per head.
+//     accumulator; rows are padded to a multiple of 128 per head.
 //  2. main (persistent, one CTA per SM): a work item is one 128-key tile of one
 //     (batch, key/value head).  K and V stay in shared memory while the item
-//     walks every 64-row query tile of every query head of the group that can
+//     walks every 128-row query tile of every query head of the group that can
 //     see the keys.  Per query tile the tensor core computes, with keys on the
-//     128 TMEM lanes,
+//     128 TMEM lanes and every MMA at M = 128, N = 128,
 //        S^T  = K Q^T          (SS)        dP^T = V dO^T        (SS)
 //        dV  += P^T dO         (TS: P^T from TMEM, written by the softmax)
-//        dK  += dS^T Q         (SS: dS^T staged in shared memory)
 //        dQ^T = K^T dS^T       (SS, both operands MN-major)
-//     dV and dK accumulate in TMEM across the item; S/dP are double-buffered
-//     and dQ^T reuses the dP buffer once dS has been formed.  Warps 0-3 form
-//     P and dS (one key row per thread), warps 4-7 drain dQ^T with fp32
-//     reductions into the accumulator, warp 8 feeds TMA, warp 9 issues MMAs.
+//        dK  += dS^T Q         (SS: dS^T staged in shared memory)
+//     dV and dK accumulate in TMEM across the item (256 columns); S^T/P^T and
+//     dP^T take the other 256, and dQ^T reuses the dP^T columns once dS has
+//     been formed.  Tensor memory holds one query tile at a time, so the
+//     issue order S^T(t), dP^T(t), dV(t), dQ^T(t), dK(t), S^T(t+1) gives each
+//     hand-off one MMA group of cover: P(t) forms while dP^T(t) runs, dS(t)
+//     while dV(t) runs, and the drain of dQ^T(t) while dK(t) and S^T(t+1) run.
+//     Warps 0-7 form P and dS (one key row per thread, two warps per row, 64
+//     query rows each), warps 8-11 drain dQ^T into the fp32 accumulator with
+//     bulk reduce-adds, warp 12 feeds TMA, warp 13 issues MMAs.
 //  3. convert: dQ = bf16(scale * accumulator).
 #pragma once
 
@@ -34,33 +39,50 @@
 
 namespace attn_bwd_impl {
 
-constexpr int BN = 128;  // keys per work item (TMEM lanes)
-constexpr int BMQ = 64;  // query rows per query tile
-constexpr int D = 128;   // head dimension handled by the main kernel
-constexpr int NQS = 3;   // query/dO ring stages
-constexpr int NTHREADS = 320;  // P/dS warpgroup, dQ warpgroup, load warp, MMA warp
+constexpr int BN = 128;   // keys per work item (TMEM lanes)
+constexpr int BMQ = 128;  // query rows per query tile
+constexpr int D = 128;    // head dimension handled by the main kernel
+constexpr int NQS = 2;    // query-tile ring stages (Q with its log2-LSE and D); dO is single-buffered
+constexpr int NSMX = 8;   // P/dS warps: 4 lane quarters x 2 halves of the query rows
+constexpr int W_DRAIN = NSMX;        // warps 8-11: dQ^T drain
+constexpr int W_LOAD = NSMX + 4;     // warp 12: TMA producer
+constexpr int W_MMA = NSMX + 5;      // warp 13: MMA issuer
+constexpr int NTHREADS = 32 * (NSMX + 6);
+constexpr int NI = 4;                          // depth of the shared-memory item ring
+constexpr int ITEM_READERS = NSMX + 4 + 1;     // warps that read each item: P/dS, drain, MMA
+constexpr int DQ_ROWS = 32;          // query rows per dQ staging round (16 KB of fp32)
 
-// shared memory map (bytes); the swizzled panels are 1024-byte aligned
-constexpr int OFF_K = 0;                              // [128 keys][d]: 2 panels of 16 KB
-constexpr int OFF_V = 32768;
-constexpr int OFF_QS = 65536;                         // stage s: Q (2 x 8 KB) then dO (2 x 8 KB)
-constexpr int QS_BYTES = 32768;
-constexpr int OFF_DS = OFF_QS + NQS * QS_BYTES;       // dS^T buffers [128 keys][64 rows], 16 KB each
-constexpr int OFF_LD = OFF_DS + 2 * 16384;            // stage s: lse2 [64] then D [64]
-constexpr int OFF_DQ = OFF_LD + NQS * 512;            // dQ tile staging [64 rows][128] fp32, 32 KB
-constexpr int OFF_BAR = OFF_DQ + 32768;
-constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;
+// shared memory map (bytes); the swizzled panels are 1024-byte aligned.  A tile
+// of 128 rows x 128 bf16 columns is two 128-byte-swizzled panels of 64 columns
+// (16 KB each).
+constexpr int TILE = 32768;
+constexpr int PANEL = 16384;
+constexpr int OFF_K = 0;                        // [128 keys][d]
+constexpr int OFF_V = TILE;
+constexpr int OFF_Q = 2 * TILE;                 // NQS stages of [128 rows][d]
+constexpr int OFF_DO = OFF_Q + NQS * TILE;      // [128 rows][d]
+constexpr int OFF_DS = OFF_DO + TILE;           // dS^T [128 keys][128 rows]: panels of 64 rows
+constexpr int OFF_DQ = OFF_DS + TILE;           // dQ staging [DQ_ROWS][d] fp32
+constexpr int OFF_LD = OFF_DQ + DQ_ROWS * D * 4;  // stage s: lse2 [128] then D [128]
+constexpr int OFF_BAR = OFF_LD + NQS * 1024;
+constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
 static_assert(SMEM_BYTES <= 232448, "dynamic shared memory limit");
 
-// TMEM columns
-constexpr uint32_t S_COL0 = 0;      // S^T / P^T, 2 buffers x 64
-constexpr uint32_t DP_COL0 = 128;   // dP^T, then dQ^T, 2 buffers x 64
+// TMEM columns (512 allocated)
+constexpr uint32_t S_COL = 0;     // S^T, overwritten by P^T (packed bf16) -- 128
+constexpr uint32_t DP_COL = 128;  // dP^T, then dQ^T of the same tile -- 128
 constexpr uint32_t DV_COL = 256;
 constexpr uint32_t DK_COL = 384;
 
 constexpr uint32_t IDESC_S = sm100::idesc_bf16_f32(128, BMQ, false, false);
 constexpr uint32_t IDESC_DV = sm100::idesc_bf16_f32(128, D, false, true);
 constexpr uint32_t IDESC_DQ = sm100::idesc_bf16_f32(128, BMQ, true, true);
+
+// Exponentials on the FMA pipe (polynomial exp2) for column pairs cp with
+// (cp & 7) >= POLY_FROM: the 16384 exponentials of a tile take 1024 cycles on
+// the special-function unit alone, more than the one MMA group (~690 cycles)
+// that covers the forming of P.
+constexpr int POLY_FROM = 5;
 
 struct Args {
   const __nv_bfloat16 *Q, *K, *V, *O, *dO;
@@ -97,8 +119,9 @@ struct Params {
   int causal;
   int window;  // > 0: a query row sees only its `window` latest keys
   int n_kv;     // ceil(Lk / 128)
-  int n_qt;     // Lqp / 64
+  int n_qt;     // Lqp / BMQ
   int n_items;  // B * Hkv * n_kv
+  int* sched;   // [0] next dynamic item, [1] finished CTAs (workspace header)
 };
 
 struct Item {
@@ -248,19 +271,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* kv_full = bars + 0;
   uint64_t* kv_empty = bars + 1;
-  uint64_t* qdo_full = bars + 2;    // [NQS]
-  uint64_t* qdo_empty = bars + 5;   // [NQS]
-  uint64_t* s_full = bars + 8;      // [2]
-  uint64_t* p_full = bars + 10;     // [2]
-  uint64_t* dp_full = bars + 12;    // [2]
-  uint64_t* ds_full = bars + 14;    // [2]
-  uint64_t* ds_empty = bars + 16;   // [2]
-  uint64_t* dq_full = bars + 18;    // [2]
-  uint64_t* dq_empty = bars + 20;   // [2]
-  uint64_t* dkv_full = bars + 22;
-  uint64_t* dkv_empty = bars + 23;
-  uint64_t* drain = bars + 24;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 25);
+  uint64_t* q_full = bars + 2;     // [NQS]
+  uint64_t* q_empty = bars + 4;    // [NQS]
+  uint64_t* do_full = bars + 6;
+  uint64_t* do_empty = bars + 7;
+  uint64_t* s_full = bars + 8;
+  uint64_t* p_full = bars + 9;
+  uint64_t* dp_full = bars + 10;
+  uint64_t* ds_full = bars + 11;
+  uint64_t* dq_full = bars + 12;
+  uint64_t* dq_empty = bars + 13;
+  uint64_t* dkv_full = bars + 14;
+  uint64_t* dkv_empty = bars + 15;
+  uint64_t* drain = bars + 16;
+  uint64_t* item_full = bars + 17;   // [NI]
+  uint64_t* item_empty = bars + 21;  // [NI]
+  int* item_ring = reinterpret_cast<int*>(bars + 25);  // [NI]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_ring + NI);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -268,31 +295,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     sm100::mbar_init(kv_full, 1);
     sm100::mbar_init(kv_empty, 1);
     for (int s = 0; s < NQS; ++s) {
-      sm100::mbar_init(&qdo_full[s], 1);
-      sm100::mbar_init(&qdo_empty[s], 1);
+      sm100::mbar_init(&q_full[s], 1);
+      sm100::mbar_init(&q_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      sm100::mbar_init(&s_full[b], 1);
-      sm100::mbar_init(&p_full[b], 128);
-      sm100::mbar_init(&dp_full[b], 1);
-      sm100::mbar_init(&ds_full[b], 128);
-      sm100::mbar_init(&ds_empty[b], 1);
-      sm100::mbar_init(&dq_full[b], 1);
-      sm100::mbar_init(&dq_empty[b], 128);
-    }
+    sm100::mbar_init(do_full, 1);
+    sm100::mbar_init(do_empty, 1);
+    sm100::mbar_init(s_full, 1);
+    sm100::mbar_init(p_full, NSMX);
+    sm100::mbar_init(dp_full, 1);
+    sm100::mbar_init(ds_full, NSMX);
+    sm100::mbar_init(dq_full, 1);
+    sm100::mbar_init(dq_empty, 4);
     sm100::mbar_init(dkv_full, 1);
-    sm100::mbar_init(dkv_empty, 128);
+    sm100::mbar_init(dkv_empty, NSMX);
     sm100::mbar_init(drain, 1);
+    for (int i = 0; i < NI; ++i) {
+      sm100::mbar_init(&item_full[i], 1);
+      sm100::mbar_init(&item_empty[i], ITEM_READERS);
+    }
     *abort_flag = 0;
     sm100::fence_barrier_init();
   }
-  if (warp == 8 && sm100::lane_id() == 0) {
+  if (warp == W_LOAD && sm100::lane_id() == 0) {
     sm100::prefetch_tmap(&tmQ);
     sm100::prefetch_tmap(&tmdO);
     sm100::prefetch_tmap(&tmK);
     sm100::prefetch_tmap(&tmV);
   }
-  if (warp == 9) {
+  if (warp == W_MMA) {
     sm100::tmem_alloc(tmem_slot, 512);
     sm100::tmem_relinquish();
   }
@@ -301,42 +331,78 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   sm100::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int off = p.Lk - p.Lq;  // bottom-right causal alignment
-  if (warp == 8) {
+  // a consumer warp's view of the item ring: the k-th item of this CTA, or -1
+  // at the end (one arrival per warp; the caller's whole warp calls this)
+  auto next_item = [&](uint32_t k, int& w) -> bool {
+    if (!sm100::mbar_wait(&item_full[k % NI], (k / NI) & 1, abort_flag, p.status)) return false;
+    w = *reinterpret_cast<volatile int*>(&item_ring[k % NI]);
+    __syncwarp();
+    if (sm100::lane_id() == 0) sm100::mbar_arrive(&item_empty[k % NI]);
+    return true;
+  };
+  if (warp == W_LOAD) {
     // ------------------------------------------------------------ TMA producer
+    // per query tile: Q (+ its log2-LSE and D) into the two-stage ring, then dO
+    // into its single buffer (free once dV of the previous tile has run)
     if (sm100::lane_id() == 0) {
       uint32_t tq = 0, ik = 0;
+      int last_q[NQS] = {-1, -1}, last_do = -1;  // last tile whose copies were issued
+      uint32_t kv_issued = 0;
       bool ok = true;
-      for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x, ++ik) {
+      for (; ok; ++ik) {
+        // dynamic scheduling: the CTA's first item is its index, the others
+        // come from the counter in the workspace (heaviest items first)
+        if (!(ok = sm100::mbar_wait(&item_empty[ik % NI], ((ik / NI) & 1) ^ 1, abort_flag,
+                                    p.status)))
+          break;
+        int w = (ik == 0) ? static_cast<int>(blockIdx.x)
+                          : atomicAdd(p.sched, 1) + static_cast<int>(gridDim.x);
+        if (w >= p.n_items) w = -1;
+        *reinterpret_cast<volatile int*>(&item_ring[ik % NI]) = w;
+        sm100::mbar_arrive(&item_full[ik % NI]);
+        if (w < 0) break;
         const Item it = get_item(p, w, nullptr);
         if (!(ok = sm100::mbar_wait(kv_empty, (ik & 1) ^ 1, abort_flag, p.status))) break;
-        sm100::mbar_arrive_expect_tx(kv_full, 2 * BN * D * 2);
+        sm100::mbar_arrive_expect_tx(kv_full, 2 * TILE);
+        ++kv_issued;
         const int kvh = it.b * p.Hkv + it.hkv;
         for (int c = 0; c < 2; ++c) {
-          sm100::tma_load_3d(&tmK, kv_full, smem + OFF_K + c * 16384, c * 64, it.n * BN, kvh);
-          sm100::tma_load_3d(&tmV, kv_full, smem + OFF_V + c * 16384, c * 64, it.n * BN, kvh);
+          sm100::tma_load_3d(&tmK, kv_full, smem + OFF_K + c * PANEL, c * 64, it.n * BN, kvh);
+          sm100::tma_load_3d(&tmV, kv_full, smem + OFF_V + c * PANEL, c * 64, it.n * BN, kvh);
         }
         const int nq = it.T > 0 ? it.T / p.G : 0;
         for (int t = 0; t < it.T && ok; ++t, ++tq) {
           const int g = t / nq, i = it.i_lo + t % nq;
           const int slot = tq % NQS;
-          if (!(ok = sm100::mbar_wait(&qdo_empty[slot], ((tq / NQS) & 1) ^ 1, abort_flag,
+          const int qh = it.b * p.Hq + it.hkv * p.G + g;
+          if (!(ok = sm100::mbar_wait(&q_empty[slot], ((tq / NQS) & 1) ^ 1, abort_flag,
                                       p.status)))
             break;
-          sm100::mbar_arrive_expect_tx(&qdo_full[slot], QS_BYTES + 512);
-          const int qh = it.b * p.Hq + it.hkv * p.G + g;
-          uint8_t* st = smem + OFF_QS + slot * QS_BYTES;
-          for (int c = 0; c < 2; ++c) {
-            sm100::tma_load_3d(&tmQ, &qdo_full[slot], st + c * 8192, c * 64, i * BMQ, qh);
-            sm100::tma_load_3d(&tmdO, &qdo_full[slot], st + 16384 + c * 8192, c * 64, i * BMQ,
-                               qh);
-          }
+          sm100::mbar_arrive_expect_tx(&q_full[slot], TILE + 1024);
+          for (int c = 0; c < 2; ++c)
+            sm100::tma_load_3d(&tmQ, &q_full[slot], smem + OFF_Q + slot * TILE + c * PANEL,
+                               c * 64, i * BMQ, qh);
           const size_t rowoff = static_cast<size_t>(qh) * p.Lqp + i * BMQ;
-          bulk_g2s(smem + OFF_LD + slot * 512, p.lse2 + rowoff, 256, &qdo_full[slot]);
-          bulk_g2s(smem + OFF_LD + slot * 512 + 256, p.Dvec + rowoff, 256, &qdo_full[slot]);
+          bulk_g2s(smem + OFF_LD + slot * 1024, p.lse2 + rowoff, 512, &q_full[slot]);
+          bulk_g2s(smem + OFF_LD + slot * 1024 + 512, p.Dvec + rowoff, 512, &q_full[slot]);
+          last_q[slot] = static_cast<int>(tq);
+          if (!(ok = sm100::mbar_wait(do_empty, (tq & 1) ^ 1, abort_flag, p.status))) break;
+          sm100::mbar_arrive_expect_tx(do_full, TILE);
+          for (int c = 0; c < 2; ++c)
+            sm100::tma_load_3d(&tmdO, do_full, smem + OFF_DO + c * PANEL, c * 64, i * BMQ, qh);
+          last_do = static_cast<int>(tq);
         }
       }
+      // the CTA must not exit while tensor copies still land in its shared
+      // memory, which an expired wait elsewhere could otherwise allow: wait
+      // (bounded) for the last issued phase of every load barrier (in normal
+      // operation the consumers have already waited for all of them)
+      if (kv_issued > 0) sm100::mbar_wait_drain(kv_full, (kv_issued - 1) & 1);
+      for (int sl = 0; sl < NQS; ++sl)
+        if (last_q[sl] >= 0) sm100::mbar_wait_drain(&q_full[sl], (last_q[sl] / NQS) & 1);
+      if (last_do >= 0) sm100::mbar_wait_drain(do_full, last_do & 1);
     }
-  } else if (warp == 9) {
+  } else if (warp == W_MMA) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs the loop (warp-uniform values stay in uniform
     // registers) and one elected lane issues; descriptors are built once per
@@ -347,25 +413,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       uint32_t tq = 0, ik = 0;
       bool ok = true;
       const uint32_t kA = sbase + OFF_K, vA = sbase + OFF_V;
-      auto qA = [&](int slot) { return sbase + OFF_QS + slot * QS_BYTES; };
-      auto doA = [&](int slot) { return sbase + OFF_QS + slot * QS_BYTES + 16384; };
-      auto dsA = [&](int b) { return sbase + OFF_DS + b * 16384; };
+      const uint32_t doA = sbase + OFF_DO, dsA = sbase + OFF_DS;
+      auto qA = [&](int slot) { return sbase + OFF_Q + slot * TILE; };
       auto commit = [&](uint64_t* bar) {
         if (leader) sm100::tc_commit(bar);
         __syncwarp();
       };
-      // S^T (or dP^T) = A_keys[128 x d] * B_rows[64 x d]^T, both K-major
+      // S^T (or dP^T) = A_keys[128 x d] * B_rows[128 x d]^T, both K-major
       auto issue_kmajor = [&](uint32_t dcol, uint32_t a, uint32_t b) {
         const uint64_t ad = sm100::sdesc_sw128(a, 16, 1024);
         const uint64_t bd = sm100::sdesc_sw128(b, 16, 1024);
         if (leader) {
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k)
-            sm100::mma_ss(tmem + dcol, ad + (((k >> 2) * 16384 + (k & 3) * 32) >> 4),
-                          bd + (((k >> 2) * 8192 + (k & 3) * 32) >> 4), IDESC_S, k > 0);
+          for (int k = 0; k < D / 16; ++k) {
+            const uint64_t o = static_cast<uint64_t>(((k >> 2) * PANEL + (k & 3) * 32) >> 4);
+            sm100::mma_ss(tmem + dcol, ad + o, bd + o, IDESC_S, k > 0);
+          }
         }
       };
-      for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x, ++ik) {
+      const uint64_t kd_mn = sm100::sdesc_sw128(kA, PANEL, 1024);   // K^T: MN-major A over d
+      const uint64_t do_mn = sm100::sdesc_sw128(doA, PANEL, 1024);  // dO: MN-major B over d
+      const uint64_t ds_k = sm100::sdesc_sw128(dsA, 16, 1024);      // dS^T: K-major A over rows
+      const uint64_t ds_mn = sm100::sdesc_sw128(dsA, PANEL, 1024);  // dS^T: MN-major B over rows
+      for (; ok; ++ik) {
+        int w;
+        if (!(ok = next_item(ik, w)) || w < 0) break;
         const Item it = get_item(p, w, nullptr);
         if (!(ok = sm100::mbar_wait(kv_full, ik & 1, abort_flag, p.status))) break;
         sm100::tc_fence_after();
@@ -375,81 +447,77 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           commit(kv_empty);
           continue;
         }
-        // Issue order per query tile t (buffers b = t & 1, nb = (t + 1) & 1):
-        //   S(t+1) | dV(t) [P(t)] | dP(t+1) [dQ^T(t-1) drained] | dK(t), dQ^T(t) [dS(t)]
-        // so each wait on another warp's signal has half an iteration of queued
-        // tensor work in front of it.
-        {
-          const int slot = tq % NQS, b = tq & 1;
-          if (!(ok = sm100::mbar_wait(&qdo_full[slot], (tq / NQS) & 1, abort_flag, p.status)))
+        {  // S^T of the item's first query tile
+          const int slot = tq % NQS;
+          if (!(ok = sm100::mbar_wait(&q_full[slot], (tq / NQS) & 1, abort_flag, p.status)))
             break;
           sm100::tc_fence_after();
-          issue_kmajor(S_COL0 + b * 64, kA, qA(slot));
-          commit(&s_full[b]);
-          if (!(ok = sm100::mbar_wait(&dq_empty[b], ((tq >> 1) & 1) ^ 1, abort_flag, p.status)))
-            break;
-          sm100::tc_fence_after();
-          issue_kmajor(DP_COL0 + b * 64, vA, doA(slot));
-          commit(&dp_full[b]);
+          issue_kmajor(S_COL, kA, qA(slot));
+          commit(s_full);
         }
-        const uint64_t kd_mn = sm100::sdesc_sw128(kA, 16384, 1024);  // K as MN-major A (over d)
-        for (int t = 0; t < it.T && ok; ++t) {
-          const uint32_t cur = tq + t;
-          const int slot = cur % NQS, b = cur & 1;
-          const uint32_t u = cur >> 1;
-          const uint32_t nx = cur + 1;
-          const int ns = nx % NQS, nb = nx & 1;
-          const bool more = t + 1 < it.T;
-          if (more) {
-            if (!(ok = sm100::mbar_wait(&qdo_full[ns], (nx / NQS) & 1, abort_flag, p.status)))
-              break;
-            sm100::tc_fence_after();
-            issue_kmajor(S_COL0 + nb * 64, kA, qA(ns));
-            commit(&s_full[nb]);
-          }
-          if (!(ok = sm100::mbar_wait(&p_full[b], u & 1, abort_flag, p.status))) break;
-          sm100::tc_fence_after();
-          if (t == 0) {
-            if (!(ok = sm100::mbar_wait(dkv_empty, (ik & 1) ^ 1, abort_flag, p.status))) break;
-            sm100::tc_fence_after();
-          }
-          const uint64_t do_mn = sm100::sdesc_sw128(doA(slot), 8192, 1024);
-          const uint64_t q_mn = sm100::sdesc_sw128(qA(slot), 8192, 1024);
-          const uint64_t ds_k = sm100::sdesc_sw128(dsA(b), 16, 1024);
-          const uint64_t ds_mn = sm100::sdesc_sw128(dsA(b), 8192, 1024);
-          // dV += P^T dO : A = P^T (TMEM, packed bf16), B = dO (MN-major)
+        // Issue order, one MMA group each (dK of a tile is issued one tile late):
+        //   S^T(t) | dK(t-1) | dP^T(t) | dV(t) [P(t)] | dQ^T(t) [dS(t)] | S^T(t+1) ...
+        // P(t) forms while dK(t-1) and dP^T(t) run, dS(t) while dV(t) runs, and
+        // the drain of dQ^T(t) has S^T(t+1) and dK(t) to hand the dP^T columns
+        // back.  dS^T(t) is read by dQ^T(t) and dK(t) before dP^T(t+1) is
+        // issued, so one shared-memory buffer serves every tile.
+        auto issue_dk = [&](uint32_t tile, bool first) {
+          const uint64_t q_mn = sm100::sdesc_sw128(qA(tile % NQS), PANEL, 1024);
           if (leader) {
 #pragma unroll
             for (int k = 0; k < BMQ / 16; ++k)
-              sm100::mma_ts(tmem + DV_COL, tmem + S_COL0 + b * 64 + k * 8, do_mn + ((k * 2048) >> 4),
-                            IDESC_DV, (t > 0 || k > 0) ? 1u : 0u);
+              sm100::mma_ss(tmem + DK_COL, ds_k + ((((k >> 2) * PANEL) + (k & 3) * 32) >> 4),
+                            q_mn + ((k * 2048) >> 4), IDESC_DV, (!first || k > 0) ? 1u : 0u);
           }
-          if (more) {
-            if (!(ok = sm100::mbar_wait(&dq_empty[nb], ((nx >> 1) & 1) ^ 1, abort_flag,
+          commit(&q_empty[tile % NQS]);
+        };
+        for (int t = 0; t < it.T && ok; ++t) {
+          const uint32_t cur = tq + t;
+          const uint32_t par = cur & 1;
+          if (t > 0) issue_dk(cur - 1, t == 1);
+          // dP^T(t) = V dO^T: needs dO(t) and the dP^T columns back from the
+          // drain of the previous tile's dQ^T
+          if (!(ok = sm100::mbar_wait(do_full, par, abort_flag, p.status))) break;
+          if (!(ok = sm100::mbar_wait(dq_empty, par ^ 1, abort_flag, p.status))) break;
+          sm100::tc_fence_after();
+          issue_kmajor(DP_COL, vA, doA);
+          commit(dp_full);
+          // dV += P^T dO : A = P^T (TMEM, packed bf16: query rows 0-63 in columns
+          // 0-31, rows 64-127 from column 64 on), B = dO (MN-major)
+          if (!(ok = sm100::mbar_wait(p_full, par, abort_flag, p.status))) break;
+          if (t == 0 && !(ok = sm100::mbar_wait(dkv_empty, (ik & 1) ^ 1, abort_flag, p.status)))
+            break;
+          sm100::tc_fence_after();
+          if (leader) {
+#pragma unroll
+            for (int k = 0; k < BMQ / 16; ++k)
+              sm100::mma_ts(tmem + DV_COL, tmem + S_COL + (k >> 2) * 64 + (k & 3) * 8,
+                            do_mn + ((k * 2048) >> 4), IDESC_DV, (t > 0 || k > 0) ? 1u : 0u);
+          }
+          commit(do_empty);
+          // dQ^T = K^T dS^T into the dP^T columns
+          if (!(ok = sm100::mbar_wait(ds_full, par, abort_flag, p.status))) break;
+          sm100::tc_fence_after();
+          if (leader) {
+#pragma unroll
+            for (int k = 0; k < BN / 16; ++k)
+              sm100::mma_ss(tmem + DP_COL, kd_mn + ((k * 2048) >> 4), ds_mn + ((k * 2048) >> 4),
+                            IDESC_DQ, k > 0 ? 1u : 0u);
+          }
+          commit(dq_full);
+          // S^T of the next query tile (P^T of this one was read by dV above)
+          if (t + 1 < it.T) {
+            const int ns = (cur + 1) % NQS;
+            if (!(ok = sm100::mbar_wait(&q_full[ns], ((cur + 1) / NQS) & 1, abort_flag,
                                         p.status)))
               break;
             sm100::tc_fence_after();
-            issue_kmajor(DP_COL0 + nb * 64, vA, doA(ns));
-            commit(&dp_full[nb]);
+            issue_kmajor(S_COL, kA, qA(ns));
+            commit(s_full);
           }
-          if (!(ok = sm100::mbar_wait(&ds_full[b], u & 1, abort_flag, p.status))) break;
-          sm100::tc_fence_after();
-          if (leader) {
-            // dK += dS^T Q : A = dS^T (K-major over rows), B = Q (MN-major)
-#pragma unroll
-            for (int k = 0; k < BMQ / 16; ++k)
-              sm100::mma_ss(tmem + DK_COL, ds_k + ((k * 32) >> 4), q_mn + ((k * 2048) >> 4),
-                            IDESC_DV, (t > 0 || k > 0) ? 1u : 0u);
-            // dQ^T = K^T dS^T : A = K (MN-major over d), B = dS^T (MN-major over rows)
-#pragma unroll
-            for (int k = 0; k < BN / 16; ++k)
-              sm100::mma_ss(tmem + DP_COL0 + b * 64, kd_mn + ((k * 2048) >> 4),
-                            ds_mn + ((k * 2048) >> 4), IDESC_DQ, k > 0 ? 1u : 0u);
-          }
-          commit(&dq_full[b]);
-          commit(&ds_empty[b]);
-          commit(&qdo_empty[slot]);
         }
+        if (!ok) break;
+        issue_dk(tq + it.T - 1, it.T == 1);  // the item's last dK
         if (!ok) break;
         tq += it.T;
         commit(dkv_full);
@@ -458,13 +526,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       commit(drain);
       sm100::mbar_wait_drain(drain, 0);
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ P and dS (one key per thread)
-    const int kl_ = threadIdx.x;  // key row within the tile = TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  } else if (warp < NSMX) {
+    // ------------------------------------------------------------ P and dS
+    // one key row per thread (= TMEM lane); the two warps of a lane quarter
+    // take query rows [0, 64) and [64, 128) of the tile
+    const int qd = warp & 3, hf = warp >> 2;
+    const int kl_ = qd * 32 + sm100::lane_id();  // key row within the tile = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
+    const uint32_t s_addr = tmem + lane_base + S_COL + 64 * hf;
+    const uint32_t dp_addr = tmem + lane_base + DP_COL + 64 * hf;
     uint32_t tq = 0, ik = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x, ++ik) {
+    for (; ok; ++ik) {
+      int w;
+      if (!(ok = next_item(ik, w)) || w < 0) break;
       bool bad = false;
       const Item it = get_item(p, w, &bad);
       if (bad && threadIdx.x == 0) atomicOr(p.status, 1);
@@ -473,105 +548,133 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int nq = it.T > 0 ? it.T / p.G : 0;
       for (int t = 0; t < it.T && ok; ++t) {
         const uint32_t cur = tq + t;
-        const int slot = cur % NQS, b = cur & 1;
-        const uint32_t u = cur >> 1;
+        const int slot = cur % NQS;
+        const uint32_t par = cur & 1;
         const int i = it.i_lo + t % nq;
-        const float* l2s = reinterpret_cast<const float*>(smem + OFF_LD + slot * 512);
-        const float* dsv = l2s + 64;
-        // lse2 / D of this stage were delivered on qdo_full
-        if (!(ok = sm100::mbar_wait(&qdo_full[slot], (cur / NQS) & 1, abort_flag, p.status)))
+        const float* l2s = reinterpret_cast<const float*>(smem + OFF_LD + slot * 1024) + 64 * hf;
+        const float* dsv = l2s + 128;
+        // lse2 / D of this tile were delivered on q_full
+        if (!(ok = sm100::mbar_wait(&q_full[slot], (cur / NQS) & 1, abort_flag, p.status)))
           break;
-        if (!(ok = sm100::mbar_wait(&s_full[b], u & 1, abort_flag, p.status))) break;
+        if (!(ok = sm100::mbar_wait(s_full, par, abort_flag, p.status))) break;
         sm100::tc_fence_after();
-        uint32_t s[64];
-        sm100::tmem_ld32(tmem + lane_base + S_COL0 + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-        sm100::tmem_ld32(tmem + lane_base + S_COL0 + b * 64 + 32,
-                         *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-        sm100::tmem_ld_wait();
-        // key visible to query row r0 + c iff key <= lim_key, c >= cmin and
-        // (sliding window) c <= cmax
-        const int r0 = i * BMQ;
-        const bool key_ok = key <= lim;
-        const int cmin = p.causal ? key - r0 - off : -1;
-        const int cmax = p.window > 0 ? key - off + p.window - 1 - r0 : BMQ;
-        // whole tile visible: no per-element test (warp-uniform; usual case)
-        const bool all_vis = __all_sync(0xffffffffu, key_ok && cmin <= 0 && cmax >= BMQ - 1);
-        const float4* l2v = reinterpret_cast<const float4*>(l2s);
-        const float2 sl2x2 = make_float2(p.scale_log2, p.scale_log2);
-        float pr[64];
-#pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const float4 lq = l2v[c4];
-          const float2 x0 = __ffma2_rn(
-              make_float2(__uint_as_float(s[4 * c4]), __uint_as_float(s[4 * c4 + 1])), sl2x2,
-              make_float2(-lq.x, -lq.y));
-          const float2 x1 = __ffma2_rn(
-              make_float2(__uint_as_float(s[4 * c4 + 2]), __uint_as_float(s[4 * c4 + 3])), sl2x2,
-              make_float2(-lq.z, -lq.w));
-          pr[4 * c4] = sm100::ex2(x0.x);
-          pr[4 * c4 + 1] = sm100::ex2(x0.y);
-          pr[4 * c4 + 2] = sm100::ex2(x1.x);
-          pr[4 * c4 + 3] = sm100::ex2(x1.y);
-        }
-        if (!all_vis) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (!key_ok || c < cmin || c > cmax) pr[c] = 0.f;
-        }
+        // P = exp2(S scale log2(e) - lse2), kept as packed bf16 pairs (the
+        // precision dV uses; dS is formed from the same values)
         uint32_t pk[32];
+        {
+          // key visible to query row r0 + c iff key <= lim, c >= cmin and
+          // (sliding window) c <= cmax
+          const int r0 = i * BMQ + 64 * hf;
+          const bool key_ok = key <= lim;
+          const int cmin = p.causal ? key - r0 - off : -1;
+          const int cmax = p.window > 0 ? key - off + p.window - 1 - r0 : 64;
+          // whole half-tile visible: no per-element test (warp-uniform; usual case)
+          const bool all_vis = __all_sync(0xffffffffu, key_ok && cmin <= 0 && cmax >= 63);
+          const float4* l2v = reinterpret_cast<const float4*>(l2s);
+          const float2 sl2x2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = sm100::pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
-        sm100::tmem_st32(tmem + lane_base + S_COL0 + b * 64, pk);
+          for (int h2 = 0; h2 < 2; ++h2) {  // 32 columns at a time (register pressure)
+            uint32_t s[32];
+            sm100::tmem_ld32(s_addr + 32 * h2, s);
+            sm100::tmem_ld_wait();
+            if (!all_vis) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) {
+                const int cc = 32 * h2 + c;
+                if (!key_ok || cc < cmin || cc > cmax) s[c] = __float_as_uint(-INFINITY);
+              }
+            }
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4) {
+              const float4 lq = l2v[8 * h2 + c4];
+              const float2 x0 = __ffma2_rn(
+                  make_float2(__uint_as_float(s[4 * c4]), __uint_as_float(s[4 * c4 + 1])), sl2x2,
+                  make_float2(-lq.x, -lq.y));
+              const float2 x1 = __ffma2_rn(
+                  make_float2(__uint_as_float(s[4 * c4 + 2]), __uint_as_float(s[4 * c4 + 3])),
+                  sl2x2, make_float2(-lq.z, -lq.w));
+              const int cp = 16 * h2 + 2 * c4;  // column pair index of x0
+              float2 e0, e1;
+              if ((cp & 7) >= POLY_FROM) {
+                e0 = sm100::ex2_poly2(x0);
+              } else {
+                e0.x = sm100::ex2(x0.x);
+                e0.y = sm100::ex2(x0.y);
+              }
+              if (((cp + 1) & 7) >= POLY_FROM) {
+                e1 = sm100::ex2_poly2(x1);
+              } else {
+                e1.x = sm100::ex2(x1.x);
+                e1.y = sm100::ex2(x1.y);
+              }
+              pk[cp] = sm100::pack_bf16x2(e0.x, e0.y);
+              pk[cp + 1] = sm100::pack_bf16x2(e1.x, e1.y);
+            }
+          }
+        }
+        sm100::tmem_st32(s_addr, pk);
         sm100::tmem_st_wait();
         sm100::tc_fence_before();
-        sm100::mbar_arrive(&p_full[b]);
+        __syncwarp();
+        if (sm100::lane_id() == 0) sm100::mbar_arrive(p_full);
 
-        if (!(ok = sm100::mbar_wait(&dp_full[b], u & 1, abort_flag, p.status))) break;
+        // dS = P o (dP - D), written K-major (row-contiguous per key) to panel hf
+        if (!(ok = sm100::mbar_wait(dp_full, par, abort_flag, p.status))) break;
         sm100::tc_fence_after();
-        sm100::tmem_ld32(tmem + lane_base + DP_COL0 + b * 64,
-                         *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-        sm100::tmem_ld32(tmem + lane_base + DP_COL0 + b * 64 + 32,
-                         *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-        sm100::tmem_ld_wait();
+        uint8_t* line = smem + OFF_DS + hf * PANEL + kl_ * 128;
         const float4* dvv = reinterpret_cast<const float4*>(dsv);
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const float4 dq = dvv[c4];
-          const float2 d0 = __fmul2_rn(
-              make_float2(pr[4 * c4], pr[4 * c4 + 1]),
-              __fadd2_rn(make_float2(__uint_as_float(s[4 * c4]), __uint_as_float(s[4 * c4 + 1])),
-                         make_float2(-dq.x, -dq.y)));
-          const float2 d1 = __fmul2_rn(
-              make_float2(pr[4 * c4 + 2], pr[4 * c4 + 3]),
-              __fadd2_rn(make_float2(__uint_as_float(s[4 * c4 + 2]), __uint_as_float(s[4 * c4 + 3])),
-                         make_float2(-dq.z, -dq.w)));
-          pk[2 * c4] = sm100::pack_bf16x2(d0.x, d0.y);
-          pk[2 * c4 + 1] = sm100::pack_bf16x2(d1.x, d1.y);
-        }
-        if (!(ok = sm100::mbar_wait(&ds_empty[b], (u & 1) ^ 1, abort_flag, p.status))) break;
-        uint8_t* line = smem + OFF_DS + b * 16384 + kl_ * 128;
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t dp[32];
+          sm100::tmem_ld32(dp_addr + 32 * h2, dp);
+          sm100::tmem_ld_wait();
+          uint32_t w[16];
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          *reinterpret_cast<uint4*>(line + ((q ^ (kl_ & 7)) << 4)) =
-              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 dq = dvv[8 * h2 + c4];
+            const int c = 32 * h2 + 4 * c4;
+            const float2 p0 = make_float2(__uint_as_float(pk[c / 2] << 16),
+                                          __uint_as_float(pk[c / 2] & 0xFFFF0000u));
+            const float2 p1 = make_float2(__uint_as_float(pk[c / 2 + 1] << 16),
+                                          __uint_as_float(pk[c / 2 + 1] & 0xFFFF0000u));
+            const float2 d0 = __fmul2_rn(
+                p0,
+                __fadd2_rn(make_float2(__uint_as_float(dp[4 * c4]), __uint_as_float(dp[4 * c4 + 1])),
+                           make_float2(-dq.x, -dq.y)));
+            const float2 d1 = __fmul2_rn(
+                p1,
+                __fadd2_rn(make_float2(__uint_as_float(dp[4 * c4 + 2]),
+                                       __uint_as_float(dp[4 * c4 + 3])),
+                           make_float2(-dq.z, -dq.w)));
+            w[2 * c4] = sm100::pack_bf16x2(d0.x, d0.y);
+            w[2 * c4 + 1] = sm100::pack_bf16x2(d1.x, d1.y);
+          }
+          // 128-byte swizzle: 16-byte chunk q of line kl_ lands at q ^ (kl_ & 7)
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(line + (((4 * h2 + q) ^ (kl_ & 7)) << 4)) =
+                make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        }
         sm100::fence_proxy_async_smem();
         sm100::tc_fence_before();
-        sm100::mbar_arrive(&ds_full[b]);
+        __syncwarp();
+        if (sm100::lane_id() == 0) sm100::mbar_arrive(ds_full);
       }
       if (!ok) break;
       tq += it.T;
-      // ---------------- epilogue: dV, dK (x scale) for this key row
+      // ---------------- epilogue: dV, dK (x scale) of this key row, this warp's
+      // half of the columns
       if (!(ok = sm100::mbar_wait(dkv_full, ik & 1, abort_flag, p.status))) break;
       sm100::tc_fence_after();
       const bool live = key < p.Lk;
       const size_t orow = (static_cast<size_t>(it.b) * p.Hkv + it.hkv) * p.Lk + (live ? key : 0);
 #pragma unroll 1
       for (int m = 0; m < 2; ++m) {
-        __nv_bfloat16* dst = (m == 0 ? p.dV : p.dK) + orow * D;
+        __nv_bfloat16* dst = (m == 0 ? p.dV : p.dK) + orow * D + 64 * hf;
         const float f = (m == 0) ? 1.f : p.scale;
-        const uint32_t col = (m == 0) ? DV_COL : DK_COL;
+        const uint32_t col = ((m == 0) ? DV_COL : DK_COL) + 64 * hf;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t v[32];
           sm100::tmem_ld32(tmem + lane_base + col + c * 32, v);
           sm100::tmem_ld_wait();
@@ -589,61 +692,86 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       sm100::tc_fence_before();
-      sm100::mbar_arrive(dkv_empty);
+      __syncwarp();
+      if (sm100::lane_id() == 0) sm100::mbar_arrive(dkv_empty);
     }
-  } else {
+  } else if (warp >= W_DRAIN && warp < W_LOAD) {
     // ------------------------------------------------------------ dQ drain (one d column per thread)
-    // dQ^T of a query tile (lanes = head-dimension index, columns = 64 rows)
-    // is staged row-major in shared memory and added into the fp32
-    // accumulator with one 32 KB bulk reduce (the tile's rows are contiguous
-    // there); the staging buffer is reused once the previous reduce has read it.
-    const int dl = threadIdx.x - 128;  // TMEM lane = head-dimension index
+    // dQ^T of a query tile (lanes = head-dimension index, columns = 128 rows)
+    // is moved to registers and staged row-major in shared memory DQ_ROWS
+    // rows at a time; each staged block is added into the fp32 accumulator
+    // with one bulk reduce-add (its rows are contiguous there).  The TMEM
+    // columns are released once every column is in registers or staged; the
+    // staging buffer is reused once the previous reduce has read it.
+    const int tid = threadIdx.x - 32 * W_DRAIN;
+    const int dl = tid;  // TMEM lane = head-dimension index
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     float* stage = reinterpret_cast<float*>(smem + OFF_DQ);
     uint32_t tq = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
+    for (uint32_t ik = 0; ok; ++ik) {
+      int w;
+      if (!(ok = next_item(ik, w)) || w < 0) break;
       const Item it = get_item(p, w, nullptr);
       const int nq = it.T > 0 ? it.T / p.G : 0;
       for (int t = 0; t < it.T && ok; ++t) {
         const uint32_t cur = tq + t;
-        const int b = cur & 1;
-        const uint32_t u = cur >> 1;
         const int g = t / nq, i = it.i_lo + t % nq;
-        if (!(ok = sm100::mbar_wait(&dq_full[b], u & 1, abort_flag, p.status))) break;
+        const int qh = it.b * p.Hq + it.hkv * p.G + g;
+        float* acc_rows = p.dq_acc + (static_cast<size_t>(qh) * p.Lqp + i * BMQ) * D;
+        if (!(ok = sm100::mbar_wait(dq_full, cur & 1, abort_flag, p.status))) break;
         sm100::tc_fence_after();
-        uint32_t v[64];
-        sm100::tmem_ld32(tmem + lane_base + DP_COL0 + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        sm100::tmem_ld32(tmem + lane_base + DP_COL0 + b * 64 + 32,
-                         *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        // DQ_ROWS rows of the tile (fp32 values `v`, one per row, of this
+        // thread's d column) through the staging buffer into the accumulator
+        auto stage_round = [&](const uint32_t* v, int row0) {
+          // the previous reduce must have finished reading the staging buffer
+          if (tid == 0) bulk_wait_read_all();
+          sm100::named_bar_sync(1, 128);
+#pragma unroll
+          for (int c = 0; c < DQ_ROWS; ++c) stage[c * D + dl] = __uint_as_float(v[c]);
+          sm100::fence_proxy_async_smem();
+          sm100::named_bar_sync(1, 128);
+          if (tid == 0) bulk_reduce_add_f32(acc_rows + row0 * D, stage, DQ_ROWS * D * 4);
+        };
+        // rows 0-63 to registers, the first 32 of them out, rows 64-127 to
+        // registers: the columns go back to the MMA warp after one staging
+        // round, with at most 96 values held
+        uint32_t a[64], b[64];
+        sm100::tmem_ld32(tmem + lane_base + DP_COL, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+        sm100::tmem_ld32(tmem + lane_base + DP_COL + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
+        sm100::tmem_ld_wait();
+        stage_round(&a[0], 0);
+        sm100::tmem_ld32(tmem + lane_base + DP_COL + 64, *reinterpret_cast<uint32_t(*)[32]>(&b[0]));
+        sm100::tmem_ld32(tmem + lane_base + DP_COL + 96, *reinterpret_cast<uint32_t(*)[32]>(&b[32]));
         sm100::tmem_ld_wait();
         sm100::tc_fence_before();
-        sm100::mbar_arrive(&dq_empty[b]);
-        // the previous tile's reduce must have finished reading the staging buffer
-        if (threadIdx.x == 128) bulk_wait_read_all();
-        sm100::named_bar_sync(1, 128);
-#pragma unroll
-        for (int c = 0; c < 64; ++c) stage[c * D + dl] = __uint_as_float(v[c]);
-        sm100::fence_proxy_async_smem();
-        sm100::named_bar_sync(1, 128);
-        if (threadIdx.x == 128) {
-          const int qh = it.b * p.Hq + it.hkv * p.G + g;
-          bulk_reduce_add_f32(p.dq_acc + (static_cast<size_t>(qh) * p.Lqp + i * BMQ) * D, stage,
-                              BMQ * D * 4);
-        }
+        __syncwarp();
+        if (sm100::lane_id() == 0) sm100::mbar_arrive(dq_empty);
+        stage_round(&a[32], 32);
+        stage_round(&b[0], 64);
+        stage_round(&b[32], 96);
       }
       tq += it.T;
     }
     // the convert pass reads the accumulator after this kernel; the reduces
     // must be complete before the CTA exits
-    if (threadIdx.x == 128) bulk_wait_all();
+    if (tid == 0) bulk_wait_all();
   }
 
   sm100::tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == W_MMA) {
     sm100::tc_fence_after();
     sm100::tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0) {
+    // the last CTA to finish re-arms the dynamic scheduler for the next launch
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+      p.sched[0] = 0;
+      p.sched[1] = 0;
+      __threadfence();
+    }
   }
 }
 
@@ -678,6 +806,7 @@ inline attn_status_t launch(const Args& a, cudaStream_t s) {
   p.n_kv = (a.Lk + BN - 1) / BN;
   p.n_qt = p.Lqp / BMQ;
   p.n_items = a.B * a.Hkv * p.n_kv;
+  p.sched = a.status + 1;
   const int BH = a.B * a.Hq;
 
   // 1. prep
@@ -685,27 +814,33 @@ inline attn_status_t launch(const Args& a, cudaStream_t s) {
     const long long warps = static_cast<long long>(BH) * p.Lqp;
     bwd_prep_kernel<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, s>>>(
         a.O, a.dO, a.lse, p.dq_acc, lse2, Dv, BH, a.Lq, p.Lqp);
-    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    if (attn_host::report_launch(bwd_prep_kernel, "bwd_prep_kernel") != cudaSuccess)
+      return ATTN_ERR_CUDA;
   }
   // 2. main
   if (p.n_items > 0) {
     CUtensorMap tq, tdo, tk, tv;
     if (!make_tmap_rows(&tq, a.Q, a.Lq, BH, BMQ) || !make_tmap_rows(&tdo, a.dO, a.Lq, BH, BMQ) ||
         !make_tmap_rows(&tk, a.K, a.Lk, static_cast<long long>(a.B) * a.Hkv, BN) ||
-        !make_tmap_rows(&tv, a.V, a.Lk, static_cast<long long>(a.B) * a.Hkv, BN))
+        !make_tmap_rows(&tv, a.V, a.Lk, static_cast<long long>(a.B) * a.Hkv, BN)) {
+      attn_host::report(cudaErrorInvalidValue, "bwd tensor maps");
       return ATTN_ERR_CUDA;
-    if (attn_host::set_smem(bwd_main_kernel, SMEM_BYTES) != cudaSuccess)
+    }
+    if (attn_host::report(attn_host::set_smem(bwd_main_kernel, SMEM_BYTES),
+                          "bwd_main_kernel shared-memory attribute") != cudaSuccess)
       return ATTN_ERR_CUDA;
     const int grid = p.n_items < a.sms ? p.n_items : a.sms;
     bwd_main_kernel<<<grid, NTHREADS, SMEM_BYTES, s>>>(tq, tdo, tk, tv, p);
-    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    if (attn_host::report_launch(bwd_main_kernel, "bwd_main_kernel") != cudaSuccess)
+      return ATTN_ERR_CUDA;
   }
   // 3. dQ
   if (a.Lq > 0) {
     const size_t n4 = static_cast<size_t>(BH) * a.Lq * (D / 4);
     bwd_dq_convert_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, s>>>(
         p.dq_acc, a.dQ, BH, a.Lq, p.Lqp, a.scale);
-    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    if (attn_host::report_launch(bwd_dq_convert_kernel, "bwd_dq_convert_kernel") != cudaSuccess)
+      return ATTN_ERR_CUDA;
   }
   return ATTN_OK;
 }

@@ -123,6 +123,112 @@ __device__ __forceinline__ float transpose_reduce16(float (&v)[16], int hl) {
   return v[0];
 }
 
+// One stage of key rows for one compute warp: this warp's rows of the stage
+// (WROWS of SR, in steps of STEP rows: a half-warp per row, 16 lanes x d/16
+// elements) update the warp's running max m_run, per-lane sum l_lane and
+// unnormalised outputs o2 of the GP (padded) query heads.  q2: the heads'
+// query slices of this lane, pre-scaled by scale * log2(e).
+template <int D, int GP>
+__device__ __forceinline__ void stage_rows(const uint8_t* kst, const uint8_t* vst, int n, int warp,
+                                           int lane, int G, const float2 (&q2)[GP][D / 32],
+                                           float2 (&o2)[GP][D / 32], float& m_run,
+                                           float& l_lane) {
+  constexpr int EPL = D / 16;    // elements of a row per lane
+  constexpr int R = 16 / GP;     // rows per half-warp per step
+  constexpr int STEP = 2 * R;    // rows per warp per step
+  constexpr int WROWS = SR / NCW;
+  constexpr int ROWB = D * 2;    // bytes per row
+  const int half = lane >> 4, hl = lane & 15;
+  const int g_own = hl % GP;        // head of this lane's score
+  const int i_own = hl / GP;        // row (within the half's R rows) of this lane's score
+#pragma unroll 1
+  for (int rb = warp * WROWS; rb < warp * WROWS + WROWS; rb += STEP) {
+    if (rb >= n) break;
+    // ---- scores: partial dots of this lane's d-slice, then transpose-reduce
+    float part[16];
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int row = rb + half * R + i;
+      uint32_t kw[EPL / 2];
+      if (row < n) {
+        if constexpr (EPL == 8) {
+          const uint4 t = *reinterpret_cast<const uint4*>(kst + row * ROWB + hl * 16);
+          kw[0] = t.x; kw[1] = t.y; kw[2] = t.z; kw[3] = t.w;
+        } else {
+          const uint2 t = *reinterpret_cast<const uint2*>(kst + row * ROWB + hl * 8);
+          kw[0] = t.x; kw[1] = t.y;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < EPL / 2; ++c) kw[c] = 0u;
+      }
+      float2 kf[EPL / 2];
+#pragma unroll
+      for (int c = 0; c < EPL / 2; ++c) kf[c] = bf2(kw[c]);
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < EPL / 2; ++c) acc = __ffma2_rn(q2[g][c], kf[c], acc);
+        part[i * GP + g] = acc.x + acc.y;
+      }
+    }
+    const float sc = transpose_reduce16(part, hl);
+    const int my_row = rb + half * R + i_own;
+    const float s2 = (my_row < n && g_own < G) ? sc : -INFINITY;
+
+    // ---- online softmax for this step's rows (per head: lanes sharing g_own)
+    float m_blk = s2;
+#pragma unroll
+    for (int o = GP; o < 32; o <<= 1) m_blk = fmaxf(m_blk, __shfl_xor_sync(0xffffffffu, m_blk, o));
+    const bool need = m_blk > m_run + 8.0f;
+    if (__any_sync(0xffffffffu, need)) {
+      const float m_new = fmaxf(m_run, m_blk);
+      const float alpha = (m_run == -INFINITY) ? 0.f : sm100::ex2(m_run - m_new);
+      l_lane *= alpha;
+      m_run = m_new;
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        const float a = __shfl_sync(0xffffffffu, alpha, g);
+        const float2 a2 = make_float2(a, a);
+#pragma unroll
+        for (int c = 0; c < EPL / 2; ++c) o2[g][c] = __fmul2_rn(o2[g][c], a2);
+      }
+    }
+    const float pv = (s2 == -INFINITY) ? 0.f : sm100::ex2(s2 - m_run);
+    l_lane += pv;
+
+    // ---- o += p V for this half's rows
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int row = rb + half * R + i;
+      uint32_t vw[EPL / 2];
+      if (row < n) {
+        if constexpr (EPL == 8) {
+          const uint4 t = *reinterpret_cast<const uint4*>(vst + row * ROWB + hl * 16);
+          vw[0] = t.x; vw[1] = t.y; vw[2] = t.z; vw[3] = t.w;
+        } else {
+          const uint2 t = *reinterpret_cast<const uint2*>(vst + row * ROWB + hl * 8);
+          vw[0] = t.x; vw[1] = t.y;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < EPL / 2; ++c) vw[c] = 0u;
+      }
+      float2 vf[EPL / 2];
+#pragma unroll
+      for (int c = 0; c < EPL / 2; ++c) vf[c] = bf2(vw[c]);
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        const float pg = __shfl_sync(0xffffffffu, pv, half * 16 + i * GP + g);
+        const float2 p2 = make_float2(pg, pg);
+#pragma unroll
+        for (int c = 0; c < EPL / 2; ++c) o2[g][c] = __ffma2_rn(p2, vf[c], o2[g][c]);
+      }
+    }
+  }
+}
+
 // GP: query heads per key/value head, padded to 4 or 8 (heads >= G are inert).
 template <int D, int GP>
 __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) decode_split_kernel(const SplitParams p) {
@@ -228,8 +334,6 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) decode_split_kernel(con
 
   // ---------------------------------------------------------------- compute warps
   const int half = lane >> 4, hl = lane & 15;
-  const int g_own = hl % GP;        // head of this lane's score
-  const int i_own = hl / GP;        // row (within the half's R rows) of this lane's score
 
   // q of every head in the group, pre-scaled by scale * log2(e)
   float2 q2[GP][EPL / 2];
@@ -264,92 +368,7 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) decode_split_kernel(con
     const int n = min(SR, rows - s * SR);
     const uint8_t* kst = sK + slot * STAGE;
     const uint8_t* vst = sV + slot * STAGE;
-#pragma unroll 1
-    for (int rb = warp * WROWS; rb < warp * WROWS + WROWS; rb += STEP) {
-      if (rb >= n) break;
-      // ---- scores: partial dots of this lane's d-slice, then transpose-reduce
-      float part[16];
-#pragma unroll
-      for (int i = 0; i < R; ++i) {
-        const int row = rb + half * R + i;
-        uint32_t kw[EPL / 2];
-        if (row < n) {
-          if constexpr (EPL == 8) {
-            const uint4 t = *reinterpret_cast<const uint4*>(kst + row * ROWB + hl * 16);
-            kw[0] = t.x; kw[1] = t.y; kw[2] = t.z; kw[3] = t.w;
-          } else {
-            const uint2 t = *reinterpret_cast<const uint2*>(kst + row * ROWB + hl * 8);
-            kw[0] = t.x; kw[1] = t.y;
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < EPL / 2; ++c) kw[c] = 0u;
-        }
-        float2 kf[EPL / 2];
-#pragma unroll
-        for (int c = 0; c < EPL / 2; ++c) kf[c] = bf2(kw[c]);
-#pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int c = 0; c < EPL / 2; ++c) acc = __ffma2_rn(q2[g][c], kf[c], acc);
-          part[i * GP + g] = acc.x + acc.y;
-        }
-      }
-      const float sc = transpose_reduce16(part, hl);
-      const int my_row = rb + half * R + i_own;
-      const float s2 = (my_row < n && g_own < p.G) ? sc : -INFINITY;
-
-      // ---- online softmax for this step's rows (per head: lanes sharing g_own)
-      float m_blk = s2;
-#pragma unroll
-      for (int o = GP; o < 32; o <<= 1) m_blk = fmaxf(m_blk, __shfl_xor_sync(0xffffffffu, m_blk, o));
-      const bool need = m_blk > m_run + 8.0f;
-      if (__any_sync(0xffffffffu, need)) {
-        const float m_new = fmaxf(m_run, m_blk);
-        const float alpha = (m_run == -INFINITY) ? 0.f : sm100::ex2(m_run - m_new);
-        l_lane *= alpha;
-        m_run = m_new;
-#pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          const float a = __shfl_sync(0xffffffffu, alpha, g);
-          const float2 a2 = make_float2(a, a);
-#pragma unroll
-          for (int c = 0; c < EPL / 2; ++c) o2[g][c] = __fmul2_rn(o2[g][c], a2);
-        }
-      }
-      const float pv = (s2 == -INFINITY) ? 0.f : sm100::ex2(s2 - m_run);
-      l_lane += pv;
-
-      // ---- o += p V for this half's rows
-#pragma unroll
-      for (int i = 0; i < R; ++i) {
-        const int row = rb + half * R + i;
-        uint32_t vw[EPL / 2];
-        if (row < n) {
-          if constexpr (EPL == 8) {
-            const uint4 t = *reinterpret_cast<const uint4*>(vst + row * ROWB + hl * 16);
-            vw[0] = t.x; vw[1] = t.y; vw[2] = t.z; vw[3] = t.w;
-          } else {
-            const uint2 t = *reinterpret_cast<const uint2*>(vst + row * ROWB + hl * 8);
-            vw[0] = t.x; vw[1] = t.y;
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < EPL / 2; ++c) vw[c] = 0u;
-        }
-        float2 vf[EPL / 2];
-#pragma unroll
-        for (int c = 0; c < EPL / 2; ++c) vf[c] = bf2(vw[c]);
-#pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          const float pg = __shfl_sync(0xffffffffu, pv, half * 16 + i * GP + g);
-          const float2 p2 = make_float2(pg, pg);
-#pragma unroll
-          for (int c = 0; c < EPL / 2; ++c) o2[g][c] = __ffma2_rn(p2, vf[c], o2[g][c]);
-        }
-      }
-    }
+    stage_rows<D, GP>(kst, vst, n, warp, lane, p.G, q2, o2, m_run, l_lane);
     __syncwarp();
     if (lane == 0) sm100::mbar_arrive(&empty[slot]);
   }
@@ -452,13 +471,16 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const CombineParams p
 template <int D, int GP>
 cudaError_t launch_t(const SplitParams& sp, const CombineParams& cp, cudaStream_t s) {
   constexpr int smem = smem_bytes<D>();
-  cudaError_t e = attn_host::set_smem(decode_split_kernel<D, GP>, smem);
+  cudaError_t e = attn_host::report(attn_host::set_smem(decode_split_kernel<D, GP>, smem),
+                                    "decode_split_kernel shared-memory attribute");
   if (e != cudaSuccess) return e;
   dim3 grid(sp.nsm, sp.Hkv, sp.B);
   decode_split_kernel<D, GP><<<grid, NTHREADS, smem, s>>>(sp);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = attn_host::report_launch(decode_split_kernel<D, GP>, "decode_split_kernel")) !=
+      cudaSuccess)
+    return e;
   decode_combine_kernel<D><<<sp.B * sp.Hq, D, 0, s>>>(cp);
-  return cudaGetLastError();
+  return attn_host::report_launch(decode_combine_kernel<D>, "decode_combine_kernel");
 }
 
 // Paged cache description for launch(); Lmax is then max_blocks * page.

@@ -13,6 +13,9 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 #include <set>
 #include <tuple>
@@ -62,6 +65,38 @@ cudaError_t set_smem(K kernel, int bytes) {
   const unsigned long long ctx_after = ctx != 0 ? ctx : current_context_id();
   if (e == cudaSuccess && ctx_after != 0)
     done.insert(std::make_tuple(reinterpret_cast<const void*>(kernel), dev, ctx_after, bytes));
+  return e;
+}
+
+// With the environment variable ATTN_DEBUG set (to anything but "0"), a failed
+// CUDA call is reported on stderr with its site; the entry point still returns
+// ATTN_ERR_CUDA.  Returns `e`.
+inline cudaError_t report(cudaError_t e, const char* where) {
+  if (e != cudaSuccess) {
+    static const bool on = [] {
+      const char* v = std::getenv("ATTN_DEBUG");
+      return v && std::strcmp(v, "0") != 0;
+    }();
+    if (on) std::fprintf(stderr, "attn: %s: %s\n", where, cudaGetErrorString(e));
+  }
+  return e;
+}
+
+// report() for a kernel launch, adding the kernel's compiled resources.
+template <typename K>
+cudaError_t report_launch(K kernel, const char* where) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess && report(e, where) != cudaSuccess) {
+    const char* v = std::getenv("ATTN_DEBUG");
+    cudaFuncAttributes a;
+    if (v && std::strcmp(v, "0") != 0 &&
+        cudaFuncGetAttributes(&a, reinterpret_cast<const void*>(kernel)) == cudaSuccess)
+      std::fprintf(stderr,
+                   "attn: %s: %d registers per thread, at most %d threads per block, "
+                   "%zu bytes static and at most %d bytes dynamic shared memory\n",
+                   where, a.numRegs, a.maxThreadsPerBlock, a.sharedSizeBytes,
+                   a.maxDynamicSharedSizeBytes);
+  }
   return e;
 }
 
