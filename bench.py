@@ -665,7 +665,29 @@ def bwd_leg(steps, warmup, world, flush):
     st = attn.attn_read_device_status(ws)
     if st[0] != attn.ATTN_OK:
         raise RuntimeError(f"device status {st}")
-    return ms
+    del q, k, v, do, O, lse, dq, dk, dv, ws
+    torch.cuda.empty_cache()
+    # d = 64: the tiny workload's shape and a larger causal one
+    d64 = {}
+    for name, (B, H, L, causal) in (("tiny B1 H2 L256 d64, no mask", (1, 2, 256, False)),
+                                    ("B4 H16 L4096 d64 causal", (4, 16, 4096, True))):
+        shp = (B, H, L, 64)
+        q, k, v, do = (synth.normal_bf16_device(synth.workload_seed(1, t) ^ L, shp, dev)
+                       for t in ("q", "k", "v", "do"))
+        O, lse = attn.attn_fwd(q, k, v, causal=causal)
+        ws = torch.zeros(attn.attn_bwd_workspace_size(B, H, H, L, L, 64), dtype=torch.uint8,
+                         device=dev)
+        call = lambda: attn.attn_bwd(q, k, v, O, do, lse, causal=causal, workspace=ws,
+                                     stream=stream)
+        barrier(world)
+        t = timed_loop(call, steps, warmup, stream, flush)
+        st = attn.attn_read_device_status(ws)
+        if st[0] != attn.ATTN_OK:
+            raise RuntimeError(f"device status {st}")
+        d64[name] = (t, 10.0 * 64 * causal_pairs(L, L, causal) * B * H)
+        del q, k, v, do, O, lse, ws
+    torch.cuda.empty_cache()
+    return ms, d64
 
 
 # ------------------------------------------------------------------ CPU baseline (oracle)
@@ -889,8 +911,9 @@ def main():
             rep["decode_GBs"] = kv_bytes / (float(np.mean(dms)) * 1e-3) / 1e9
             rep["decode_paged_GBs"] = kv_bytes / (float(np.mean(pms)) * 1e-3) / 1e9
         if bms is not None:
-            rep["bwd_ms"] = float(np.mean(bms))
-            rep["bwd_TFLOPs"] = bwd_flops(BWD) / (float(np.mean(bms)) * 1e-3) / 1e12
+            rep["bwd_ms"] = float(np.mean(bms[0]))
+            rep["bwd_TFLOPs"] = bwd_flops(BWD) / (float(np.mean(bms[0])) * 1e-3) / 1e12
+            rep["bwd_d64"] = {n: float(np.mean(t)) for n, (t, _) in bms[1].items()}
         if lng is not None:
             for name in ("causal", "padded"):
                 rep[f"long_{name}_ms"] = float(np.mean(lng[0][name]))
@@ -993,6 +1016,7 @@ def main():
         }
         line["gpu_launches"] += 4 * args.steps
     if bms is not None:
+        bms, bd64 = bms
         bfl = bwd_flops(BWD)
         t_b = max_over_ranks(float(np.mean(bms)), world)
         ach = bfl / (float(np.mean(bms)) * 1e-3) / 1e12
@@ -1001,9 +1025,13 @@ def main():
             "unit": "TFLOP/s", "ms_per_step": t_b, "flops_per_step": bfl,
             "roofline": {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"],
-                         "traffic": traffic_per_launch("attn_bwd_impl::bwd_main_kernel")},
+                         "traffic": traffic_per_launch("attn_bwd_impl::bwd_main_kernel<128>")},
+            "d64": {name: {"ms_per_step": max_over_ranks(float(np.mean(t)), world),
+                           "value": world * fl / (max_over_ranks(float(np.mean(t)), world) * 1e-3)
+                           / 1e12, "unit": "TFLOP/s", "flops_per_step": fl}
+                    for name, (t, fl) in bd64.items()},
         }
-        line["gpu_launches"] += 3 * max(3, args.steps // 2)
+        line["gpu_launches"] += 3 * max(3, args.steps // 2) + 3 * 2 * max(3, args.steps // 2)
     if lng is not None:
         lms, lflops, kl = lng
         entry = {}

@@ -17,7 +17,6 @@
 #include "fwd_kernel.cuh"
 #include "launch_cache.cuh"
 #include "merge_kernel.cuh"
-#include "pad_kernel.cuh"
 
 namespace {
 
@@ -114,9 +113,9 @@ using attn_host::set_smem;
 
 }  // namespace
 
-bool attn_bwd_impl::make_tmap_rows(CUtensorMap* m, const void* base, int L, long long heads,
-                                   int box_rows) {
-  return make_tmap(m, base, attn_bwd_impl::D, L, heads, box_rows);
+bool attn_bwd_impl::make_tmap_rows(CUtensorMap* m, const void* base, int d, int L,
+                                   long long heads, int box_rows) {
+  return make_tmap(m, base, d, L, heads, box_rows);
 }
 
 // Shared launch of the forward kernel; p carries the layout-specific fields.
@@ -465,33 +464,8 @@ attn_status_t attn_fwd_splitkv_decode_paged(const attn_bf16_t* Q, const attn_bf1
 
 // ------------------------------------------------------------------ backward
 
-// d = 64 runs the d = 128 backward on zero-padded copies held in the workspace
-// after that backward's own scratch: Q, O, dO, dQ (query rows) then K, V, dK, dV
-// (key rows), 128 bf16 columns each.
-static size_t pad_region_bytes(int B, int Hq, int Hkv, int Lq, int Lk) {
-  const size_t q_rows = static_cast<size_t>(B) * Hq * (Lq > 0 ? Lq : 0);
-  const size_t k_rows = static_cast<size_t>(B) * Hkv * (Lk > 0 ? Lk : 0);
-  return 4 * (q_rows + k_rows) * 128 * 2;  // a multiple of 256
-}
-
 size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d) {
-  if (d == 64)
-    return kStatusBytes + attn_bwd_impl::scratch_bytes(B, Hq, Hkv, Lq, Lk, 128) +
-           pad_region_bytes(B, Hq, Hkv, Lq, Lk);
   return kStatusBytes + attn_bwd_impl::scratch_bytes(B, Hq, Hkv, Lq, Lk, d);
-}
-
-static cudaError_t copy_rows(const void* src, int src_cols, void* dst, int dst_cols,
-                             long long rows, int sms, cudaStream_t s) {
-  if (rows <= 0) return cudaSuccess;
-  const int sw = src_cols / 8, dw = dst_cols / 8;  // 16-byte chunks of bf16
-  const long long n = rows * dw;
-  const long long need = (n + attn_pad_impl::NTHREADS - 1) / attn_pad_impl::NTHREADS;
-  const long long cap = static_cast<long long>(sms) * 8;
-  attn_pad_impl::copy_rows_kernel<<<static_cast<int>(need < cap ? need : cap),
-                                    attn_pad_impl::NTHREADS, 0, s>>>(
-      reinterpret_cast<const uint4*>(src), sw, reinterpret_cast<uint4*>(dst), dw, rows);
-  return cudaGetLastError();
 }
 
 static attn_status_t bwd_batched(const attn_bf16_t* Q, const attn_bf16_t* K,
@@ -539,45 +513,6 @@ static attn_status_t bwd_batched(const attn_bf16_t* Q, const attn_bf16_t* K,
   a.status = reinterpret_cast<int*>(workspace);
   a.scratch = reinterpret_cast<uint8_t*>(workspace) + kStatusBytes;
   a.sms = sms;
-  if (d == 64) {
-    // pad to d = 128 (zero columns), run the d = 128 kernels, take the first 64
-    // columns of the gradients back out
-    const long long q_rows = static_cast<long long>(B) * Hq * Lq;
-    const long long k_rows = static_cast<long long>(B) * Hkv * Lk;
-    __nv_bfloat16* w = reinterpret_cast<__nv_bfloat16*>(
-        reinterpret_cast<uint8_t*>(workspace) + kStatusBytes +
-        attn_bwd_impl::scratch_bytes(B, Hq, Hkv, Lq, Lk, 128));
-    __nv_bfloat16* Qp = w;
-    __nv_bfloat16* Op = Qp + q_rows * 128;
-    __nv_bfloat16* dOp = Op + q_rows * 128;
-    __nv_bfloat16* dQp = dOp + q_rows * 128;
-    __nv_bfloat16* Kp = dQp + q_rows * 128;
-    __nv_bfloat16* Vp = Kp + k_rows * 128;
-    __nv_bfloat16* dKp = Vp + k_rows * 128;
-    __nv_bfloat16* dVp = dKp + k_rows * 128;
-    if (copy_rows(Q, 64, Qp, 128, q_rows, sms, s) != cudaSuccess ||
-        copy_rows(O, 64, Op, 128, q_rows, sms, s) != cudaSuccess ||
-        copy_rows(dO, 64, dOp, 128, q_rows, sms, s) != cudaSuccess ||
-        copy_rows(K, 64, Kp, 128, k_rows, sms, s) != cudaSuccess ||
-        copy_rows(V, 64, Vp, 128, k_rows, sms, s) != cudaSuccess)
-      return ATTN_ERR_CUDA;
-    a.Q = Qp;
-    a.O = Op;
-    a.dO = dOp;
-    a.K = Kp;
-    a.V = Vp;
-    a.dQ = dQp;
-    a.dK = dKp;
-    a.dV = dVp;
-    a.d = 128;
-    const attn_status_t st = attn_bwd_impl::launch(a, s);
-    if (st != ATTN_OK) return st;
-    if (copy_rows(dQp, 128, dQ, 64, q_rows, sms, s) != cudaSuccess ||
-        copy_rows(dKp, 128, dK, 64, k_rows, sms, s) != cudaSuccess ||
-        copy_rows(dVp, 128, dV, 64, k_rows, sms, s) != cudaSuccess)
-      return ATTN_ERR_CUDA;
-    return ATTN_OK;
-  }
   return attn_bwd_impl::launch(a, s);
 }
 

@@ -41,42 +41,53 @@ namespace attn_bwd_impl {
 
 constexpr int BN = 128;   // keys per work item (TMEM lanes)
 constexpr int BMQ = 128;  // query rows per query tile
-constexpr int D = 128;    // head dimension handled by the main kernel
 constexpr int NQS = 2;    // query-tile ring stages (Q with its log2-LSE and D); dO is single-buffered
 constexpr int NSMX = 8;   // P/dS warps: 4 lane quarters x 2 halves of the query rows
-constexpr int W_DRAIN = NSMX;        // warps 8-11: dQ^T drain
+constexpr int W_DRAIN = NSMX;        // warps 8-11: dQ drain
 constexpr int W_LOAD = NSMX + 4;     // warp 12: TMA producer
 constexpr int W_MMA = NSMX + 5;      // warp 13: MMA issuer
 constexpr int NTHREADS = 32 * (NSMX + 6);
 constexpr int NI = 4;                          // depth of the shared-memory item ring
 constexpr int ITEM_READERS = NSMX + 4 + 1;     // warps that read each item: P/dS, drain, MMA
-constexpr int DQ_ROWS = 32;          // query rows per dQ staging round (16 KB of fp32)
+constexpr int PANEL = 16384;  // one 128-byte-swizzled panel: 128 rows x 64 bf16 columns
+constexpr int DQ_ROWS = 32;   // query rows per dQ staging round (16 KB of fp32 at d = 128)
 
-// shared memory map (bytes); the swizzled panels are 1024-byte aligned.  A tile
-// of 128 rows x 128 bf16 columns is two 128-byte-swizzled panels of 64 columns
-// (16 KB each).
-constexpr int TILE = 32768;
-constexpr int PANEL = 16384;
-constexpr int OFF_K = 0;                        // [128 keys][d]
-constexpr int OFF_V = TILE;
-constexpr int OFF_Q = 2 * TILE;                 // NQS stages of [128 rows][d]
-constexpr int OFF_DO = OFF_Q + NQS * TILE;      // [128 rows][d]
-constexpr int OFF_DS = OFF_DO + TILE;           // dS^T [128 keys][128 rows]: panels of 64 rows
-constexpr int OFF_DQ = OFF_DS + TILE;           // dQ staging [DQ_ROWS][d] fp32
-constexpr int OFF_LD = OFF_DQ + DQ_ROWS * D * 4;  // stage s: lse2 [128] then D [128]
-constexpr int OFF_BAR = OFF_LD + NQS * 1024;
-constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
-static_assert(SMEM_BYTES <= 232448, "dynamic shared memory limit");
+// Layout for head dimension DH (64 or 128): shared memory map (bytes; the
+// swizzled panels are 1024-byte aligned; a 128-row tile is DH / 64 panels) and
+// the instruction descriptors whose N is the head dimension.
+template <int DH>
+struct Cfg {
+  static_assert(DH == 64 || DH == 128, "head dimension");
+  static constexpr int PANELS = DH / 64;
+  static constexpr int TILE = PANELS * PANEL;     // one 128-row bf16 tile
+  static constexpr int OFF_K = 0;                 // [128 keys][d]
+  static constexpr int OFF_V = TILE;
+  static constexpr int OFF_Q = 2 * TILE;          // NQS stages of [128 rows][d]
+  static constexpr int OFF_DO = OFF_Q + NQS * TILE;  // [128 rows][d]
+  static constexpr int OFF_DS = OFF_DO + TILE;    // dS^T [128 keys][128 rows]: panels of 64 rows
+  // d = 128: dQ^T (lanes = d) is staged row-major DQ_ROWS query rows at a time
+  // for bulk reduce-adds; d = 64 adds dQ rows straight from registers
+  static constexpr bool STAGED_DQ = DH == 128;
+  static constexpr int OFF_DQ = OFF_DS + 2 * PANEL;
+  static constexpr int OFF_LD = OFF_DQ + (STAGED_DQ ? DQ_ROWS * DH * 4 : 0);  // lse2 [128], D [128]
+  static constexpr int OFF_BAR = OFF_LD + NQS * 1024;
+  static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
+  static_assert(SMEM_BYTES <= 232448, "dynamic shared memory limit");
+  // dV += P^T dO and dK += dS^T Q (A K-major, B MN-major); dQ^T = K^T dS^T
+  // (M = d = 128, N = 128 rows) or dQ = dS K (M = 128 rows, N = d = 64), both
+  // operands MN-major
+  static constexpr uint32_t IDESC_DV = sm100::idesc_bf16_f32(128, DH, false, true);
+  static constexpr uint32_t IDESC_DQ = STAGED_DQ ? sm100::idesc_bf16_f32(128, BMQ, true, true)
+                                                 : sm100::idesc_bf16_f32(128, DH, true, true);
+};
 
 // TMEM columns (512 allocated)
 constexpr uint32_t S_COL = 0;     // S^T, overwritten by P^T (packed bf16) -- 128
-constexpr uint32_t DP_COL = 128;  // dP^T, then dQ^T of the same tile -- 128
-constexpr uint32_t DV_COL = 256;
-constexpr uint32_t DK_COL = 384;
+constexpr uint32_t DP_COL = 128;  // dP^T, then dQ of the same tile -- 128 (DH of them for dQ)
+constexpr uint32_t DV_COL = 256;  // DH columns
+constexpr uint32_t DK_COL = 384;  // DH columns
 
 constexpr uint32_t IDESC_S = sm100::idesc_bf16_f32(128, BMQ, false, false);
-constexpr uint32_t IDESC_DV = sm100::idesc_bf16_f32(128, D, false, true);
-constexpr uint32_t IDESC_DQ = sm100::idesc_bf16_f32(128, BMQ, true, true);
 
 // Exponentials on the FMA pipe (polynomial exp2) for column pairs cp with
 // (cp & 7) >= POLY_FROM: the 16384 exponentials of a tile take 1024 cycles on
@@ -107,7 +118,7 @@ inline size_t scratch_bytes(int B, int Hq, int, int Lq, int, int d) {
 }
 
 struct Params {
-  float* dq_acc;       // [B*Hq][Lqp][D] fp32
+  float* dq_acc;       // [B*Hq][Lqp][d] fp32
   const float* lse2;   // [B*Hq][Lqp]
   const float* Dvec;   // [B*Hq][Lqp]
   __nv_bfloat16* dK;
@@ -175,6 +186,12 @@ __device__ __forceinline__ Item get_item(const Params& p, int w, bool* bad) {
   return it;
 }
 
+// The t-th query tile an item visits: query head g of the group and query tile i.
+__device__ __forceinline__ void tile_of(const Item& it, int t, int nq, int& g, int& i) {
+  g = t / nq;
+  i = it.i_lo + t % nq;
+}
+
 // Bulk reduce-add of `bytes` fp32 values from shared to global memory (the
 // TMA unit performs the additions at L2), tracked by a bulk async-group.
 __device__ __forceinline__ void bulk_reduce_add_f32(float* gdst, const void* ssrc, uint32_t bytes) {
@@ -194,6 +211,13 @@ __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// acc[0..3] += (a, b, c, d): one 16-byte vector reduction, performed at L2.
+__device__ __forceinline__ void red_add_v4_f32(float* acc, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(acc), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
                                          uint64_t* bar) {
   asm volatile(
@@ -205,29 +229,41 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 
 // ------------------------------------------------------------------ prep
 
+template <int DH>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* O,
                                                         const __nv_bfloat16* dO,
                                                         const float* lse, float* dq_acc,
                                                         float* lse2, float* Dv, int BH, int Lq,
                                                         int Lqp) {
+  constexpr int EPL = DH / 32;  // elements per lane
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= BH * Lqp) return;
   const int bh = warp / Lqp, r = warp % Lqp;
   float acc = 0.f;
   if (r < Lq) {
-    const size_t off = (static_cast<size_t>(bh) * Lq + r) * D + lane * 4;
-    const uint2 a = *reinterpret_cast<const uint2*>(O + off);
-    const uint2 g = *reinterpret_cast<const uint2*>(dO + off);
-    acc = __uint_as_float(a.x << 16) * __uint_as_float(g.x << 16) +
-          __uint_as_float(a.x & 0xFFFF0000u) * __uint_as_float(g.x & 0xFFFF0000u) +
-          __uint_as_float(a.y << 16) * __uint_as_float(g.y << 16) +
-          __uint_as_float(a.y & 0xFFFF0000u) * __uint_as_float(g.y & 0xFFFF0000u);
+    const size_t off = (static_cast<size_t>(bh) * Lq + r) * DH + lane * EPL;
+    uint32_t a[EPL / 2], g[EPL / 2];
+    if constexpr (EPL == 4) {
+      const uint2 ta = *reinterpret_cast<const uint2*>(O + off);
+      const uint2 tg = *reinterpret_cast<const uint2*>(dO + off);
+      a[0] = ta.x; a[1] = ta.y; g[0] = tg.x; g[1] = tg.y;
+    } else {
+      a[0] = *reinterpret_cast<const uint32_t*>(O + off);
+      g[0] = *reinterpret_cast<const uint32_t*>(dO + off);
+    }
+#pragma unroll
+    for (int e = 0; e < EPL / 2; ++e)
+      acc += __uint_as_float(a[e] << 16) * __uint_as_float(g[e] << 16) +
+             __uint_as_float(a[e] & 0xFFFF0000u) * __uint_as_float(g[e] & 0xFFFF0000u);
   }
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  reinterpret_cast<float4*>(dq_acc + static_cast<size_t>(warp) * D)[lane] =
-      make_float4(0.f, 0.f, 0.f, 0.f);
+  float* zrow = dq_acc + static_cast<size_t>(warp) * DH + lane * EPL;
+  if constexpr (EPL == 4)
+    *reinterpret_cast<float4*>(zrow) = make_float4(0.f, 0.f, 0.f, 0.f);
+  else
+    *reinterpret_cast<float2*>(zrow) = make_float2(0.f, 0.f);
   if (lane == 0) {
     Dv[warp] = acc;
     float l2 = INFINITY;
@@ -239,36 +275,39 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* O,
   }
 }
 
+template <int DH>
 __global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const float* dq_acc,
                                                               __nv_bfloat16* dQ, int BH, int Lq,
                                                               int Lqp, float scale) {
   const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // 4 elements
-  const size_t total = static_cast<size_t>(BH) * Lq * (D / 4);
+  const size_t total = static_cast<size_t>(BH) * Lq * (DH / 4);
   if (i >= total) return;
-  const size_t row = i / (D / 4);
-  const int c4 = static_cast<int>(i % (D / 4));
+  const size_t row = i / (DH / 4);
+  const int c4 = static_cast<int>(i % (DH / 4));
   const int bh = static_cast<int>(row / Lq), r = static_cast<int>(row % Lq);
   const float4 v =
-      reinterpret_cast<const float4*>(dq_acc + (static_cast<size_t>(bh) * Lqp + r) * D)[c4];
+      reinterpret_cast<const float4*>(dq_acc + (static_cast<size_t>(bh) * Lqp + r) * DH)[c4];
   uint2 o;
   o.x = sm100::pack_bf16x2(v.x * scale, v.y * scale);
   o.y = sm100::pack_bf16x2(v.z * scale, v.w * scale);
-  reinterpret_cast<uint2*>(dQ + row * D)[c4] = o;
+  reinterpret_cast<uint2*>(dQ + row * DH)[c4] = o;
 }
 
 // ------------------------------------------------------------------ main
 
+template <int DH>
 __global__ void __launch_bounds__(NTHREADS, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmdO,
                     const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const Params p) {
+  using C = Cfg<DH>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = sm100::smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
   const uint32_t sbase = sm100::smem_u32(smem);
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* kv_full = bars + 0;
   uint64_t* kv_empty = bars + 1;
   uint64_t* q_full = bars + 2;     // [NQS]
@@ -363,33 +402,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (w < 0) break;
         const Item it = get_item(p, w, nullptr);
         if (!(ok = sm100::mbar_wait(kv_empty, (ik & 1) ^ 1, abort_flag, p.status))) break;
-        sm100::mbar_arrive_expect_tx(kv_full, 2 * TILE);
+        sm100::mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
         ++kv_issued;
         const int kvh = it.b * p.Hkv + it.hkv;
-        for (int c = 0; c < 2; ++c) {
-          sm100::tma_load_3d(&tmK, kv_full, smem + OFF_K + c * PANEL, c * 64, it.n * BN, kvh);
-          sm100::tma_load_3d(&tmV, kv_full, smem + OFF_V + c * PANEL, c * 64, it.n * BN, kvh);
+        for (int c = 0; c < C::PANELS; ++c) {
+          sm100::tma_load_3d(&tmK, kv_full, smem + C::OFF_K + c * PANEL, c * 64, it.n * BN, kvh);
+          sm100::tma_load_3d(&tmV, kv_full, smem + C::OFF_V + c * PANEL, c * 64, it.n * BN, kvh);
         }
         const int nq = it.T > 0 ? it.T / p.G : 0;
         for (int t = 0; t < it.T && ok; ++t, ++tq) {
-          const int g = t / nq, i = it.i_lo + t % nq;
+          int g, i;
+          tile_of(it, t, nq, g, i);
           const int slot = tq % NQS;
           const int qh = it.b * p.Hq + it.hkv * p.G + g;
           if (!(ok = sm100::mbar_wait(&q_empty[slot], ((tq / NQS) & 1) ^ 1, abort_flag,
                                       p.status)))
             break;
-          sm100::mbar_arrive_expect_tx(&q_full[slot], TILE + 1024);
-          for (int c = 0; c < 2; ++c)
-            sm100::tma_load_3d(&tmQ, &q_full[slot], smem + OFF_Q + slot * TILE + c * PANEL,
+          sm100::mbar_arrive_expect_tx(&q_full[slot], C::TILE + 1024);
+          for (int c = 0; c < C::PANELS; ++c)
+            sm100::tma_load_3d(&tmQ, &q_full[slot], smem + C::OFF_Q + slot * C::TILE + c * PANEL,
                                c * 64, i * BMQ, qh);
           const size_t rowoff = static_cast<size_t>(qh) * p.Lqp + i * BMQ;
-          bulk_g2s(smem + OFF_LD + slot * 1024, p.lse2 + rowoff, 512, &q_full[slot]);
-          bulk_g2s(smem + OFF_LD + slot * 1024 + 512, p.Dvec + rowoff, 512, &q_full[slot]);
+          bulk_g2s(smem + C::OFF_LD + slot * 1024, p.lse2 + rowoff, 512, &q_full[slot]);
+          bulk_g2s(smem + C::OFF_LD + slot * 1024 + 512, p.Dvec + rowoff, 512, &q_full[slot]);
           last_q[slot] = static_cast<int>(tq);
           if (!(ok = sm100::mbar_wait(do_empty, (tq & 1) ^ 1, abort_flag, p.status))) break;
-          sm100::mbar_arrive_expect_tx(do_full, TILE);
-          for (int c = 0; c < 2; ++c)
-            sm100::tma_load_3d(&tmdO, do_full, smem + OFF_DO + c * PANEL, c * 64, i * BMQ, qh);
+          sm100::mbar_arrive_expect_tx(do_full, C::TILE);
+          for (int c = 0; c < C::PANELS; ++c)
+            sm100::tma_load_3d(&tmdO, do_full, smem + C::OFF_DO + c * PANEL, c * 64, i * BMQ, qh);
           last_do = static_cast<int>(tq);
         }
       }
@@ -412,9 +452,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     {
       uint32_t tq = 0, ik = 0;
       bool ok = true;
-      const uint32_t kA = sbase + OFF_K, vA = sbase + OFF_V;
-      const uint32_t doA = sbase + OFF_DO, dsA = sbase + OFF_DS;
-      auto qA = [&](int slot) { return sbase + OFF_Q + slot * TILE; };
+      const uint32_t kA = sbase + C::OFF_K, vA = sbase + C::OFF_V;
+      const uint32_t doA = sbase + C::OFF_DO, dsA = sbase + C::OFF_DS;
+      auto qA = [&](int slot) { return sbase + C::OFF_Q + slot * C::TILE; };
       auto commit = [&](uint64_t* bar) {
         if (leader) sm100::tc_commit(bar);
         __syncwarp();
@@ -425,16 +465,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint64_t bd = sm100::sdesc_sw128(b, 16, 1024);
         if (leader) {
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
+          for (int k = 0; k < DH / 16; ++k) {
             const uint64_t o = static_cast<uint64_t>(((k >> 2) * PANEL + (k & 3) * 32) >> 4);
             sm100::mma_ss(tmem + dcol, ad + o, bd + o, IDESC_S, k > 0);
           }
         }
       };
-      const uint64_t kd_mn = sm100::sdesc_sw128(kA, PANEL, 1024);   // K^T: MN-major A over d
+      const uint64_t kd_mn = sm100::sdesc_sw128(kA, PANEL, 1024);   // K: MN-major B over d
       const uint64_t do_mn = sm100::sdesc_sw128(doA, PANEL, 1024);  // dO: MN-major B over d
       const uint64_t ds_k = sm100::sdesc_sw128(dsA, 16, 1024);      // dS^T: K-major A over rows
-      const uint64_t ds_mn = sm100::sdesc_sw128(dsA, PANEL, 1024);  // dS^T: MN-major B over rows
+      const uint64_t ds_mn = sm100::sdesc_sw128(dsA, PANEL, 1024);  // dS: MN-major A over rows
       for (; ok; ++ik) {
         int w;
         if (!(ok = next_item(ik, w)) || w < 0) break;
@@ -467,7 +507,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int k = 0; k < BMQ / 16; ++k)
               sm100::mma_ss(tmem + DK_COL, ds_k + ((((k >> 2) * PANEL) + (k & 3) * 32) >> 4),
-                            q_mn + ((k * 2048) >> 4), IDESC_DV, (!first || k > 0) ? 1u : 0u);
+                            q_mn + ((k * 2048) >> 4), C::IDESC_DV, (!first || k > 0) ? 1u : 0u);
           }
           commit(&q_empty[tile % NQS]);
         };
@@ -492,17 +532,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int k = 0; k < BMQ / 16; ++k)
               sm100::mma_ts(tmem + DV_COL, tmem + S_COL + (k >> 2) * 64 + (k & 3) * 8,
-                            do_mn + ((k * 2048) >> 4), IDESC_DV, (t > 0 || k > 0) ? 1u : 0u);
+                            do_mn + ((k * 2048) >> 4), C::IDESC_DV, (t > 0 || k > 0) ? 1u : 0u);
           }
           commit(do_empty);
-          // dQ^T = K^T dS^T into the dP^T columns
+          // into the dP^T columns: d = 128, dQ^T = K^T dS^T (lanes = d; A = K^T,
+          // B = dS^T, both MN-major); d = 64, dQ = dS K (lanes = query rows;
+          // A = dS, B = K, both MN-major)
           if (!(ok = sm100::mbar_wait(ds_full, par, abort_flag, p.status))) break;
           sm100::tc_fence_after();
           if (leader) {
 #pragma unroll
-            for (int k = 0; k < BN / 16; ++k)
-              sm100::mma_ss(tmem + DP_COL, kd_mn + ((k * 2048) >> 4), ds_mn + ((k * 2048) >> 4),
-                            IDESC_DQ, k > 0 ? 1u : 0u);
+            for (int k = 0; k < BN / 16; ++k) {
+              const uint64_t kk = kd_mn + ((k * 2048) >> 4), dd = ds_mn + ((k * 2048) >> 4);
+              if constexpr (C::STAGED_DQ)
+                sm100::mma_ss(tmem + DP_COL, kk, dd, C::IDESC_DQ, k > 0 ? 1u : 0u);
+              else
+                sm100::mma_ss(tmem + DP_COL, dd, kk, C::IDESC_DQ, k > 0 ? 1u : 0u);
+            }
           }
           commit(dq_full);
           // S^T of the next query tile (P^T of this one was read by dV above)
@@ -550,8 +596,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t cur = tq + t;
         const int slot = cur % NQS;
         const uint32_t par = cur & 1;
-        const int i = it.i_lo + t % nq;
-        const float* l2s = reinterpret_cast<const float*>(smem + OFF_LD + slot * 1024) + 64 * hf;
+        int g_unused, i;
+        tile_of(it, t, nq, g_unused, i);
+        const float* l2s = reinterpret_cast<const float*>(smem + C::OFF_LD + slot * 1024) + 64 * hf;
         const float* dsv = l2s + 128;
         // lse2 / D of this tile were delivered on q_full
         if (!(ok = sm100::mbar_wait(&q_full[slot], (cur / NQS) & 1, abort_flag, p.status)))
@@ -621,7 +668,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // dS = P o (dP - D), written K-major (row-contiguous per key) to panel hf
         if (!(ok = sm100::mbar_wait(dp_full, par, abort_flag, p.status))) break;
         sm100::tc_fence_after();
-        uint8_t* line = smem + OFF_DS + hf * PANEL + kl_ * 128;
+        uint8_t* line = smem + C::OFF_DS + hf * PANEL + kl_ * 128;
         const float4* dvv = reinterpret_cast<const float4*>(dsv);
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -670,11 +717,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const size_t orow = (static_cast<size_t>(it.b) * p.Hkv + it.hkv) * p.Lk + (live ? key : 0);
 #pragma unroll 1
       for (int m = 0; m < 2; ++m) {
-        __nv_bfloat16* dst = (m == 0 ? p.dV : p.dK) + orow * D + 64 * hf;
+        __nv_bfloat16* dst = (m == 0 ? p.dV : p.dK) + orow * DH + (DH / 2) * hf;
         const float f = (m == 0) ? 1.f : p.scale;
-        const uint32_t col = ((m == 0) ? DV_COL : DK_COL) + 64 * hf;
+        const uint32_t col = ((m == 0) ? DV_COL : DK_COL) + (DH / 2) * hf;
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < DH / 64; ++c) {
           uint32_t v[32];
           sm100::tmem_ld32(tmem + lane_base + col + c * 32, v);
           sm100::tmem_ld_wait();
@@ -696,17 +743,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (sm100::lane_id() == 0) sm100::mbar_arrive(dkv_empty);
     }
   } else if (warp >= W_DRAIN && warp < W_LOAD) {
-    // ------------------------------------------------------------ dQ drain (one d column per thread)
-    // dQ^T of a query tile (lanes = head-dimension index, columns = 128 rows)
-    // is moved to registers and staged row-major in shared memory DQ_ROWS
-    // rows at a time; each staged block is added into the fp32 accumulator
-    // with one bulk reduce-add (its rows are contiguous there).  The TMEM
-    // columns are released once every column is in registers or staged; the
-    // staging buffer is reused once the previous reduce has read it.
-    const int tid = threadIdx.x - 32 * W_DRAIN;
-    const int dl = tid;  // TMEM lane = head-dimension index
+    // ------------------------------------------------------------ dQ drain
+    // d = 128: dQ^T of a query tile (lanes = head-dimension index, columns =
+    // the tile's 128 rows) is moved to registers and staged row-major in shared
+    // memory DQ_ROWS rows at a time; each staged block is added into the fp32
+    // accumulator with one bulk reduce-add (its rows are contiguous there).
+    // The TMEM columns are released once every column is in registers or
+    // staged; the staging buffer is reused once the previous reduce has read it.
+    // d = 64: dQ (lanes = the tile's rows) goes to registers one row per thread
+    // and is added with 16-byte vector reductions straight from registers.
+    const int tid = threadIdx.x - 32 * W_DRAIN;  // = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    float* stage = reinterpret_cast<float*>(smem + OFF_DQ);
+    float* stage = reinterpret_cast<float*>(smem + C::OFF_DQ);
     uint32_t tq = 0;
     bool ok = true;
     for (uint32_t ik = 0; ok; ++ik) {
@@ -716,46 +764,67 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int nq = it.T > 0 ? it.T / p.G : 0;
       for (int t = 0; t < it.T && ok; ++t) {
         const uint32_t cur = tq + t;
-        const int g = t / nq, i = it.i_lo + t % nq;
+        int g, i;
+        tile_of(it, t, nq, g, i);
         const int qh = it.b * p.Hq + it.hkv * p.G + g;
-        float* acc_rows = p.dq_acc + (static_cast<size_t>(qh) * p.Lqp + i * BMQ) * D;
+        float* acc_rows = p.dq_acc + (static_cast<size_t>(qh) * p.Lqp + i * BMQ) * DH;
         if (!(ok = sm100::mbar_wait(dq_full, cur & 1, abort_flag, p.status))) break;
         sm100::tc_fence_after();
-        // DQ_ROWS rows of the tile (fp32 values `v`, one per row, of this
-        // thread's d column) through the staging buffer into the accumulator
-        auto stage_round = [&](const uint32_t* v, int row0) {
-          // the previous reduce must have finished reading the staging buffer
-          if (tid == 0) bulk_wait_read_all();
-          sm100::named_bar_sync(1, 128);
+        if constexpr (C::STAGED_DQ) {
+          // DQ_ROWS rows of the tile (fp32 values `v`, one per row, of this
+          // thread's d column) through the staging buffer into the accumulator
+          auto stage_round = [&](const uint32_t* v, int row0) {
+            // the previous reduce must have finished reading the staging buffer
+            if (tid == 0) bulk_wait_read_all();
+            sm100::named_bar_sync(1, 128);
 #pragma unroll
-          for (int c = 0; c < DQ_ROWS; ++c) stage[c * D + dl] = __uint_as_float(v[c]);
-          sm100::fence_proxy_async_smem();
-          sm100::named_bar_sync(1, 128);
-          if (tid == 0) bulk_reduce_add_f32(acc_rows + row0 * D, stage, DQ_ROWS * D * 4);
-        };
-        // rows 0-63 to registers, the first 32 of them out, rows 64-127 to
-        // registers: the columns go back to the MMA warp after one staging
-        // round, with at most 96 values held
-        uint32_t a[64], b[64];
-        sm100::tmem_ld32(tmem + lane_base + DP_COL, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
-        sm100::tmem_ld32(tmem + lane_base + DP_COL + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
-        sm100::tmem_ld_wait();
-        stage_round(&a[0], 0);
-        sm100::tmem_ld32(tmem + lane_base + DP_COL + 64, *reinterpret_cast<uint32_t(*)[32]>(&b[0]));
-        sm100::tmem_ld32(tmem + lane_base + DP_COL + 96, *reinterpret_cast<uint32_t(*)[32]>(&b[32]));
-        sm100::tmem_ld_wait();
-        sm100::tc_fence_before();
-        __syncwarp();
-        if (sm100::lane_id() == 0) sm100::mbar_arrive(dq_empty);
-        stage_round(&a[32], 32);
-        stage_round(&b[0], 64);
-        stage_round(&b[32], 96);
+            for (int c = 0; c < DQ_ROWS; ++c) stage[c * DH + tid] = __uint_as_float(v[c]);
+            sm100::fence_proxy_async_smem();
+            sm100::named_bar_sync(1, 128);
+            if (tid == 0) bulk_reduce_add_f32(acc_rows + row0 * DH, stage, DQ_ROWS * DH * 4);
+          };
+          // rows 0-63 to registers, the first 32 of them out, rows 64-127 to
+          // registers: the columns go back to the MMA warp after one staging
+          // round, with at most 96 values held
+          uint32_t a[64], b[64];
+          sm100::tmem_ld32(tmem + lane_base + DP_COL, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+          sm100::tmem_ld32(tmem + lane_base + DP_COL + 32,
+                           *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
+          sm100::tmem_ld_wait();
+          stage_round(&a[0], 0);
+          sm100::tmem_ld32(tmem + lane_base + DP_COL + 64,
+                           *reinterpret_cast<uint32_t(*)[32]>(&b[0]));
+          sm100::tmem_ld32(tmem + lane_base + DP_COL + 96,
+                           *reinterpret_cast<uint32_t(*)[32]>(&b[32]));
+          sm100::tmem_ld_wait();
+          sm100::tc_fence_before();
+          __syncwarp();
+          if (sm100::lane_id() == 0) sm100::mbar_arrive(dq_empty);
+          stage_round(&a[32], 32);
+          stage_round(&b[0], 64);
+          stage_round(&b[32], 96);
+        } else {
+          uint32_t v[64];
+          sm100::tmem_ld32(tmem + lane_base + DP_COL, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+          sm100::tmem_ld32(tmem + lane_base + DP_COL + 32,
+                           *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+          sm100::tmem_ld_wait();
+          // the whole row has left TMEM: the columns are free for dP^T
+          sm100::tc_fence_before();
+          __syncwarp();
+          if (sm100::lane_id() == 0) sm100::mbar_arrive(dq_empty);
+          float* acc_row = acc_rows + tid * DH;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            red_add_v4_f32(acc_row + 4 * j, __uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                           __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+        }
       }
       tq += it.T;
     }
-    // the convert pass reads the accumulator after this kernel; the reduces
-    // must be complete before the CTA exits
-    if (tid == 0) bulk_wait_all();
+    // the convert pass reads the accumulator after this kernel; the bulk
+    // reduces must be complete before the CTA exits
+    if (C::STAGED_DQ && tid == 0) bulk_wait_all();
   }
 
   sm100::tc_fence_before();
@@ -777,10 +846,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 // ------------------------------------------------------------------ host side
 
-bool make_tmap_rows(CUtensorMap* m, const void* base, int L, long long heads, int box_rows);
+bool make_tmap_rows(CUtensorMap* m, const void* base, int d, int L, long long heads,
+                    int box_rows);
 
-inline attn_status_t launch(const Args& a, cudaStream_t s) {
-  if (a.d != D) return ATTN_ERR_UNSUPPORTED;
+template <int DH>
+attn_status_t launch_d(const Args& a, cudaStream_t s) {
+  using C = Cfg<DH>;
   Params p;
   p.B = a.B;
   p.Hq = a.Hq;
@@ -797,7 +868,7 @@ inline attn_status_t launch(const Args& a, cudaStream_t s) {
   p.status = a.status;
   const size_t rows = static_cast<size_t>(a.B) * a.Hq * p.Lqp;
   p.dq_acc = reinterpret_cast<float*>(a.scratch);
-  float* lse2 = reinterpret_cast<float*>(a.scratch + rows * D * 4);
+  float* lse2 = reinterpret_cast<float*>(a.scratch + rows * DH * 4);
   float* Dv = lse2 + rows;
   p.lse2 = lse2;
   p.Dvec = Dv;
@@ -812,37 +883,44 @@ inline attn_status_t launch(const Args& a, cudaStream_t s) {
   // 1. prep
   if (a.Lq > 0) {
     const long long warps = static_cast<long long>(BH) * p.Lqp;
-    bwd_prep_kernel<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, s>>>(
+    bwd_prep_kernel<DH><<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, s>>>(
         a.O, a.dO, a.lse, p.dq_acc, lse2, Dv, BH, a.Lq, p.Lqp);
-    if (attn_host::report_launch(bwd_prep_kernel, "bwd_prep_kernel") != cudaSuccess)
+    if (attn_host::report_launch(bwd_prep_kernel<DH>, "bwd_prep_kernel") != cudaSuccess)
       return ATTN_ERR_CUDA;
   }
   // 2. main
   if (p.n_items > 0) {
     CUtensorMap tq, tdo, tk, tv;
-    if (!make_tmap_rows(&tq, a.Q, a.Lq, BH, BMQ) || !make_tmap_rows(&tdo, a.dO, a.Lq, BH, BMQ) ||
-        !make_tmap_rows(&tk, a.K, a.Lk, static_cast<long long>(a.B) * a.Hkv, BN) ||
-        !make_tmap_rows(&tv, a.V, a.Lk, static_cast<long long>(a.B) * a.Hkv, BN)) {
+    if (!make_tmap_rows(&tq, a.Q, DH, a.Lq, BH, BMQ) || !make_tmap_rows(&tdo, a.dO, DH, a.Lq, BH, BMQ) ||
+        !make_tmap_rows(&tk, a.K, DH, a.Lk, static_cast<long long>(a.B) * a.Hkv, BN) ||
+        !make_tmap_rows(&tv, a.V, DH, a.Lk, static_cast<long long>(a.B) * a.Hkv, BN)) {
       attn_host::report(cudaErrorInvalidValue, "bwd tensor maps");
       return ATTN_ERR_CUDA;
     }
-    if (attn_host::report(attn_host::set_smem(bwd_main_kernel, SMEM_BYTES),
+    if (attn_host::report(attn_host::set_smem(bwd_main_kernel<DH>, C::SMEM_BYTES),
                           "bwd_main_kernel shared-memory attribute") != cudaSuccess)
       return ATTN_ERR_CUDA;
     const int grid = p.n_items < a.sms ? p.n_items : a.sms;
-    bwd_main_kernel<<<grid, NTHREADS, SMEM_BYTES, s>>>(tq, tdo, tk, tv, p);
-    if (attn_host::report_launch(bwd_main_kernel, "bwd_main_kernel") != cudaSuccess)
+    bwd_main_kernel<DH><<<grid, NTHREADS, C::SMEM_BYTES, s>>>(tq, tdo, tk, tv, p);
+    if (attn_host::report_launch(bwd_main_kernel<DH>, "bwd_main_kernel") != cudaSuccess)
       return ATTN_ERR_CUDA;
   }
   // 3. dQ
   if (a.Lq > 0) {
-    const size_t n4 = static_cast<size_t>(BH) * a.Lq * (D / 4);
-    bwd_dq_convert_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, s>>>(
+    const size_t n4 = static_cast<size_t>(BH) * a.Lq * (DH / 4);
+    bwd_dq_convert_kernel<DH><<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, s>>>(
         p.dq_acc, a.dQ, BH, a.Lq, p.Lqp, a.scale);
-    if (attn_host::report_launch(bwd_dq_convert_kernel, "bwd_dq_convert_kernel") != cudaSuccess)
+    if (attn_host::report_launch(bwd_dq_convert_kernel<DH>, "bwd_dq_convert_kernel") !=
+        cudaSuccess)
       return ATTN_ERR_CUDA;
   }
   return ATTN_OK;
+}
+
+inline attn_status_t launch(const Args& a, cudaStream_t s) {
+  if (a.d == 128) return launch_d<128>(a, s);
+  if (a.d == 64) return launch_d<64>(a, s);
+  return ATTN_ERR_UNSUPPORTED;
 }
 
 }  // namespace attn_bwd_impl

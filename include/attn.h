@@ -274,11 +274,9 @@ attn_status_t attn_fwd_splitkv_decode_paged(const attn_bf16_t* Q, const attn_bf1
  *   Q, O, dO [B,Hq,Lq,d] bf16; K, V [B,Hkv,Lk,d] bf16; lse [B,Hq,Lq] fp32 as
  *   written by attn_fwd for the same arguments.  dQ [B,Hq,Lq,d], dK, dV
  *   [B,Hkv,Lk,d] bf16 are written.  Same mask arguments as attn_fwd.
- *   The workspace holds fp32 accumulators for dQ and D.  The kernels are
- *   written for d = 128; d = 64 runs them on zero-padded 128-column copies of
- *   Q, K, V, O and dO held in the workspace (zero columns change neither P nor
- *   dS) and copies out the gradients' first 64 columns: exact, at twice the
- *   minimum tensor work (attn_bwd_workspace_size includes the copies).
+ *   The workspace holds the fp32 accumulator for dQ and the per-row log2-LSE
+ *   and D (query rows padded to a multiple of 128 per head): nothing of size
+ *   Lq x Lk.  d = 64 and d = 128 each have their own kernels.
  */
 size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d);
 attn_status_t attn_bwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf16_t* V,

@@ -43,15 +43,14 @@ def test_workspace_sizes_are_closed_forms(lib):
     # decode: fp32 partial output and log-sum-exp per (sequence, head, 2048-key chunk)
     n = 64 * 32 * 16
     assert attn.attn_decode_workspace_size(64, 32, 8, 32768, 128) == 256 + ((n * 128 * 4 + n * 4 + 255) // 256) * 256
-    # backward: fp32 dQ accumulator and D per query row; nothing of size Lq x Lk
-    rows = 2 * 16 * 8192  # query rows, padded per head to a multiple of 64
+    # backward: fp32 dQ accumulator (d columns), log2-LSE and D per query row;
+    # nothing of size Lq x Lk
+    rows = 2 * 16 * 8192  # query rows, padded per head to a multiple of 128
     assert attn.attn_bwd_workspace_size(2, 16, 16, 8192, 8192, 128) == 256 + ((rows * 128 * 4 + rows * 8 + 255) // 256) * 256
     rows = 1 * 2 * 128  # Lq = 100 pads to 128
     assert attn.attn_bwd_workspace_size(1, 2, 1, 100, 300, 128) == 256 + ((rows * 128 * 4 + rows * 8 + 255) // 256) * 256
-    # d = 64: the d = 128 scratch plus zero-padded 128-column copies of Q, O, dO, dQ
-    # (query rows) and K, V, dK, dV (key rows), bf16
-    pad = 4 * (1 * 2 * 100 + 1 * 1 * 300) * 128 * 2
-    assert attn.attn_bwd_workspace_size(1, 2, 1, 100, 300, 64) == 256 + ((rows * 128 * 4 + rows * 8 + 255) // 256) * 256 + pad
+    rows = 1 * 2 * 256  # Lq = 200 pads to 256; d = 64 accumulates 64 columns
+    assert attn.attn_bwd_workspace_size(1, 2, 1, 200, 300, 64) == 256 + ((rows * 64 * 4 + rows * 8 + 255) // 256) * 256
 
 
 def test_status_strings(lib):

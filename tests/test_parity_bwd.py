@@ -76,8 +76,8 @@ D64_CASES = [
 
 @pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,causal,k_lens", D64_CASES)
 def test_bwd_d64_matches_oracle(B, Hq, Hkv, Lq, Lk, causal, k_lens):
-    """d = 64: the d = 128 kernels on zero-padded copies (the zero columns change
-    neither P nor dS); the gradients' first 64 columns against the oracle."""
+    """d = 64: the kernels' 64-column instantiation (S^T and dP^T over one
+    64-column panel, dV, dK and dQ at N = 64) against the oracle."""
     import torch
 
     attn = _lib()
