@@ -118,6 +118,19 @@ bool attn_bwd_impl::make_tmap_rows(CUtensorMap* m, const void* base, int d, int 
   return make_tmap(m, base, d, L, heads, box_rows);
 }
 
+bool attn_bwd_impl::make_tmap_acc64(CUtensorMap* m, float* base, int Lqp, long long heads) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(Lqp), static_cast<cuuint64_t>(heads)};
+  cuuint64_t strides[2] = {64 * 4, static_cast<cuuint64_t>(Lqp) * 64 * 4};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Shared launch of the forward kernel; p carries the layout-specific fields.
 static attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          attn_fwd_impl::Params p, attn_bf16_t* O, float* lse, int B, int Hq,

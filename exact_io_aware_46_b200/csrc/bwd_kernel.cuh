@@ -66,10 +66,12 @@ struct Cfg {
   static constexpr int OFF_DO = OFF_Q + NQS * TILE;  // [128 rows][d]
   static constexpr int OFF_DS = OFF_DO + TILE;    // dS^T [128 keys][128 rows]: panels of 64 rows
   // d = 128: dQ^T (lanes = d) is staged row-major DQ_ROWS query rows at a time
-  // for bulk reduce-adds; d = 64 adds dQ rows straight from registers
+  // for bulk reduce-adds; d = 64: the tile's dQ (lanes = query rows) is staged
+  // as two 128-byte-swizzled boxes of 32 columns for tensor reduce-adds
   static constexpr bool STAGED_DQ = DH == 128;
-  static constexpr int OFF_DQ = OFF_DS + 2 * PANEL;
-  static constexpr int OFF_LD = OFF_DQ + (STAGED_DQ ? DQ_ROWS * DH * 4 : 0);  // lse2 [128], D [128]
+  static constexpr int OFF_DQ = OFF_DS + 2 * PANEL;  // 1024-byte aligned
+  static constexpr int DQ_STAGE = STAGED_DQ ? DQ_ROWS * DH * 4 : BMQ * DH * 4;
+  static constexpr int OFF_LD = OFF_DQ + DQ_STAGE;  // lse2 [128], D [128]
   static constexpr int OFF_BAR = OFF_LD + NQS * 1024;
   static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
   static_assert(SMEM_BYTES <= 232448, "dynamic shared memory limit");
@@ -217,11 +219,17 @@ __device__ __forceinline__ void red_add_f32(float* acc, float a) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(acc), "f"(a) : "memory");
 }
 
-// acc[0..3] += (a, b, c, d): one 16-byte vector reduction, performed at L2.
-__device__ __forceinline__ void red_add_v4_f32(float* acc, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(acc), "f"(a), "f"(b), "f"(c),
-               "f"(d)
-               : "memory");
+
+// Tensor reduce-add of one shared-memory box into global memory through the
+// tensor map `m` at coordinates (c0, c1, c2); the TMA unit performs the
+// additions at L2.  Tracked by the calling thread's bulk async-group.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m, const void* ssrc, int c0,
+                                                  int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(m)),
+      "r"(sm100::smem_u32(ssrc)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
 }
 
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
@@ -306,7 +314,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmdO,
                     const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const Params p) {
+                    const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmAcc, const Params p) {
   using C = Cfg<DH>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = sm100::smem_u32(smem_raw);
@@ -366,6 +375,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     sm100::prefetch_tmap(&tmdO);
     sm100::prefetch_tmap(&tmK);
     sm100::prefetch_tmap(&tmV);
+    if constexpr (!C::STAGED_DQ) sm100::prefetch_tmap(&tmAcc);
   }
   if (warp == W_MMA) {
     sm100::tmem_alloc(tmem_slot, 512);
@@ -762,8 +772,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // rounds staged 1.457-1.486 ms; the first round by reductions 1.342-1.379
     // ms (shipped); the last one instead 1.420-1.442 ms; the first two
     // 1.402 ms; the last three 1.650 ms.
-    // d = 64: dQ (lanes = the tile's rows) goes to registers one row per thread
-    // and is added with 16-byte vector reductions straight from registers.
+    // d = 64: dQ (lanes = the tile's rows) goes to registers one row per thread;
+    // the rows are staged as two boxes of 128 rows x 32 columns in the 128-byte
+    // swizzle of the accumulator's tensor map (a thread's 16-byte chunk c of row
+    // r lands at chunk c ^ (r & 7) of the row's 128-byte line, so the eight
+    // threads of a quarter-warp hit distinct banks) and added with two tensor
+    // reduce-adds.
     const int tid = threadIdx.x - 32 * W_DRAIN;  // = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     float* stage = reinterpret_cast<float*>(smem + C::OFF_DQ);
@@ -827,18 +841,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           sm100::tc_fence_before();
           __syncwarp();
           if (sm100::lane_id() == 0) sm100::mbar_arrive(dq_empty);
-          float* acc_row = acc_rows + tid * DH;
+          // the previous tile's reduces must have finished reading the staging boxes
+          if (tid == 0) bulk_wait_read_all();
+          sm100::named_bar_sync(1, 128);
+          uint8_t* line = smem + C::OFF_DQ + tid * 128;
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            red_add_v4_f32(acc_row + 4 * j, __uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                           __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(line + h * (BMQ * 128) + ((c ^ (tid & 7)) << 4)) =
+                  make_uint4(v[32 * h + 4 * c], v[32 * h + 4 * c + 1], v[32 * h + 4 * c + 2],
+                             v[32 * h + 4 * c + 3]);
+          sm100::fence_proxy_async_smem();
+          sm100::named_bar_sync(1, 128);
+          if (tid == 0) {
+            tma_reduce_add_3d(&tmAcc, smem + C::OFF_DQ, 0, i * BMQ, qh);
+            tma_reduce_add_3d(&tmAcc, smem + C::OFF_DQ + BMQ * 128, 32, i * BMQ, qh);
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          }
         }
       }
       tq += it.T;
     }
     // the convert pass reads the accumulator after this kernel; the bulk
     // reduces must be complete before the CTA exits
-    if (C::STAGED_DQ && tid == 0) bulk_wait_all();
+    if (tid == 0) bulk_wait_all();
   }
 
   sm100::tc_fence_before();
@@ -862,6 +889,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 bool make_tmap_rows(CUtensorMap* m, const void* base, int d, int L, long long heads,
                     int box_rows);
+// fp32 view [heads][Lqp][64] of the d = 64 dQ accumulator, boxes of 32 columns x
+// 128 rows x 1 head, 128-byte swizzle (the staging layout of the drain)
+bool make_tmap_acc64(CUtensorMap* m, float* base, int Lqp, long long heads);
 
 template <int DH>
 attn_status_t launch_d(const Args& a, cudaStream_t s) {
@@ -904,10 +934,11 @@ attn_status_t launch_d(const Args& a, cudaStream_t s) {
   }
   // 2. main
   if (p.n_items > 0) {
-    CUtensorMap tq, tdo, tk, tv;
+    CUtensorMap tq, tdo, tk, tv, tacc;
     if (!make_tmap_rows(&tq, a.Q, DH, a.Lq, BH, BMQ) || !make_tmap_rows(&tdo, a.dO, DH, a.Lq, BH, BMQ) ||
         !make_tmap_rows(&tk, a.K, DH, a.Lk, static_cast<long long>(a.B) * a.Hkv, BN) ||
-        !make_tmap_rows(&tv, a.V, DH, a.Lk, static_cast<long long>(a.B) * a.Hkv, BN)) {
+        !make_tmap_rows(&tv, a.V, DH, a.Lk, static_cast<long long>(a.B) * a.Hkv, BN) ||
+        !(C::STAGED_DQ ? (tacc = tq, true) : make_tmap_acc64(&tacc, p.dq_acc, p.Lqp, BH))) {
       attn_host::report(cudaErrorInvalidValue, "bwd tensor maps");
       return ATTN_ERR_CUDA;
     }
@@ -915,7 +946,7 @@ attn_status_t launch_d(const Args& a, cudaStream_t s) {
                           "bwd_main_kernel shared-memory attribute") != cudaSuccess)
       return ATTN_ERR_CUDA;
     const int grid = p.n_items < a.sms ? p.n_items : a.sms;
-    bwd_main_kernel<DH><<<grid, NTHREADS, C::SMEM_BYTES, s>>>(tq, tdo, tk, tv, p);
+    bwd_main_kernel<DH><<<grid, NTHREADS, C::SMEM_BYTES, s>>>(tq, tdo, tk, tv, tacc, p);
     if (attn_host::report_launch(bwd_main_kernel<DH>, "bwd_main_kernel") != cudaSuccess)
       return ATTN_ERR_CUDA;
   }
