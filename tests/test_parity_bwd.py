@@ -127,3 +127,35 @@ def test_bwd_full_size_sampled():
         _check(to_f64(dq[b, h, rows]), rQ[0], f"dQ[{b},{h}]")
         _check(to_f64(dk[b, h, cols]), rK, f"dK[{b},{h}]")
         _check(to_f64(dv[b, h, cols]), rV, f"dV[{b},{h}]")
+
+
+def test_bwd_d64_full_size_sampled():
+    """B=4, H=16, L=4096, d=64, causal (the d = 64 backward as timed): sampled
+    rows of dQ and keys of dK, dV of the first and the last head, so the dQ
+    accumulator's tensor-map coordinates (query tile, head) reach their ends."""
+    import torch
+
+    attn = _lib()
+    B, H, L, d = 4, 16, 4096, 64
+    seed = 4664
+    shp = (B, H, L, d)
+    q = synth.normal_bf16_device(seed * 16 + 1, shp, "cuda")
+    k = synth.normal_bf16_device(seed * 16 + 2, shp, "cuda")
+    v = synth.normal_bf16_device(seed * 16 + 3, shp, "cuda")
+    do = synth.normal_bf16_device(seed * 16 + 4, shp, "cuda")
+    O, Lse = attn.attn_fwd(q, k, v, causal=True)
+    dq, dk, dv = attn.attn_bwd(q, k, v, O, do, Lse, causal=True)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, 2047, L - 129, L - 1],
+                                     rng.choice(L, 40, replace=False)])).astype(np.int32)
+    cols = np.unique(np.concatenate([[0, 127, 128, L - 128, L - 1],
+                                     rng.choice(L, 40, replace=False)])).astype(np.int32)
+    for b, h in ((0, 0), (3, 15)):
+        sl = lambda t: bits(t[b:b + 1, h:h + 1])
+        Qh, Kh, Vh, dOh = sl(q), sl(k), sl(v), sl(do)
+        rQ, rK, rV = oracle.bwd_sampled(Qh, Kh, Vh, dOh, 1 / math.sqrt(d), True, None, 0, 0,
+                                        rows, cols)
+        _check(to_f64(dq[b, h, rows]), rQ[0], f"dQ[{b},{h}]")
+        _check(to_f64(dk[b, h, cols]), rK, f"dK[{b},{h}]")
+        _check(to_f64(dv[b, h, cols]), rV, f"dV[{b},{h}]")
