@@ -301,8 +301,8 @@ attn_status_t attn_bwd(const attn_bf16_t* Q, const attn_bf16_t* K, const attn_bf
  * partials need more (256 + B*Hq*ceil(Lmax/2048)*(4*d + 4) bytes, rounded up to
  * 256) returns ATTN_ERR_CAPACITY before anything is launched.  The first call
  * on a device looks up the array's device address (cudaGetSymbolAddress, with
- * that device current) and raises the kernels' shared-memory limit; make that
- * first call before any stream capture.  The set-up is repeated when the
+ * that device current) and raises the kernels' shared-memory limit; later
+ * calls make neither API call.  The set-up is repeated when the
  * device's CUDA context changes (after cudaDeviceReset, the next call is a
  * first call again).  The call allocates and frees nothing.
  *
