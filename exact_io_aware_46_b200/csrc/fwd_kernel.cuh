@@ -345,7 +345,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == W_LOAD) {
     // ------------------------------------------------------------ scheduler + TMA producer
     if (sm100::lane_id() == 0) {
-      uint32_t use = 0;
+      uint32_t use = 0;     // K/V tile copies issued
+      int q_issued = 0;     // Q copies issued (one per item)
       for (uint32_t k = 0;; ++k) {
         if (!sm100::mbar_wait(&item_empty[k % NI], ((k / NI) & 1) ^ 1, abort_flag, p.status))
           break;
@@ -358,6 +359,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const Item it = get_item<D, MODE>(p, w, nullptr);
         if (!sm100::mbar_wait(q_empty, (k & 1) ^ 1, abort_flag, p.status)) break;
         sm100::mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
+        ++q_issued;
         const int qh = it.q_head;
         for (int t = 0; t < 2; ++t)
           for (int c = 0; c < C::CHUNKS; ++c)
@@ -382,6 +384,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
         if (!ok) break;
+      }
+      // the CTA must not exit while tensor copies still land in its shared
+      // memory, which an expired wait elsewhere could otherwise allow: wait
+      // (bounded, ignoring the abort flag) for the last issued phase of every
+      // load barrier; in normal operation the consumers already waited for them
+      if (q_issued > 0) sm100::mbar_wait_drain(q_full, (q_issued - 1) & 1);
+      for (uint32_t sl = 0; sl < C::NS && sl < use; ++sl) {
+        const uint32_t last = sl + C::NS * ((use - 1 - sl) / C::NS);
+        sm100::mbar_wait_drain(&kv_full[sl], (last / C::NS) & 1);
       }
     }
   } else if (warp == W_MMA) {
