@@ -4,10 +4,13 @@
 // long context: three ledgers" (prefill vs decode): per step the whole cache
 // row range [0, k_len) is read once and the arithmetic per byte is tiny
 // (4 FLOP/B with 4 query heads per key/value head), so the kernel is bound by
-// HBM bandwidth, not by the tensor core.  It therefore runs on CUDA cores:
+// HBM bandwidth.  Two split kernels compute the same partials:
 //
-//  * split kernel: one CTA per (sequence, key/value head, chunk of CH keys),
-//    three CTAs per SM.
+//  * tensor-core split kernel (contiguous cache, d = 128; further below): the
+//    scores and the PV product as small tcgen05 MMAs (16 heads padded), so the
+//    CUDA cores only form the exponentials and the kernel streams the cache;
+//  * CUDA-core split kernel (paged caches and d = 64): one CTA per (sequence,
+//    key/value head, chunk of CH keys), three CTAs per SM.
 //    A producer thread streams the chunk's K and V rows (contiguous in the
 //    cache) with 1-D bulk copies into a ring of shared-memory stages; four
 //    compute warps each own 16 rows of every stage.  A half-warp covers one
@@ -25,6 +28,13 @@
 
 #include "launch_cache.cuh"
 #include "sm100.cuh"
+
+namespace attn_bwd_impl {
+// 3-D bf16 tensor map [heads][rows][d], boxes of 64 columns x box_rows rows,
+// 128-byte swizzle (defined with the C entry points)
+bool make_tmap_rows(CUtensorMap* m, const void* base, int d, int L, long long heads,
+                    int box_rows);
+}
 
 namespace attn_decode_impl {
 
@@ -456,6 +466,317 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) decode_split_kernel(con
   }
 }
 
+// ---------------------------------------------------------------- tensor-core split kernel
+//
+// The same split (one CTA per chunk of CH keys of one sequence and kv head)
+// with the two products on the tensor core instead of the CUDA cores, for a
+// contiguous cache at d = 128: per block of 128 keys,
+//     S^T = K Q^T     (M = 128 keys on the TMEM lanes, N = 16 query heads
+//                      padded, K = d; both operands K-major in shared memory)
+//     O^T += V^T P^T  (M = d = 128 lanes, N = 16 heads, K = 128 keys; V^T is
+//                      the V tile read MN-major, P is written by the softmax
+//                      threads as a 16-row K-major tile)
+// so the CUDA cores only form the scores' exponentials (G per key) and the
+// kernel streams the cache (measured on B200, B64 Hq32 Hkv8 d128, cache
+// 32768, k_len ~ U[1024, 32768]: 6902 against 6400 GB/s for the CUDA-core
+// kernel in the same process).  Warp 0 loads K and V blocks with TMA (128-byte
+// swizzle) into a ring of three 32 KB slots, warp 1 issues the MMAs, warps
+// 2-5 (one key row, then one d index, per thread) run the online softmax of
+// the three-ledgers page per block with the stale-max threshold and write the
+// chunk's normalised partial.  The block chain (S, softmax, PV) is serial;
+// with two CTAs per SM and the next block's K and V in flight during it, the
+// copies are the limit.
+namespace tc {
+
+constexpr int BK = 128;        // keys per block
+constexpr int NH = 16;         // query heads per group, padded (the MMA's N)
+constexpr int NSLOT = 3;       // ring slots (one K or V block of 32 KB each)
+constexpr int SLOT = BK * 128 * 2;  // 32 KB: two 128-row x 64-column panels
+constexpr int PANEL = BK * 128;     // 16 KB
+constexpr int HPANEL = NH * 128;    // 2 KB: a 16-row x 64-column panel
+constexpr int OFF_RING = 0;
+constexpr int OFF_Q = NSLOT * SLOT;            // Q tile, 2 panels
+constexpr int OFF_P = OFF_Q + 2 * HPANEL;      // P tile, 2 panels
+constexpr int OFF_RED = OFF_P + 2 * HPANEL;    // [2][4 warps][NH] block maxima, [4][NH] sums
+constexpr int OFF_BAR = OFF_RED + 3 * 4 * NH * 4;
+constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
+constexpr int NTHREADS = 6 * 32;
+constexpr uint32_t IDESC_S = sm100::idesc_bf16_f32(128, NH, false, false);
+constexpr uint32_t IDESC_PV = sm100::idesc_bf16_f32(128, NH, true, false);
+constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 2)
+    split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const SplitParams p) {
+  static_assert(D == 128, "one 128-lane d tile");
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = sm100::smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+  const uint32_t sbase = sm100::smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* kv_full = bars;              // [NSLOT]
+  uint64_t* kv_empty = bars + NSLOT;     // [NSLOT]
+  uint64_t* s_full = bars + 2 * NSLOT;
+  uint64_t* p_full = s_full + 1;
+  uint64_t* o_full = s_full + 2;
+  uint64_t* q_ready = s_full + 3;
+  uint64_t* drain = s_full + 4;
+  uint64_t* mx_bar = s_full + 5;   // [2]: the softmax warps' block maxima are in
+  uint64_t* sum_bar = s_full + 7;  // the softmax warps' row sums are in
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* red = reinterpret_cast<float*>(smem + OFF_RED);
+
+  // the same chunk order as the CUDA-core kernel (from_end layout)
+  const int hkv = blockIdx.x % p.Hkv, b = blockIdx.x / p.Hkv;
+  const int kl = valid_klen(p.k_lens, b, p.Lmax, p.status,
+                            blockIdx.y == gridDim.y - 1 && hkv == 0 && threadIdx.x == 0);
+  const int chunk = (kl + CH - 1) / CH - static_cast<int>(gridDim.y - blockIdx.y);
+  if (chunk < 0) return;
+  const int k0 = chunk * CH;
+  const int rows = min(CH, kl - k0);
+  const int nblk = (rows + BK - 1) / BK;
+  const int warp = threadIdx.x >> 5;
+  const int head_kv = b * p.Hkv + hkv;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NSLOT; ++i) {
+      sm100::mbar_init(&kv_full[i], 1);
+      sm100::mbar_init(&kv_empty[i], 1);
+    }
+    sm100::mbar_init(s_full, 1);
+    sm100::mbar_init(p_full, 4);
+    sm100::mbar_init(o_full, 1);
+    sm100::mbar_init(q_ready, 4);
+    sm100::mbar_init(drain, 1);
+    sm100::mbar_init(&mx_bar[0], 4);
+    sm100::mbar_init(&mx_bar[1], 4);
+    sm100::mbar_init(sum_bar, 4);
+    *abort_flag = 0;
+    sm100::fence_barrier_init();
+  }
+  if (warp == 0 && sm100::lane_id() == 0) {
+    sm100::prefetch_tmap(&tmK);
+    sm100::prefetch_tmap(&tmV);
+  }
+  if (warp == 1) {
+    sm100::tmem_alloc(tmem_slot, 32);
+    sm100::tmem_relinquish();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tO = tmem + NH;  // S^T: columns 0-15, O^T: 16-31
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (sm100::lane_id() == 0) {
+      int issued = 0;
+      for (int u = 0; u < 2 * nblk; ++u) {
+        const int slot = u % NSLOT;
+        if (!sm100::mbar_wait(&kv_empty[slot], ((u / NSLOT) & 1) ^ 1, abort_flag, p.status, 21))
+          break;
+        sm100::mbar_arrive_expect_tx(&kv_full[slot], SLOT);
+        ++issued;
+        const int row = k0 + (u >> 1) * BK;
+        for (int c = 0; c < 2; ++c)
+          sm100::tma_load_3d((u & 1) ? &tmV : &tmK, &kv_full[slot],
+                             smem + OFF_RING + slot * SLOT + c * PANEL, c * 64, row, head_kv);
+      }
+      // the CTA must not exit while copies still land in its shared memory
+      for (int u = issued - 1; u >= 0 && u >= issued - NSLOT; --u)
+        sm100::mbar_wait_drain(&kv_full[u % NSLOT], (u / NSLOT) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    const bool leader = sm100::elect_one();
+    auto commit = [&](uint64_t* bar) {
+      if (leader) sm100::tc_commit(bar);
+      __syncwarp();
+    };
+    const uint64_t qd = sm100::sdesc_sw128(sbase + OFF_Q, 16, 1024);
+    const uint64_t pd = sm100::sdesc_sw128(sbase + OFF_P, 16, 1024);
+    bool ok = sm100::mbar_wait(q_ready, 0, abort_flag, p.status, 22);
+    for (int j = 0; j < nblk && ok; ++j) {
+      const int uk = 2 * j, uv = 2 * j + 1;
+      const int ks = uk % NSLOT, vs = uv % NSLOT;
+      if (!(ok = sm100::mbar_wait(&kv_full[ks], (uk / NSLOT) & 1, abort_flag, p.status, 23))) break;
+      sm100::tc_fence_after();
+      if (leader) {
+        // S^T = K Q^T: both K-major; K steps of 16 d (32 bytes) inside a panel
+        const uint64_t kd = sm100::sdesc_sw128(sbase + OFF_RING + ks * SLOT, 16, 1024);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          sm100::mma_ss(tS, kd + static_cast<uint64_t>(((k >> 2) * PANEL + (k & 3) * 32) >> 4),
+                        qd + static_cast<uint64_t>(((k >> 2) * HPANEL + (k & 3) * 32) >> 4),
+                        IDESC_S, k > 0 ? 1u : 0u);
+      }
+      commit(s_full);
+      commit(&kv_empty[ks]);
+      if (!(ok = sm100::mbar_wait(p_full, j & 1, abort_flag, p.status, 24))) break;
+      if (!(ok = sm100::mbar_wait(&kv_full[vs], (uv / NSLOT) & 1, abort_flag, p.status, 25))) break;
+      sm100::tc_fence_after();
+      if (leader) {
+        // O^T += V^T P^T: A = the V tile read MN-major (64-wide d panels 16 KB
+        // apart, 8-key groups 1 KB apart), B = P K-major; K steps of 16 keys
+        const uint64_t vd = sm100::sdesc_sw128(sbase + OFF_RING + vs * SLOT, PANEL, 1024);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k)
+          sm100::mma_ss(tO, vd + static_cast<uint64_t>((k * 2048) >> 4),
+                        pd + static_cast<uint64_t>(((k >> 2) * HPANEL + (k & 3) * 32) >> 4),
+                        IDESC_PV, (j > 0 || k > 0) ? 1u : 0u);
+      }
+      commit(&kv_empty[vs]);
+    }
+    commit(o_full);
+    // every issued MMA must complete before the tensor memory is released
+    commit(drain);
+    sm100::mbar_wait_drain(drain, 0);
+  } else {
+    // ------------------------------------------------------------ softmax (warps 2-5)
+    const int t = threadIdx.x - 64;              // 0..127
+    const int q = warp & 3;                      // TMEM lane quarter of this warp
+    const int r = q * 32 + sm100::lane_id();     // TMEM lane: key row of the block, then d
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const int G = p.G;
+    // Q tile (16 rows, heads >= G zero) and the constant zero rows of P
+    for (int e = t; e < NH * 16; e += 128) {
+      const int g = e >> 4, c16 = e & 15;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (g < G)
+        v = __ldg(reinterpret_cast<const uint4*>(
+                      p.Q + (static_cast<size_t>(b) * p.Hq + hkv * G + g) * D) + c16);
+      *reinterpret_cast<uint4*>(smem + OFF_Q + (c16 >> 3) * HPANEL + g * 128 +
+                                (((c16 & 7) ^ (g & 7)) << 4)) = v;
+      if (g >= G)
+        *reinterpret_cast<uint4*>(smem + OFF_P + (c16 >> 3) * HPANEL + g * 128 + ((c16 & 7) << 4)) =
+            make_uint4(0u, 0u, 0u, 0u);
+    }
+    sm100::fence_proxy_async_smem();
+    __syncwarp();
+    if (sm100::lane_id() == 0) sm100::mbar_arrive(q_ready);
+
+    float m_use[NH], l[NH];
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      m_use[h] = -INFINITY;
+      l[h] = 0.f;
+    }
+    // this thread's P entries: row h, key r -> panel r / 64, 16-byte chunk
+    // (r % 64) / 8 swizzled by the row, element r % 8
+    uint8_t* p_col = smem + OFF_P + (r >> 6) * HPANEL + ((r & 7) << 1);
+    const int p_chunk = (r & 63) >> 3;
+    bool ok = true;
+    for (int j = 0; j < nblk && ok; ++j) {
+      if (!(ok = sm100::mbar_wait(s_full, j & 1, abort_flag, p.status, 26))) break;
+      sm100::tc_fence_after();
+      uint32_t s[NH];
+      sm100::tmem_ld16(tS + lane_base, s);
+      sm100::tmem_ld_wait();
+      const bool valid = j * BK + r < rows;
+      float v[NH];
+#pragma unroll
+      for (int h = 0; h < NH; ++h)
+        v[h] = (valid && h < G) ? __uint_as_float(s[h]) * p.scale_log2 : -INFINITY;
+      // block maxima per head: within the warp, then across the four warps
+      // (through shared memory and an mbarrier, so that every wait is bounded;
+      // two buffers: a warp writes block j + 2's maxima only after all four
+      // warps arrived for block j + 1, i.e. after they read block j's)
+      float* rw = red + (j & 1) * 4 * NH;
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        float m = v[h];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (sm100::lane_id() == h) rw[q * NH + h] = m;
+      }
+      __syncwarp();
+      if (sm100::lane_id() == 0) sm100::mbar_arrive(&mx_bar[j & 1]);
+      if (!(ok = sm100::mbar_wait(&mx_bar[j & 1], (j >> 1) & 1, abort_flag, p.status, 28))) break;
+      bool need = false;
+      float mb[NH];
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        mb[h] = fmaxf(fmaxf(rw[h], rw[NH + h]), fmaxf(rw[2 * NH + h], rw[3 * NH + h]));
+        need |= mb[h] > m_use[h] + RESCALE_THRESHOLD;
+      }
+      if (need) {  // uniform: every thread saw the same maxima
+        float alpha[NH];
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          const float mn = fmaxf(m_use[h], mb[h]);
+          alpha[h] = (m_use[h] == -INFINITY) ? 0.f : sm100::ex2(m_use[h] - mn);
+          m_use[h] = mn;
+          l[h] *= alpha[h];
+        }
+        if (j > 0) {
+          // O^T holds PV of the previous blocks (complete: this block's S^T was
+          // issued after them); rescale this thread's row (one d index)
+          uint32_t o[NH];
+          sm100::tmem_ld16(tO + lane_base, o);
+          sm100::tmem_ld_wait();
+#pragma unroll
+          for (int h = 0; h < NH; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+          sm100::tmem_st16(tO + lane_base, o);
+          sm100::tmem_st_wait();
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        if (h < G) {
+          const float pv = (v[h] == -INFINITY) ? 0.f : sm100::ex2(v[h] - m_use[h]);
+          l[h] += pv;
+          *reinterpret_cast<__nv_bfloat16*>(p_col + h * 128 + ((p_chunk ^ (h & 7)) << 4)) =
+              __float2bfloat16_rn(pv);
+        }
+      }
+      sm100::fence_proxy_async_smem();
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (sm100::lane_id() == 0) sm100::mbar_arrive(p_full);
+    }
+    // ---- partial of the chunk: l over the 128 key rows, O^T row d = r
+    if (ok) ok = sm100::mbar_wait(o_full, 0, abort_flag, p.status, 27);
+    float* rs = red + 2 * 4 * NH;
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      float x = l[h];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+      if (sm100::lane_id() == h) rs[q * NH + h] = x;
+    }
+    __syncwarp();
+    if (sm100::lane_id() == 0) sm100::mbar_arrive(sum_bar);
+    if (ok) ok = sm100::mbar_wait(sum_bar, 0, abort_flag, p.status, 29);
+    uint32_t o[NH];
+    if (ok && !*abort_flag) {
+      sm100::tc_fence_after();
+      sm100::tmem_ld16(tO + lane_base, o);
+      sm100::tmem_ld_wait();
+    }
+    const bool live = ok && !*abort_flag;
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      if (h >= G) break;
+      const float ls = rs[h] + rs[NH + h] + rs[2 * NH + h] + rs[3 * NH + h];
+      const size_t ph = (static_cast<size_t>(b) * p.Hq + hkv * G + h) * p.nsm + chunk;
+      const bool has = live && ls > 0.f;
+      p.part_o[ph * D + r] = has ? __uint_as_float(o[h]) / ls : 0.f;
+      if (r == 0) p.part_lse[ph] = has ? m_use[h] + log2f(ls) : -INFINITY;
+    }
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc(tmem, 32);
+  }
+}
+
+}  // namespace tc
+
 struct CombineParams {
   const float* part_o;
   const float* part_lse;
@@ -507,6 +828,27 @@ cudaError_t launch_t(const SplitParams& sp, const CombineParams& cp, cudaStream_
   return attn_host::report_launch(decode_combine_kernel<D>, "decode_combine_kernel");
 }
 
+// The tensor-core split kernel (contiguous cache, d = 128) and the combine.
+inline cudaError_t launch_tc(const SplitParams& sp, const CombineParams& cp, cudaStream_t s) {
+  CUtensorMap tk, tv;
+  const long long heads = static_cast<long long>(sp.B) * sp.Hkv;
+  if (!attn_bwd_impl::make_tmap_rows(&tk, sp.K, 128, sp.Lmax, heads, tc::BK) ||
+      !attn_bwd_impl::make_tmap_rows(&tv, sp.V, 128, sp.Lmax, heads, tc::BK))
+    return attn_host::report(cudaErrorInvalidValue, "decode tensor maps");
+  cudaError_t e = attn_host::report(attn_host::set_smem(tc::split_kernel<128>, tc::SMEM_BYTES),
+                                    "decode tensor-core kernel shared-memory attribute");
+  if (e != cudaSuccess) return e;
+  SplitParams spl = sp;
+  spl.from_end = 1;
+  tc::split_kernel<128><<<dim3(static_cast<unsigned>(sp.Hkv * sp.B), sp.nsm, 1), tc::NTHREADS,
+                     tc::SMEM_BYTES, s>>>(tk, tv, spl);
+  if ((e = attn_host::report_launch(tc::split_kernel<128>, "decode tensor-core split kernel")) !=
+      cudaSuccess)
+    return e;
+  decode_combine_kernel<128><<<sp.B * sp.Hq, 128, 0, s>>>(cp);
+  return attn_host::report_launch(decode_combine_kernel<128>, "decode_combine_kernel");
+}
+
 // Paged cache description for launch(); Lmax is then max_blocks * page.
 struct PagedKV {
   const int* block_table;  // device [B][max_blocks]
@@ -548,6 +890,10 @@ inline cudaError_t launch(const __nv_bfloat16* Q, const __nv_bfloat16* K, const 
   cp.Lmax = Lmax;
   cp.nsm = sp.nsm;
   const bool wide = sp.G > 4;
+  // contiguous cache at d = 128: the tensor-core kernel
+  if (d == 128 && !paged && sp.nsm <= 65535 &&
+      static_cast<long long>(Hkv) * B <= 0x7fffffffLL)
+    return launch_tc(sp, cp, s);
   if (d == 128) return wide ? launch_t<128, 8>(sp, cp, s) : launch_t<128, 4>(sp, cp, s);
   return wide ? launch_t<64, 8>(sp, cp, s) : launch_t<64, 4>(sp, cp, s);
 }
