@@ -1003,8 +1003,8 @@ def main():
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "frac_of_8TBs": gbs / 8000.0,
                          "traffic": traffic_per_launch(
-                             "attn_decode_impl::decode_split_kernel<128,4>", kv_bytes),
-                         "kernel": "attn_decode_impl::decode_split_kernel<128,4> + combine"},
+                             "attn_decode_impl::tc::split_kernel<128>", kv_bytes),
+                         "kernel": "attn_decode_impl::tc::split_kernel<128> + combine"},
             "gpu_launches": 4 * args.steps,
         }
         t_p = max_over_ranks(float(np.mean(pms)), world)
