@@ -118,6 +118,23 @@ bool attn_bwd_impl::make_tmap_rows(CUtensorMap* m, const void* base, int d, int 
   return make_tmap(m, base, d, L, heads, box_rows);
 }
 
+bool attn_decode_impl::make_tmap_paged(CUtensorMap* m, const void* base, int d, int page,
+                                       int Hkv, int n_pages, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(page),
+                        static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(n_pages)};
+  const cuuint64_t row = static_cast<cuuint64_t>(d) * 2;
+  cuuint64_t strides[3] = {row, row * static_cast<cuuint64_t>(page),
+                           row * static_cast<cuuint64_t>(page) * static_cast<cuuint64_t>(Hkv)};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool attn_bwd_impl::make_tmap_acc64(CUtensorMap* m, float* base, int Lqp, long long heads) {
   auto fn = encode_fn();
   if (!fn) return false;
