@@ -37,6 +37,7 @@ CASES = [
     (2, 4, 2, 1300, 64, [1300, 65]),              # d = 64, G = 2
     (2, 8, 2, 1200, 128, [0, 1200]),              # an empty sequence
     (1, 4, 1, 70, 128, [70]),                     # shorter than one stage
+    (2, 4, 2, 2200, 128, [128, 2177]),            # G = 2; one whole 128-key block; a chunk of 129 keys
 ]
 
 

@@ -53,6 +53,7 @@ CASES = [
     (2, 4, 2, 1300, 64, [1300, 65], 32),           # d = 64
     (2, 8, 2, 1200, 128, [0, 1200], 128),          # an empty sequence
     (1, 4, 1, 5000, 128, [4097], 1024),            # three chunks inside large pages
+    (2, 4, 2, 2200, 128, [128, 2177], 32),         # G = 2; a chunk of 129 keys over 32-row pages
 ]
 
 
