@@ -543,13 +543,23 @@ def ring_leg(steps, warmup, world, flush):
             torch.empty((c["B"], c["Hq"], Lc, c["d"]), dtype=torch.bfloat16, device=dev))
            for _ in range(W)]
     plans = [ring_steps(r, W, True) for r in range(W)]
+    # the emulated ranks are independent: each rank's folds run in order on a
+    # stream of its own (its own scheduler workspace), the ranks side by side
+    rstreams = [torch.cuda.Stream() for _ in range(W)]
+    rws = [torch.zeros(256, dtype=torch.uint8, device=dev) for _ in range(W)]
 
     def step():
+        main = torch.cuda.current_stream()  # the capture stream while a graph records
         for r in range(W):
+            rstreams[r].wait_stream(main)
             last = max(s for s, _, kind in plans[r] if kind != "skip")
-            for s, src, kind in plans[r]:
-                fold_chunk(qs[r], ks[src], vs[src], kind, acc[r][0], acc[r][1], first=(s == 0),
-                           O_out=acc[r][2] if s == last else None, workspace=ws)
+            with torch.cuda.stream(rstreams[r]):
+                for s, src, kind in plans[r]:
+                    fold_chunk(qs[r], ks[src], vs[src], kind, acc[r][0], acc[r][1],
+                               first=(s == 0), O_out=acc[r][2] if s == last else None,
+                               workspace=rws[r])
+        for r in range(W):
+            main.wait_stream(rstreams[r])
 
     # one emulated step is ten launches with Python between them: capture it in a
     # CUDA graph so that the timed region holds the kernels back to back (first
@@ -567,9 +577,10 @@ def ring_leg(steps, warmup, world, flush):
         torch.cuda.synchronize()
     barrier(world)
     ms = timed_loop(run, steps, warmup, torch.cuda.current_stream(), flush)
-    st = attn.attn_read_device_status(ws)
-    if st[0] != attn.ATTN_OK:
-        raise RuntimeError(f"device status {st}")
+    for w_ in rws:
+        st = attn.attn_read_device_status(w_)
+        if st[0] != attn.ATTN_OK:
+            raise RuntimeError(f"device status {st}")
     flops = 4.0 * c["d"] * causal_pairs(c["L"], c["L"], True) * c["Hq"] * c["B"]
     n_fold = sum(1 for p in plans for _, _, kind in p if kind != "skip")
 
@@ -600,12 +611,22 @@ def ring_leg(steps, warmup, world, flush):
     zplans = [zigzag_folds(r, W) for r in range(W)]
 
     def zigzag_rank(r):
+        # as ring_attn_fwd_zigzag runs them: per step, the folds into the early
+        # chunk's accumulator on the main stream and into the late chunk's on a
+        # side stream, joined before the next step's chunk would be swapped in
         mine = zigzag_chunks(r, W)
-        for _, src, qi, ki, kind, first, last in zplans[r]:
-            ch = zigzag_chunks(src, W)[ki]
-            a = zacc[r][qi]
-            fold_chunk(zq[mine[qi]], zk[ch], zv[ch], kind, a[0], a[1], first=first,
-                       O_out=a[2] if last else None, workspace=ws)
+        main = torch.cuda.current_stream()  # the capture stream while a graph records
+        for s in range(W):
+            rstreams[1].wait_stream(main)
+            for s_, src, qi, ki, kind, first, last in zplans[r]:
+                if s_ != s:
+                    continue
+                ch = zigzag_chunks(src, W)[ki]
+                a = zacc[r][qi]
+                with torch.cuda.stream(rstreams[1] if qi == 1 else main):
+                    fold_chunk(zq[mine[qi]], zk[ch], zv[ch], kind, a[0], a[1], first=first,
+                               O_out=a[2] if last else None, workspace=rws[qi])
+            main.wait_stream(rstreams[1])
 
     per_rank = {}
     graphs = []
@@ -618,9 +639,10 @@ def ring_leg(steps, warmup, world, flush):
                                               flush))))
         per_rank[name] = t
     n_zfold = sum(len(p) for p in zplans)
-    st = attn.attn_read_device_status(ws)
-    if st[0] != attn.ATTN_OK:
-        raise RuntimeError(f"device status {st}")
+    for w_ in [ws] + rws:
+        st = attn.attn_read_device_status(w_)
+        if st[0] != attn.ATTN_OK:
+            raise RuntimeError(f"device status {st}")
     del graphs, zq, zk, zv, zacc
     # the merge kernel alone: one chunk's rows folded into an accumulator
     Op = acc[0][2]
@@ -923,6 +945,7 @@ def main():
             rep["ring_TFLOPs"] = ring[1] / (float(np.mean(ring[0])) * 1e-3) / 1e12
             rep["merge_GBs"] = ring[4] / (float(np.mean(ring[3])) * 1e-3) / 1e9
             rep["ring_launch"] = ring[6]
+            rep["ring_per_rank_ms"] = ring[8][0]
         if rank == 0:
             print(json.dumps(rep), flush=True)
         return
@@ -1058,7 +1081,8 @@ def main():
         line["ring"] = {
             "workload": f"ring attention's decomposition of the causal B1 Hq32 Hkv8 L16384 d128 "
                         f"forward into {RING['world']} chunks, every rank's steps run on this "
-                        f"GPU (one attn_fwd_merge per visible chunk; no exchange: "
+                        f"GPU (one attn_fwd_merge per visible chunk, each rank's folds in "
+                        f"order on a stream of its own, the ranks side by side; no exchange: "
                         f"one GPU)",
             "value": world * rflops / (t_r * 1e-3) / 1e12, "unit": "TFLOP/s",
             "ms_per_step": t_r, "flops_per_step": rflops, "chunk_folds_per_step": n_fold,
@@ -1066,7 +1090,8 @@ def main():
             "per_rank": {
                 "what": "each rank's own folds timed alone on this GPU (CUDA graph): the "
                         "compute of one step of a 4-GPU ring, exchange aside; the slowest "
-                        "rank sets the step time",
+                        "rank sets the step time; zigzag: per step the folds into the two "
+                        "query chunks on two streams, as ring_attn_fwd_zigzag runs them",
                 "contiguous_ms": prank["contiguous"], "contiguous_max_ms": max(prank["contiguous"]),
                 "zigzag_ms": prank["zigzag"], "zigzag_max_ms": max(prank["zigzag"]),
                 "zigzag_TFLOPs_per_gpu_modelled": rflops / RING["world"]

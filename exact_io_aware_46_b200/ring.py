@@ -315,13 +315,24 @@ def ring_attn_fwd_zigzag(q, k, v, group=None, scale=None):
     lse_acc = [torch.empty(t.shape[:-1], dtype=torch.float32, device=t.device) for t in q]
     O = [torch.empty_like(t) for t in q]
     ex = RingExchange((k[0], k[1], v[0], v[1]), group)
+    # the folds into the two query chunks' accumulators are independent: the
+    # late chunk's run on a side stream (its own scheduler workspace), so one
+    # launch's last partial wave overlaps the other's; both join before the
+    # exchange reuses the chunk buffers
+    main = torch.cuda.current_stream(q[0].device)
+    side = torch.cuda.Stream(device=q[0].device)
+    ws = [torch.zeros(256, dtype=torch.uint8, device=q[0].device) for _ in range(2)]
     for s in range(world):
         if s + 1 < world:
             ex.start()
         k0, k1, v0, v1 = ex.cur
+        side.wait_stream(main)
         for _, _, qi, ki, kind, first, last in (f for f in folds if f[0] == s):
-            fold_chunk(q[qi], (k0, k1)[ki], (v0, v1)[ki], kind, O_acc[qi], lse_acc[qi],
-                       first=first, O_out=O[qi] if last else None, scale=scale)
+            with torch.cuda.stream(side if qi == 1 else main):
+                fold_chunk(q[qi], (k0, k1)[ki], (v0, v1)[ki], kind, O_acc[qi], lse_acc[qi],
+                           first=first, O_out=O[qi] if last else None, scale=scale,
+                           workspace=ws[qi])
+        main.wait_stream(side)
         if s + 1 < world:
             ex.finish()
     return tuple(O), tuple(lse_acc)
