@@ -23,7 +23,7 @@
 //    per half of the key columns, and agree on the row max through shared
 //    memory; two warps per scheduler and tile hide the latency of the
 //    exponential chains that a single warp left exposed.
-//  * a quarter of the exponentials (an eighth with 8-bit inputs) run on the
+//  * a quarter of the exponentials (an eighth with 8-bit inputs or d = 64) run on the
 //    FMA pipe (polynomial exp2), the rest on the special-function unit;
 //  * the running max is kept in the log2 domain and is only moved when a row's
 //    new max exceeds it by more than 8 (a factor 256): o and l only need a
@@ -223,17 +223,19 @@ __device__ __forceinline__ Item get_item(const Params& p, int w, bool* bad) {
 }
 
 // Polynomial (FMA-pipe) instead of MUFU exp2 for column pairs whose index
-// cp = c / 2 satisfies cp % 8 >= 6 (bf16: a quarter of the exponentials) or
-// cp % 8 == 7 (8-bit inputs: an eighth).  The softmax warps are issue-bound as
+// cp = c / 2 satisfies cp % 8 >= 6 (bf16 at d = 128: a quarter of the
+// exponentials) or cp % 8 == 7 (8-bit inputs, and d = 64: an eighth; at d = 64,
+// causal B4 H16 L4096, an eighth 0.2007-0.2016 ms, a quarter 0.2038, three
+// eighths 0.2140, a half 0.2304).  The softmax warps are issue-bound as
 // much as MUFU-bound, so the best share is small.  Measured on B200 (causal
 // B4 H16 L4096 d128): with one softmax warp per row 0 % 0.313 ms, 12.5 % 0.310
 // ms, 25 % 0.325 ms, 50 % 0.349 ms; with two warps per row (this kernel)
 // 12.5 % 0.2519-0.2540 ms, 25 % 0.2499-0.2509 ms, 37.5 % 0.2601-0.2621 ms;
 // the 8-bit kernel, whose XU pipe also carries the E4M3 conversions, 12.5 %
 // 0.2263 ms and 25 % 0.2304 ms.
-template <int EB>
+template <int D, int EB>
 __device__ __forceinline__ constexpr bool poly_pair(int cp) {
-  return EB == 2 ? (cp & 7) >= 6 : (cp & 7) == 7;
+  return (EB == 2 && D == 128) ? (cp & 7) >= 6 : (cp & 7) == 7;
 }
 
 // S_t = Q_t K_j^T: 128 x 128 (keys) x D, both operands K-major SW128 panels.
@@ -689,7 +691,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               make_float2(__uint_as_float(s[2 * cp]), __uint_as_float(s[2 * cp + 1])), sl2x2,
               negm);
           float2 e;
-          if (poly_pair<EB>(cp)) {
+          if (poly_pair<D, EB>(cp)) {
             e = sm100::ex2_poly2(x);
           } else {
             e.x = sm100::ex2(x.x);
