@@ -328,8 +328,23 @@ def fwd_leg(steps, warmup, world, flush):
         raise RuntimeError(f"device status {st}")
     del q8, k8, v8, qs, ks, vs, O, lse
     torch.cuda.empty_cache()
+    # the same shape at d = 64
+    shp64 = (c["B"], c["Hq"], c["L"], 64)
+    q6, k6, v6 = (synth.normal_bf16_device(synth.workload_seed(2, t) ^ 64, shp64, dev)
+                  for t in ("q", "k", "v"))
+    O6 = torch.empty_like(q6)
+    lse6 = torch.empty((c["B"], c["Hq"], c["L"]), dtype=torch.float32, device=dev)
+    call_6 = lambda: attn.attn_fwd(q6, k6, v6, causal=True, O=O6, lse=lse6, workspace=ws,
+                                   stream=stream)
+    barrier(world)
+    ms64 = timed_loop(call_6, steps, warmup, stream, flush)
+    st = attn.attn_read_device_status(ws)
+    if st[0] != attn.ATTN_OK:
+        raise RuntimeError(f"device status {st}")
+    del q6, k6, v6, O6, lse6
+    torch.cuda.empty_cache()
     return (ms, ms_e2e, h2d, d2h, varlen_leg(steps, warmup, world, flush), (W, wms, wflops),
-            fms)
+            fms, ms64)
 
 
 WINDOW = 1024
@@ -915,7 +930,7 @@ def main():
     with Clocks(gpu_idx) as clk:
         if "fwd" in legs:
             (ms, ms_e2e, h2d, d2h, (vms, vflops, vtotal),
-             (W, wms, wflops), fms) = fwd_leg(args.steps, args.warmup, world, flush)
+             (W, wms, wflops), fms, ms64) = fwd_leg(args.steps, args.warmup, world, flush)
         if "decode" in legs:
             dms, kv_bytes, dec_klens, (page, pms) = decode_leg(args.steps, args.warmup, world,
                                                                flush)
@@ -955,10 +970,10 @@ def main():
     t_e2e = max_over_ranks(float(np.mean(ms_e2e)), world)
     value = world * flops / (t_step * 1e-3) / 1e12
     achieved = flops / (float(np.mean(ms)) * 1e-3) / 1e12
-    # one persistent forward kernel per step: timed forward, e2e, sliding-window, 8-bit and
-    # packed-prefill loops
+    # one persistent forward kernel per step: timed forward, e2e, sliding-window, 8-bit,
+    # d = 64 and packed-prefill loops
     launches = (args.steps + FWD["B"] * max(3, args.steps // 2) + args.steps + args.steps
-                + args.steps)
+                + args.steps + args.steps)
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -1014,6 +1029,13 @@ def main():
                      "peak_source": f"{pk['source']} burst bf16 x 2 (the nominal 8-bit:bf16 "
                                     f"dense ratio, 4.5 : 2.25 PFLOP/s)",
                      "kernel": "attn_fwd_impl::fwd_kernel<128,MODE_FP8>"},
+    }
+    t_64 = max_over_ranks(float(np.mean(ms64)), world)
+    fl64 = flops * 64 / FWD["d"]
+    line["d64"] = {
+        "workload": "the causal prefill forward B4 H16 L4096 at d = 64",
+        "value": world * fl64 / (t_64 * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": t_64,
+        "flops_per_step": fl64,
     }
     if "decode" in legs:
         t_d = max_over_ranks(float(np.mean(dms)), world)
