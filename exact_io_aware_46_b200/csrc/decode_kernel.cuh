@@ -475,8 +475,8 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) decode_split_kernel(con
 // ---------------------------------------------------------------- tensor-core split kernel
 //
 // The same split (one CTA per chunk of CH keys of one sequence and kv head)
-// with the two products on the tensor core instead of the CUDA cores, for a
-// contiguous cache at d = 128: per block of 128 keys,
+// with the two products on the tensor core instead of the CUDA cores, at
+// d = 128 (contiguous or paged cache): per block of 128 keys,
 //     S^T = K Q^T     (M = 128 keys on the TMEM lanes, N = 16 query heads
 //                      padded, K = d; both operands K-major in shared memory)
 //     O^T += V^T P^T  (M = d = 128 lanes, N = 16 heads, K = 128 keys; V^T is
