@@ -6,11 +6,12 @@
 // (4 FLOP/B with 4 query heads per key/value head), so the kernel is bound by
 // HBM bandwidth.  Two split kernels compute the same partials:
 //
-//  * tensor-core split kernel (d = 128, contiguous or paged cache; further
-//    below): the scores and the PV product as small tcgen05 MMAs (16 heads
-//    padded), so the CUDA cores only form the exponentials and the kernel
+//  * tensor-core split kernel (d = 64 and 128, contiguous or paged cache;
+//    further below): the scores and the PV product as small tcgen05 MMAs (16
+//    heads padded), so the CUDA cores only form the exponentials and the kernel
 //    streams the cache;
-//  * CUDA-core split kernel (d = 64): one CTA per (sequence, key/value head,
+//  * CUDA-core split kernel (the fallback for caches of more than 65535 chunks
+//    or pages of fewer than 8 rows): one CTA per (sequence, key/value head,
 //    chunk of CH keys), three CTAs per SM.
 //    A producer thread streams the chunk's K and V rows (contiguous in the
 //    cache) with 1-D bulk copies into a ring of shared-memory stages; four
@@ -475,17 +476,17 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) decode_split_kernel(con
 // ---------------------------------------------------------------- tensor-core split kernel
 //
 // The same split (one CTA per chunk of CH keys of one sequence and kv head)
-// with the two products on the tensor core instead of the CUDA cores, at
-// d = 128 (contiguous or paged cache): per block of 128 keys,
+// with the two products on the tensor core instead of the CUDA cores (d = 64
+// or 128, contiguous or paged cache): per block of 128 keys,
 //     S^T = K Q^T     (M = 128 keys on the TMEM lanes, N = 16 query heads
 //                      padded, K = d; both operands K-major in shared memory)
 //     O^T += V^T P^T  (M = d = 128 lanes, N = 16 heads, K = 128 keys; V^T is
 //                      the V tile read MN-major, P is written by the softmax
 //                      threads as a 16-row K-major tile)
 // so the CUDA cores only form the scores' exponentials (G per key) and the
-// kernel streams the cache (measured on B200, B64 Hq32 Hkv8 d128, cache
-// 32768, k_len ~ U[1024, 32768]: 6902 against 6400 GB/s for the CUDA-core
-// kernel in the same process).  Warp 0 loads K and V blocks with TMA (128-byte
+// kernel streams the cache (measured on B200, B64 Hq32 Hkv8, cache 32768,
+// k_len ~ U[1024, 32768]: 6902 against 6400 GB/s for the CUDA-core kernel in
+// the same process at d = 128, 4900 against 4486 GB/s at d = 64).  Warp 0 loads K and V blocks with TMA (128-byte
 // swizzle) into a ring of three 32 KB slots, warp 1 issues the MMAs, warps
 // 2-5 (one key row, then one d index, per thread) run the online softmax of
 // the three-ledgers page per block with the stale-max threshold and write the
@@ -530,7 +531,11 @@ template <int D, bool PAGED>
 __global__ void __launch_bounds__(NTHREADS, 2)
     split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const SplitParams p) {
-  static_assert(D == 128, "one 128-lane d tile");
+  // d = 64: K and V tiles are one 64-column panel; O^T = V^T P^T still runs at
+  // M = 128 over the slot's two panels, and the second (zero-filled once) only
+  // feeds lanes 64-127, which are never read
+  static_assert(D == 128 || D == 64, "head dimension");
+  constexpr int DP = D / 64;  // 64-column panels per K or V tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = sm100::smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
@@ -619,7 +624,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         const int slot = u % NSLOT;
         if (!sm100::mbar_wait(&kv_empty[slot], ((u / NSLOT) & 1) ^ 1, abort_flag, p.status, 21))
           break;
-        sm100::mbar_arrive_expect_tx(&kv_full[slot], SLOT);
+        sm100::mbar_arrive_expect_tx(&kv_full[slot], BK * D * 2);
         ++issued;
         const int row = k0 + (u >> 1) * BK;
         if constexpr (PAGED) {
@@ -630,13 +635,13 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             const int r = row + sg * br;
             const int blk = r >> p.page_log2;
             const int pg = blk <= last_blk ? __ldg(bt + blk) : p.n_pages;
-            for (int c = 0; c < 2; ++c)
+            for (int c = 0; c < DP; ++c)
               tma_load_4d((u & 1) ? &tmV : &tmK, &kv_full[slot],
                           smem + OFF_RING + slot * SLOT + c * PANEL + sg * br * 128, c * 64,
                           r & (page - 1), hkv, pg);
           }
         } else {
-          for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < DP; ++c)
             sm100::tma_load_3d((u & 1) ? &tmV : &tmK, &kv_full[slot],
                                smem + OFF_RING + slot * SLOT + c * PANEL, c * 64, row, head_kv);
         }
@@ -697,18 +702,27 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     const int r = q * 32 + sm100::lane_id();     // TMEM lane: key row of the block, then d
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const int G = p.G;
-    // Q tile (16 rows, heads >= G zero) and the constant zero rows of P
-    for (int e = t; e < NH * 16; e += 128) {
-      const int g = e >> 4, c16 = e & 15;
+    // Q tile (16 rows of D / 8 16-byte chunks, heads >= G zero) and the
+    // constant zero rows of P (16 chunks per row: 128 keys)
+    for (int e = t; e < NH * (D / 8); e += 128) {
+      const int g = e / (D / 8), c16 = e % (D / 8);
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
       if (g < G)
         v = __ldg(reinterpret_cast<const uint4*>(
                       p.Q + (static_cast<size_t>(b) * p.Hq + hkv * G + g) * D) + c16);
       *reinterpret_cast<uint4*>(smem + OFF_Q + (c16 >> 3) * HPANEL + g * 128 +
                                 (((c16 & 7) ^ (g & 7)) << 4)) = v;
+    }
+    for (int e = t; e < NH * 16; e += 128) {
+      const int g = e >> 4, c16 = e & 15;
       if (g >= G)
         *reinterpret_cast<uint4*>(smem + OFF_P + (c16 >> 3) * HPANEL + g * 128 + ((c16 & 7) << 4)) =
             make_uint4(0u, 0u, 0u, 0u);
+    }
+    if constexpr (DP == 1) {  // the second panel of every ring slot: zeros
+      for (int e = t; e < NSLOT * (PANEL / 16); e += 128)
+        *reinterpret_cast<uint4*>(smem + OFF_RING + (e / (PANEL / 16)) * SLOT + PANEL +
+                                  (e % (PANEL / 16)) * 16) = make_uint4(0u, 0u, 0u, 0u);
     }
     sm100::fence_proxy_async_smem();
     __syncwarp();
@@ -819,7 +833,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       const float ls = rs[h] + rs[NH + h] + rs[2 * NH + h] + rs[3 * NH + h];
       const size_t ph = (static_cast<size_t>(b) * p.Hq + hkv * G + h) * p.nsm + chunk;
       const bool has = live && ls > 0.f;
-      p.part_o[ph * D + r] = has ? __uint_as_float(o[h]) / ls : 0.f;
+      if (r < D) p.part_o[ph * D + r] = has ? __uint_as_float(o[h]) / ls : 0.f;
       if (r == 0) p.part_lse[ph] = has ? m_use[h] + log2f(ls) : -INFINITY;
     }
   }
@@ -888,19 +902,19 @@ cudaError_t launch_t(const SplitParams& sp, const CombineParams& cp, cudaStream_
 // (B64 Hq32 Hkv8 d128, cache 32768, k_len ~ U[1024, 32768], 64-row pages in a
 // random order): the paged cache reads at 6951 GB/s on it against 6066-6171
 // GB/s on the CUDA-core kernel, the same rate as the contiguous cache.
-template <bool PAGED>
+template <int D, bool PAGED>
 cudaError_t launch_tc(const SplitParams& sp, const CombineParams& cp, cudaStream_t s) {
   CUtensorMap tk, tv;
   const long long heads = static_cast<long long>(sp.B) * sp.Hkv;
   const int page = 1 << sp.page_log2;
   const int br = page < tc::BK ? page : tc::BK;
   const bool maps =
-      PAGED ? make_tmap_paged(&tk, sp.K, 128, page, sp.Hkv, sp.n_pages, br) &&
-                  make_tmap_paged(&tv, sp.V, 128, page, sp.Hkv, sp.n_pages, br)
-            : attn_bwd_impl::make_tmap_rows(&tk, sp.K, 128, sp.Lmax, heads, tc::BK) &&
-                  attn_bwd_impl::make_tmap_rows(&tv, sp.V, 128, sp.Lmax, heads, tc::BK);
+      PAGED ? make_tmap_paged(&tk, sp.K, D, page, sp.Hkv, sp.n_pages, br) &&
+                  make_tmap_paged(&tv, sp.V, D, page, sp.Hkv, sp.n_pages, br)
+            : attn_bwd_impl::make_tmap_rows(&tk, sp.K, D, sp.Lmax, heads, tc::BK) &&
+                  attn_bwd_impl::make_tmap_rows(&tv, sp.V, D, sp.Lmax, heads, tc::BK);
   if (!maps) return attn_host::report(cudaErrorInvalidValue, "decode tensor maps");
-  auto kernel = tc::split_kernel<128, PAGED>;
+  auto kernel = tc::split_kernel<D, PAGED>;
   cudaError_t e = attn_host::report(attn_host::set_smem(kernel, tc::SMEM_BYTES),
                                     "decode tensor-core kernel shared-memory attribute");
   if (e != cudaSuccess) return e;
@@ -910,8 +924,8 @@ cudaError_t launch_tc(const SplitParams& sp, const CombineParams& cp, cudaStream
            s>>>(tk, tv, spl);
   if ((e = attn_host::report_launch(kernel, "decode tensor-core split kernel")) != cudaSuccess)
     return e;
-  decode_combine_kernel<128><<<sp.B * sp.Hq, 128, 0, s>>>(cp);
-  return attn_host::report_launch(decode_combine_kernel<128>, "decode_combine_kernel");
+  decode_combine_kernel<D><<<sp.B * sp.Hq, D, 0, s>>>(cp);
+  return attn_host::report_launch(decode_combine_kernel<D>, "decode_combine_kernel");
 }
 
 // Paged cache description for launch(); Lmax is then max_blocks * page.
@@ -955,11 +969,13 @@ inline cudaError_t launch(const __nv_bfloat16* Q, const __nv_bfloat16* K, const 
   cp.Lmax = Lmax;
   cp.nsm = sp.nsm;
   const bool wide = sp.G > 4;
-  // d = 128: the tensor-core kernel (paged caches with pages of at least 8
-  // rows, so that every page segment starts on a 1024-byte swizzle atom)
-  if (d == 128 && sp.nsm <= 65535 && static_cast<long long>(Hkv) * B <= 0x7fffffffLL &&
-      (!paged || paged->page_log2 >= 3))
-    return paged ? launch_tc<true>(sp, cp, s) : launch_tc<false>(sp, cp, s);
+  // the tensor-core kernel (paged caches with pages of at least 8 rows, so
+  // that every page segment starts on a 1024-byte swizzle atom)
+  if (sp.nsm <= 65535 && static_cast<long long>(Hkv) * B <= 0x7fffffffLL &&
+      (!paged || paged->page_log2 >= 3)) {
+    if (d == 128) return paged ? launch_tc<128, true>(sp, cp, s) : launch_tc<128, false>(sp, cp, s);
+    return paged ? launch_tc<64, true>(sp, cp, s) : launch_tc<64, false>(sp, cp, s);
+  }
   if (d == 128) return wide ? launch_t<128, 8>(sp, cp, s) : launch_t<128, 4>(sp, cp, s);
   return wide ? launch_t<64, 8>(sp, cp, s) : launch_t<64, 4>(sp, cp, s);
 }
