@@ -446,6 +446,7 @@ attn_status_t attn_fwd_splitkv_decode(const attn_bf16_t* Q, const attn_bf16_t* K
   if (ws_bytes < attn_decode_workspace_size(B, Hq, Hkv, Lmax, d)) return ATTN_ERR_INVALID;
   if (d != 128 && d != 64) return ATTN_ERR_UNSUPPORTED;
   if (!attn_decode_impl::supported_group(Hq / Hkv)) return ATTN_ERR_UNSUPPORTED;
+  if (!attn_decode_impl::supported_shape(B, Hkv, Lmax, 0)) return ATTN_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int sms = device_sms();
   if (sms <= 0) return ATTN_ERR_CUDA;
@@ -480,6 +481,7 @@ attn_status_t attn_fwd_splitkv_decode_paged(const attn_bf16_t* Q, const attn_bf1
   if (ws_bytes < attn_decode_workspace_size(B, Hq, Hkv, Lmax, d)) return ATTN_ERR_INVALID;
   if (d != 128 && d != 64) return ATTN_ERR_UNSUPPORTED;
   if (!attn_decode_impl::supported_group(Hq / Hkv)) return ATTN_ERR_UNSUPPORTED;
+  if (!attn_decode_impl::supported_shape(B, Hkv, Lmax, page_size)) return ATTN_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int sms = device_sms();
   if (sms <= 0) return ATTN_ERR_CUDA;

@@ -3,25 +3,15 @@
 // Decode is the "short query scans a long history" case of "FlashAttention and
 // long context: three ledgers" (prefill vs decode): per step the whole cache
 // row range [0, k_len) is read once and the arithmetic per byte is tiny
-// (4 FLOP/B with 4 query heads per key/value head), so the kernel is bound by
-// HBM bandwidth.  Two split kernels compute the same partials:
+// (4 FLOP/B with 4 query heads per key/value head), so the kernels are bound by
+// HBM bandwidth:
 //
-//  * tensor-core split kernel (d = 64 and 128, contiguous or paged cache;
-//    further below): the scores and the PV product as small tcgen05 MMAs (16
-//    heads padded), so the CUDA cores only form the exponentials and the kernel
-//    streams the cache;
-//  * CUDA-core split kernel (the fallback for caches of more than 65535 chunks
-//    or pages of fewer than 8 rows): one CTA per (sequence, key/value head,
-//    chunk of CH keys), three CTAs per SM.
-//    A producer thread streams the chunk's K and V rows (contiguous in the
-//    cache) with 1-D bulk copies into a ring of shared-memory stages; four
-//    compute warps each own 16 rows of every stage.  A half-warp covers one
-//    key row (16 lanes x d/16 elements), forms partial dot products with all
-//    query heads of the group (packed fp32x2 FMA), and a transpose-reduction
-//    across the 16 lanes leaves every lane with one complete (row, head)
-//    score.  The online softmax of the three-ledgers page runs per warp with a stale-max
-//    rescale threshold; warps are merged at the end and the chunk's
-//    normalised output and log2-sum-exp are written as a partial.
+//  * split kernel (tensor cores; below): one CTA per (sequence, key/value
+//    head, chunk of CH keys); the scores and the PV product of each 128-key
+//    block run as small tcgen05 MMAs (16 heads padded) over a TMA-fed ring, so
+//    the CUDA cores only form the exponentials and the kernel streams the
+//    cache; every chunk writes its normalised output and log2-sum-exp as a
+//    partial;
 //  * combine kernel: merges a sequence's partials with the normalised rule of
 //    the FlashAttention-2 tutorial, 2.1.3.  Writing each partial as
 //    (O_c, LSE_c) with e^{LSE_c} = e^{m_c} l_c gives exactly that rule's
@@ -45,21 +35,7 @@ namespace attn_decode_impl {
 bool make_tmap_paged(CUtensorMap* m, const void* base, int d, int page, int Hkv, int n_pages,
                      int box_rows);
 
-// Measured on B200 (B64 Hq32 Hkv8 d128, cache 32768, k_len ~ U[1024, 32768]):
-// chunk 1024 / 3 stages of 64 rows / 2 CTAs per SM 5.56 TB/s; 2 stages / 3
-// CTAs per SM 5.98 TB/s; chunk 2048, 2 x 64-row stages, 3 CTAs per SM 6.08-6.11
-// TB/s; chunk 2048, 4 x 32-row stages, 3 CTAs per SM 6.23 TB/s (shipped);
-// chunk 4096 5.88 TB/s, chunk 512 5.01 TB/s; 4 CTAs per SM (96 registers,
-// spills) 5.53-5.64 TB/s.  More resident warps hide the shared-memory and
-// shuffle latency of the compute warps, finer stages release ring space
-// sooner, and longer chunks amortise a CTA's start (query load, first copy)
-// and its final merge.
-constexpr int CH = 2048;  // keys per split
-constexpr int SR = 32;    // key rows per shared-memory stage
-constexpr int NST = 4;    // stages
-constexpr int CTAS_PER_SM = 3;
-constexpr int NCW = 4;    // compute warps
-constexpr int NTHREADS = (NCW + 1) * 32;
+constexpr int CH = 2048;  // keys per split (measured on B200 against 1024, 3072, 4096 and 8192)
 
 inline bool supported_group(int G) { return G == 1 || G == 2 || G == 4 || G == 8; }
 
@@ -69,11 +45,6 @@ inline size_t partials_bytes(int B, int Hq, int, int Lmax, int d) {
   const size_t n = static_cast<size_t>(B) * Hq * n_split_max(Lmax);
   size_t bytes = n * d * 4 + n * 4;
   return (bytes + 255) & ~static_cast<size_t>(255);
-}
-
-template <int D>
-constexpr int smem_bytes() {
-  return NST * SR * D * 2 * 2 + 256;
 }
 
 struct SplitParams {
@@ -90,10 +61,17 @@ struct SplitParams {
   // row r of sequence b lives in page block_table[b * max_blocks + r / page]
   const int* block_table;
   int max_blocks, page_log2, n_pages;
-  // grid layout: 1 = (sequence x kv head, chunk counted from the sequence's
-  // end), 0 = (chunk, kv head, sequence)
-  int from_end;
 };
+
+// The grid is (sequence x kv head, chunk position counted from the sequence's
+// end): every sequence's last (partial, shorter) chunk is dispatched last, so
+// the grid's tail is short.  Its second dimension limits the cache to 65535
+// chunks; paged caches need pages of at least 8 rows (a page segment must
+// start on a 1024-byte swizzle atom).  page_rows = 0 for a contiguous cache.
+inline bool supported_shape(long long B, int Hkv, int Lmax, int page_rows) {
+  return n_split_max(Lmax) <= 65535 && B * Hkv <= 0x7fffffffLL &&
+         (page_rows == 0 || page_rows >= 8);
+}
 
 __device__ __forceinline__ int valid_klen(const int* k_lens, int b, int Lmax, int* status,
                                           bool report) {
@@ -105,379 +83,11 @@ __device__ __forceinline__ int valid_klen(const int* k_lens, int b, int Lmax, in
   return kl;
 }
 
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
-                                         uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          sm100::smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(sm100::smem_u32(bar))
-      : "memory");
-}
-
-// bf16x2 word -> two floats (exact widening)
-__device__ __forceinline__ float2 bf2(uint32_t w) {
-  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-}
-
-// One stage of the transpose-reduction: lanes whose bit `O` is clear keep the
-// lower half of their N values, the others the upper half; each adds the half
-// its partner (lane ^ O) gives away.
-template <int O, int N>
-__device__ __forceinline__ void tr_stage(float (&v)[16], bool upper) {
-#pragma unroll
-  for (int i = 0; i < N / 2; ++i) {
-    const float send = upper ? v[i] : v[i + N / 2];
-    const float keep = upper ? v[i + N / 2] : v[i];
-    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
-  }
-}
-
-// Transpose-reduction of 16 values per lane across the 16 lanes of a
-// half-warp (15 shuffles instead of 64): afterwards lane hl holds the full sum
-// of value index hl.
-__device__ __forceinline__ float transpose_reduce16(float (&v)[16], int hl) {
-  tr_stage<8, 16>(v, (hl & 8) != 0);
-  tr_stage<4, 8>(v, (hl & 4) != 0);
-  tr_stage<2, 4>(v, (hl & 2) != 0);
-  tr_stage<1, 2>(v, (hl & 1) != 0);
-  return v[0];
-}
-
-// One stage of key rows for one compute warp: this warp's rows of the stage
-// (WROWS of SR, in steps of STEP rows: a half-warp per row, 16 lanes x d/16
-// elements) update the warp's running max m_run, per-lane sum l_lane and
-// unnormalised outputs o2 of the GP (padded) query heads.  q2: the heads'
-// query slices of this lane, pre-scaled by scale * log2(e).
-template <int D, int GP>
-__device__ __forceinline__ void stage_rows(const uint8_t* kst, const uint8_t* vst, int n, int warp,
-                                           int lane, int G, const float2 (&q2)[GP][D / 32],
-                                           float2 (&o2)[GP][D / 32], float& m_run,
-                                           float& l_lane) {
-  constexpr int EPL = D / 16;    // elements of a row per lane
-  constexpr int R = 16 / GP;     // rows per half-warp per step
-  constexpr int STEP = 2 * R;    // rows per warp per step
-  constexpr int WROWS = SR / NCW;
-  constexpr int ROWB = D * 2;    // bytes per row
-  const int half = lane >> 4, hl = lane & 15;
-  const int g_own = hl % GP;        // head of this lane's score
-  const int i_own = hl / GP;        // row (within the half's R rows) of this lane's score
-#pragma unroll 1
-  for (int rb = warp * WROWS; rb < warp * WROWS + WROWS; rb += STEP) {
-    if (rb >= n) break;
-    // ---- scores: partial dots of this lane's d-slice, then transpose-reduce
-    float part[16];
-#pragma unroll
-    for (int i = 0; i < R; ++i) {
-      const int row = rb + half * R + i;
-      uint32_t kw[EPL / 2];
-      if (row < n) {
-        if constexpr (EPL == 8) {
-          const uint4 t = *reinterpret_cast<const uint4*>(kst + row * ROWB + hl * 16);
-          kw[0] = t.x; kw[1] = t.y; kw[2] = t.z; kw[3] = t.w;
-        } else {
-          const uint2 t = *reinterpret_cast<const uint2*>(kst + row * ROWB + hl * 8);
-          kw[0] = t.x; kw[1] = t.y;
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < EPL / 2; ++c) kw[c] = 0u;
-      }
-      float2 kf[EPL / 2];
-#pragma unroll
-      for (int c = 0; c < EPL / 2; ++c) kf[c] = bf2(kw[c]);
-#pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < EPL / 2; ++c) acc = __ffma2_rn(q2[g][c], kf[c], acc);
-        part[i * GP + g] = acc.x + acc.y;
-      }
-    }
-    const float sc = transpose_reduce16(part, hl);
-    const int my_row = rb + half * R + i_own;
-    const float s2 = (my_row < n && g_own < G) ? sc : -INFINITY;
-
-    // ---- online softmax for this step's rows (per head: lanes sharing g_own)
-    float m_blk = s2;
-#pragma unroll
-    for (int o = GP; o < 32; o <<= 1) m_blk = fmaxf(m_blk, __shfl_xor_sync(0xffffffffu, m_blk, o));
-    const bool need = m_blk > m_run + 8.0f;
-    if (__any_sync(0xffffffffu, need)) {
-      const float m_new = fmaxf(m_run, m_blk);
-      const float alpha = (m_run == -INFINITY) ? 0.f : sm100::ex2(m_run - m_new);
-      l_lane *= alpha;
-      m_run = m_new;
-#pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        const float a = __shfl_sync(0xffffffffu, alpha, g);
-        const float2 a2 = make_float2(a, a);
-#pragma unroll
-        for (int c = 0; c < EPL / 2; ++c) o2[g][c] = __fmul2_rn(o2[g][c], a2);
-      }
-    }
-    const float pv = (s2 == -INFINITY) ? 0.f : sm100::ex2(s2 - m_run);
-    l_lane += pv;
-
-    // ---- o += p V for this half's rows
-#pragma unroll
-    for (int i = 0; i < R; ++i) {
-      const int row = rb + half * R + i;
-      uint32_t vw[EPL / 2];
-      if (row < n) {
-        if constexpr (EPL == 8) {
-          const uint4 t = *reinterpret_cast<const uint4*>(vst + row * ROWB + hl * 16);
-          vw[0] = t.x; vw[1] = t.y; vw[2] = t.z; vw[3] = t.w;
-        } else {
-          const uint2 t = *reinterpret_cast<const uint2*>(vst + row * ROWB + hl * 8);
-          vw[0] = t.x; vw[1] = t.y;
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < EPL / 2; ++c) vw[c] = 0u;
-      }
-      float2 vf[EPL / 2];
-#pragma unroll
-      for (int c = 0; c < EPL / 2; ++c) vf[c] = bf2(vw[c]);
-#pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        const float pg = __shfl_sync(0xffffffffu, pv, half * 16 + i * GP + g);
-        const float2 p2 = make_float2(pg, pg);
-#pragma unroll
-        for (int c = 0; c < EPL / 2; ++c) o2[g][c] = __ffma2_rn(p2, vf[c], o2[g][c]);
-      }
-    }
-  }
-}
-
-// GP: query heads per key/value head, padded to 4 or 8 (heads >= G are inert).
-template <int D, int GP>
-__global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) decode_split_kernel(const SplitParams p) {
-  constexpr int EPL = D / 16;    // elements of a row per lane
-  constexpr int R = 16 / GP;     // rows per half-warp per step
-  constexpr int STEP = 2 * R;    // rows per warp per step
-  constexpr int WROWS = SR / NCW;
-  static_assert(SR % NCW == 0 && WROWS % STEP == 0, "a warp's rows of a stage must be whole steps");
-  constexpr int ROWB = D * 2;    // bytes per row
-  constexpr int STAGE = SR * ROWB;  // bytes of K (or V) per stage
-
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* sK = smem;
-  uint8_t* sV = smem + NST * STAGE;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + 2 * NST * STAGE);
-  uint64_t* empty = full + NST;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NST);
-
-  // With from_end, blocks are dispatched chunk position by chunk position
-  // counted from each sequence's end, so the sequences' last (partial, shorter)
-  // chunks run last and the grid's tail is short: measured on B200 (B64 Hq32
-  // Hkv8 d128, cache 32768, k_len ~ U[1024, 32768]) 6382 against 6242 GB/s for
-  // chunk-major order within each sequence, output bit-identical.
-  int chunk, hkv, b;
-  bool reporter;
-  if (p.from_end) {
-    hkv = blockIdx.x % p.Hkv;
-    b = blockIdx.x / p.Hkv;
-    reporter = blockIdx.y == gridDim.y - 1 && hkv == 0;
-  } else {
-    chunk = blockIdx.x;
-    hkv = blockIdx.y;
-    b = blockIdx.z;
-    reporter = chunk == 0 && hkv == 0;
-  }
-  const int kl = valid_klen(p.k_lens, b, p.Lmax, p.status, reporter && threadIdx.x == 0);
-  if (p.from_end) chunk = (kl + CH - 1) / CH - static_cast<int>(gridDim.y - blockIdx.y);
-  if (chunk < 0) return;
-  const int k0 = chunk * CH;
-  if (k0 >= kl) return;
-  const int rows = min(CH, kl - k0);
-  const int nstages = (rows + SR - 1) / SR;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < NST; ++i) {
-      sm100::mbar_init(&full[i], 1);
-      sm100::mbar_init(&empty[i], NCW);
-    }
-    *abort_flag = 0;
-    sm100::fence_barrier_init();
-  }
-  // paged cache: every block-table entry of this chunk is checked before any
-  // copy is issued; a chunk with a bad entry reads nothing and contributes an
-  // empty partial
-  const int* bt = p.block_table ? p.block_table + static_cast<size_t>(b) * p.max_blocks : nullptr;
-  bool bad_page = false;
-  if (bt) {
-    const int blk1 = (k0 + rows - 1) >> p.page_log2;
-    for (int bb = (k0 >> p.page_log2) + threadIdx.x; bb <= blk1; bb += NTHREADS) {
-      const int pg = __ldg(bt + bb);
-      if (pg < 0 || pg >= p.n_pages) bad_page = true;
-    }
-  }
-  if (__syncthreads_or(bad_page)) {
-    if (threadIdx.x == 0) atomicOr(p.status, ATTN_DEV_BAD_PAGE);
-    for (int e = threadIdx.x; e < p.G * D; e += NTHREADS) {
-      const size_t ph = (static_cast<size_t>(b) * p.Hq + hkv * p.G + e / D) * p.nsm + chunk;
-      p.part_o[ph * D + e % D] = 0.f;
-      if (e % D == 0) p.part_lse[ph] = -INFINITY;
-    }
-    return;
-  }
-
-  if (warp == NCW) {
-    if (lane == 0) {
-      const uint8_t* gK = reinterpret_cast<const uint8_t*>(p.K);
-      const uint8_t* gV = reinterpret_cast<const uint8_t*>(p.V);
-      const size_t head_row0 = (static_cast<size_t>(b) * p.Hkv + hkv) * p.Lmax + k0;
-      const int page = 1 << p.page_log2;
-      int issued = 0;  // stages whose copies were issued
-      for (int s = 0; s < nstages; ++s) {
-        const int slot = s % NST;
-        if (!sm100::mbar_wait(&empty[slot], ((s / NST) & 1) ^ 1, abort_flag, p.status)) break;
-        ++issued;
-        const int n = min(SR, rows - s * SR);
-        const uint32_t bytes = static_cast<uint32_t>(n * ROWB);
-        sm100::mbar_arrive_expect_tx(&full[slot], 2 * bytes);
-        if (!bt) {
-          const size_t off = (head_row0 + static_cast<size_t>(s) * SR) * ROWB;
-          bulk_g2s(sK + slot * STAGE, gK + off, bytes, &full[slot]);
-          bulk_g2s(sV + slot * STAGE, gV + off, bytes, &full[slot]);
-        } else {
-          // one copy per page segment of the stage's rows
-          int row = k0 + s * SR;
-          const int end = row + n;
-          uint32_t dst = static_cast<uint32_t>(slot * STAGE);
-          while (row < end) {
-            const int in_page = row & (page - 1);
-            const int seg = min(page - in_page, end - row);
-            const int pg = __ldg(bt + (row >> p.page_log2));
-            const size_t off =
-                ((static_cast<size_t>(pg) * p.Hkv + hkv) * page + in_page) * ROWB;
-            const uint32_t sb = static_cast<uint32_t>(seg * ROWB);
-            bulk_g2s(sK + dst, gK + off, sb, &full[slot]);
-            bulk_g2s(sV + dst, gV + off, sb, &full[slot]);
-            dst += sb;
-            row += seg;
-          }
-        }
-      }
-      // the CTA must not exit while bulk copies still write into its shared
-      // memory, which can happen once a wait has expired (the compute warps
-      // then stop reading the ring): wait, bounded, for the last issued stage
-      // of every slot (in normal operation these have long landed)
-      for (int s = issued - 1; s >= 0 && s >= issued - NST; --s)
-        sm100::mbar_wait_drain(&full[s % NST], (s / NST) & 1);
-    }
-    return;  // the producer takes no part in the merge below
-  }
-
-  // ---------------------------------------------------------------- compute warps
-  const int half = lane >> 4, hl = lane & 15;
-
-  // q of every head in the group, pre-scaled by scale * log2(e)
-  float2 q2[GP][EPL / 2];
-#pragma unroll
-  for (int g = 0; g < GP; ++g) {
-    if (g < p.G) {
-      const __nv_bfloat16* qp =
-          p.Q + (static_cast<size_t>(b) * p.Hq + hkv * p.G + g) * D + hl * EPL;
-      const uint32_t* qw = reinterpret_cast<const uint32_t*>(qp);
-#pragma unroll
-      for (int c = 0; c < EPL / 2; ++c) {
-        const float2 f = bf2(__ldg(qw + c));
-        q2[g][c] = make_float2(f.x * p.scale_log2, f.y * p.scale_log2);
-      }
-    } else {
-#pragma unroll
-      for (int c = 0; c < EPL / 2; ++c) q2[g][c] = make_float2(0.f, 0.f);
-    }
-  }
-
-  float2 o2[GP][EPL / 2];
-#pragma unroll
-  for (int g = 0; g < GP; ++g)
-#pragma unroll
-    for (int c = 0; c < EPL / 2; ++c) o2[g][c] = make_float2(0.f, 0.f);
-  float m_run = -INFINITY, l_lane = 0.f;
-  bool ok = true;
-
-  for (int s = 0; s < nstages && ok; ++s) {
-    const int slot = s % NST;
-    if (!(ok = sm100::mbar_wait(&full[slot], (s / NST) & 1, abort_flag, p.status))) break;
-    const int n = min(SR, rows - s * SR);
-    const uint8_t* kst = sK + slot * STAGE;
-    const uint8_t* vst = sV + slot * STAGE;
-    stage_rows<D, GP>(kst, vst, n, warp, lane, p.G, q2, o2, m_run, l_lane);
-    __syncwarp();
-    if (lane == 0) sm100::mbar_arrive(&empty[slot]);
-  }
-
-  // ---------------------------------------------------------------- merge warps
-  // per head: l over the lanes sharing g_own; o over the two half-warps
-#pragma unroll
-  for (int o = GP; o < 32; o <<= 1) l_lane += __shfl_xor_sync(0xffffffffu, l_lane, o);
-#pragma unroll
-  for (int g = 0; g < GP; ++g)
-#pragma unroll
-    for (int c = 0; c < EPL / 2; ++c) {
-      o2[g][c].x += __shfl_xor_sync(0xffffffffu, o2[g][c].x, 16);
-      o2[g][c].y += __shfl_xor_sync(0xffffffffu, o2[g][c].y, 16);
-    }
-  // all stages are consumed: reuse the K ring for the per-warp partials --
-  // unless a wait expired (every compute warp that stopped early set the
-  // abort flag before this barrier): bulk copies may then still be landing in
-  // the ring, so the chunk contributes an empty partial written directly
-  sm100::named_bar_sync(1, NCW * 32);
-  if (*abort_flag) {
-    for (int e = threadIdx.x; e < p.G * D; e += NCW * 32) {
-      const size_t ph = (static_cast<size_t>(b) * p.Hq + hkv * p.G + e / D) * p.nsm + chunk;
-      p.part_o[ph * D + e % D] = 0.f;
-      if (e % D == 0) p.part_lse[ph] = -INFINITY;
-    }
-    return;
-  }
-  float* wm = reinterpret_cast<float*>(sK);        // [NCW][GP]
-  float* wl = wm + NCW * GP;                       // [NCW][GP]
-  float* wo = wl + NCW * GP;                       // [NCW][GP][D]
-  if (lane < GP) {  // lane g (half 0, row 0) owns head g's statistics
-    wm[warp * GP + lane] = ok ? m_run : -INFINITY;
-    wl[warp * GP + lane] = ok ? l_lane : 0.f;
-  }
-  if (half == 0) {
-#pragma unroll
-    for (int g = 0; g < GP; ++g)
-#pragma unroll
-      for (int c = 0; c < EPL / 2; ++c) {
-        wo[(warp * GP + g) * D + hl * EPL + 2 * c] = o2[g][c].x;
-        wo[(warp * GP + g) * D + hl * EPL + 2 * c + 1] = o2[g][c].y;
-      }
-  }
-  sm100::named_bar_sync(1, NCW * 32);
-  for (int e = threadIdx.x; e < p.G * D; e += NCW * 32) {
-    const int g = e / D, dd = e % D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < NCW; ++w) M = fmaxf(M, wm[w * GP + g]);
-    float lsum = 0.f, acc = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < NCW; ++w) {
-        const float mw = wm[w * GP + g];
-        const float f = (mw == -INFINITY) ? 0.f : sm100::ex2(mw - M);
-        lsum += f * wl[w * GP + g];
-        acc += f * wo[(w * GP + g) * D + dd];
-      }
-    }
-    const size_t ph = (static_cast<size_t>(b) * p.Hq + hkv * p.G + g) * p.nsm + chunk;
-    p.part_o[ph * D + dd] = lsum > 0.f ? acc / lsum : 0.f;
-    if (dd == 0) p.part_lse[ph] = lsum > 0.f ? M + log2f(lsum) : -INFINITY;
-  }
-}
-
 // ---------------------------------------------------------------- tensor-core split kernel
 //
-// The same split (one CTA per chunk of CH keys of one sequence and kv head)
-// with the two products on the tensor core instead of the CUDA cores (d = 64
-// or 128, contiguous or paged cache): per block of 128 keys,
+// One CTA per chunk of CH keys of one sequence and kv head, the two products
+// on the tensor core (d = 64 or 128, contiguous or paged cache): per block of
+// 128 keys,
 //     S^T = K Q^T     (M = 128 keys on the TMEM lanes, N = 16 query heads
 //                      padded, K = d; both operands K-major in shared memory)
 //     O^T += V^T P^T  (M = d = 128 lanes, N = 16 heads, K = 128 keys; V^T is
@@ -485,12 +95,13 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) decode_split_kernel(con
 //                      threads as a 16-row K-major tile)
 // so the CUDA cores only form the scores' exponentials (G per key) and the
 // kernel streams the cache (measured on B200, B64 Hq32 Hkv8, cache 32768,
-// k_len ~ U[1024, 32768]: 6902 against 6400 GB/s for the CUDA-core kernel in
-// the same process at d = 128, 4900 against 4486 GB/s at d = 64).  Warp 0 loads K and V blocks with TMA (128-byte
-// swizzle) into a ring of three 32 KB slots, warp 1 issues the MMAs, warps
-// 2-5 (one key row, then one d index, per thread) run the online softmax of
-// the three-ledgers page per block with the stale-max threshold and write the
-// chunk's normalised partial.  The block chain (S, softmax, PV) is serial;
+// k_len ~ U[1024, 32768]: 6902 GB/s at d = 128 and 4900 GB/s at d = 64,
+// against 6400 and 4486 GB/s for an earlier split kernel that formed both
+// products on the CUDA cores, timed in the same process).  Warp 0 loads K and
+// V blocks with TMA (128-byte swizzle) into a ring of three 32 KB slots, warp
+// 1 issues the MMAs, warps 2-5 (one key row, then one d index, per thread) run
+// the online softmax of the three-ledgers page per block with the stale-max
+// threshold and write the chunk's normalised partial.  The block chain (S, softmax, PV) is serial;
 // with two CTAs per SM and the next block's K and V in flight during it, the
 // copies are the limit.
 namespace tc {
@@ -554,7 +165,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red = reinterpret_cast<float*>(smem + OFF_RED);
 
-  // the same chunk order as the CUDA-core kernel (from_end layout)
+  // grid (sequence x kv head, chunk position counted from the sequence's end)
   const int hkv = blockIdx.x % p.Hkv, b = blockIdx.x / p.Hkv;
   const int kl = valid_klen(p.k_lens, b, p.Lmax, p.status,
                             blockIdx.y == gridDim.y - 1 && hkv == 0 && threadIdx.x == 0);
@@ -880,28 +491,10 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const CombineParams p
     p.lse[bh] = wsum > 0.f ? (M + log2f(wsum)) * 0.69314718055994531f : -INFINITY;
 }
 
-template <int D, int GP>
-cudaError_t launch_t(const SplitParams& sp, const CombineParams& cp, cudaStream_t s) {
-  constexpr int smem = smem_bytes<D>();
-  cudaError_t e = attn_host::report(attn_host::set_smem(decode_split_kernel<D, GP>, smem),
-                                    "decode_split_kernel shared-memory attribute");
-  if (e != cudaSuccess) return e;
-  SplitParams spl = sp;
-  spl.from_end = sp.nsm <= 65535 && static_cast<long long>(sp.Hkv) * sp.B <= 0x7fffffffLL;
-  const dim3 grid = spl.from_end ? dim3(static_cast<unsigned>(sp.Hkv * sp.B), sp.nsm, 1)
-                                 : dim3(sp.nsm, sp.Hkv, sp.B);
-  decode_split_kernel<D, GP><<<grid, NTHREADS, smem, s>>>(spl);
-  if ((e = attn_host::report_launch(decode_split_kernel<D, GP>, "decode_split_kernel")) !=
-      cudaSuccess)
-    return e;
-  decode_combine_kernel<D><<<sp.B * sp.Hq, D, 0, s>>>(cp);
-  return attn_host::report_launch(decode_combine_kernel<D>, "decode_combine_kernel");
-}
-
-// The tensor-core split kernel (d = 128) and the combine.  Measured on B200
+// The split kernel and the combine.  Measured on B200
 // (B64 Hq32 Hkv8 d128, cache 32768, k_len ~ U[1024, 32768], 64-row pages in a
-// random order): the paged cache reads at 6951 GB/s on it against 6066-6171
-// GB/s on the CUDA-core kernel, the same rate as the contiguous cache.
+// random order): the paged cache reads at 6951 GB/s, the same rate as the
+// contiguous cache (the earlier CUDA-core split kernel: 6066-6171 GB/s).
 template <int D, bool PAGED>
 cudaError_t launch_tc(const SplitParams& sp, const CombineParams& cp, cudaStream_t s) {
   CUtensorMap tk, tv;
@@ -918,10 +511,8 @@ cudaError_t launch_tc(const SplitParams& sp, const CombineParams& cp, cudaStream
   cudaError_t e = attn_host::report(attn_host::set_smem(kernel, tc::SMEM_BYTES),
                                     "decode tensor-core kernel shared-memory attribute");
   if (e != cudaSuccess) return e;
-  SplitParams spl = sp;
-  spl.from_end = 1;
   kernel<<<dim3(static_cast<unsigned>(sp.Hkv * sp.B), sp.nsm, 1), tc::NTHREADS, tc::SMEM_BYTES,
-           s>>>(tk, tv, spl);
+           s>>>(tk, tv, sp);
   if ((e = attn_host::report_launch(kernel, "decode tensor-core split kernel")) != cudaSuccess)
     return e;
   decode_combine_kernel<D><<<sp.B * sp.Hq, D, 0, s>>>(cp);
@@ -968,16 +559,9 @@ inline cudaError_t launch(const __nv_bfloat16* Q, const __nv_bfloat16* K, const 
   cp.Hq = Hq;
   cp.Lmax = Lmax;
   cp.nsm = sp.nsm;
-  const bool wide = sp.G > 4;
-  // the tensor-core kernel (paged caches with pages of at least 8 rows, so
-  // that every page segment starts on a 1024-byte swizzle atom)
-  if (sp.nsm <= 65535 && static_cast<long long>(Hkv) * B <= 0x7fffffffLL &&
-      (!paged || paged->page_log2 >= 3)) {
-    if (d == 128) return paged ? launch_tc<128, true>(sp, cp, s) : launch_tc<128, false>(sp, cp, s);
-    return paged ? launch_tc<64, true>(sp, cp, s) : launch_tc<64, false>(sp, cp, s);
-  }
-  if (d == 128) return wide ? launch_t<128, 8>(sp, cp, s) : launch_t<128, 4>(sp, cp, s);
-  return wide ? launch_t<64, 8>(sp, cp, s) : launch_t<64, 4>(sp, cp, s);
+  // the caller checked supported_shape()
+  if (d == 128) return paged ? launch_tc<128, true>(sp, cp, s) : launch_tc<128, false>(sp, cp, s);
+  return paged ? launch_tc<64, true>(sp, cp, s) : launch_tc<64, false>(sp, cp, s);
 }
 
 }  // namespace attn_decode_impl

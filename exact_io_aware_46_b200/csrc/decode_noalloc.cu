@@ -78,6 +78,7 @@ extern "C" attn_status_t attn_fwd_splitkv_decode_noalloc(
   if (!(std::isfinite(scale) && scale > 0.f)) return ATTN_ERR_INVALID;
   if (d != 128 && d != 64) return ATTN_ERR_UNSUPPORTED;
   if (!attn_decode_impl::supported_group(Hq / Hkv)) return ATTN_ERR_UNSUPPORTED;
+  if (!attn_decode_impl::supported_shape(B, Hkv, Lmax, 0)) return ATTN_ERR_UNSUPPORTED;
   if (kHeader + attn_decode_impl::partials_bytes(B, Hq, Hkv, Lmax, d) >
       static_cast<size_t>(ATTN_NOALLOC_SCRATCH_BYTES))
     return ATTN_ERR_CAPACITY;

@@ -229,6 +229,9 @@ attn_status_t attn_fwd_varlen(const attn_bf16_t* Q, const attn_bf16_t* K, const 
  *   [B], required, each in [0, Lmax] (no causal mask inside the cache).
  *   O [B,Hq,1,d] bf16 and lse [B,Hq] fp32 (lse may be NULL).
  *   The workspace holds the fp32 partials; its size depends on Lmax.
+ *   Hq / Hkv must be 1, 2, 4 or 8, and Lmax at most 65535 * 2048 =
+ *   134,215,680 rows (the cache is split into chunks of 2048 keys, at most
+ *   65535 per sequence); else ATTN_ERR_UNSUPPORTED.
  */
 size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d);
 attn_status_t attn_fwd_splitkv_decode(const attn_bf16_t* Q, const attn_bf16_t* Kcache,
@@ -249,7 +252,8 @@ attn_status_t attn_fwd_splitkv_decode(const attn_bf16_t* Q, const attn_bf16_t* K
  *   Only the entries covering rows [0, k_lens[b]) are read; they must lie in
  *   [0, n_pages).  k_lens device int32 [B], required, each in
  *   [0, max_blocks * page_size].  page_size is a power of two in [16, 65536]
- *   (else ATTN_ERR_UNSUPPORTED).  Q, O, lse, scale as attn_fwd_splitkv_decode.
+ *   (else ATTN_ERR_UNSUPPORTED).  Q, O, lse, scale, the group sizes and the
+ *   limit on max_blocks * page_size as attn_fwd_splitkv_decode.
  *   The workspace is attn_decode_workspace_size(B, Hq, Hkv,
  *   max_blocks * page_size, d) bytes.
  *   A chunk whose block-table entries are out of range reads no page: it sets

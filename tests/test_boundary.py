@@ -92,6 +92,12 @@ def test_decode_and_bwd_reject_on_host(lib):
                                        1 << 20, None) == 2
     assert lib.attn_fwd_splitkv_decode(P, P, P, P, None, 1, 4, 1, 64, 72, 0.1, P, P,
                                        1 << 20, None) == 2
+    # a cache of more than 65535 chunks of 2048 keys is refused, noalloc entry included
+    big = 65535 * 2048 + 1
+    assert lib.attn_fwd_splitkv_decode(P, P, P, P, None, 1, 4, 1, big, 128, 0.1, P, P,
+                                       1 << 40, None) == 2
+    assert lib.attn_fwd_splitkv_decode_noalloc(P, P, P, P, None, 1, 4, 1, big, 128, 0.1, P,
+                                               None) == 2
     # bwd: lse is required; d must be 64 or 128
     assert lib.attn_bwd(P, P, P, P, P, None, P, P, P, 1, 1, 1, 8, 8, 128, 0.1, 0, None, P,
                         1 << 20, None) == 1
@@ -108,6 +114,8 @@ def test_paged_decode_rejects_on_host(lib):
     assert call(page=24) == 2 and call(page=8) == 2 and call(page=1 << 17) == 2
     assert call(ws_bytes=64) == 1
     assert call(d=96) == 2 and call(Hq=3) == 2
+    # 65536 pages of 2048 rows: more than 65535 chunks of 2048 keys
+    assert call(max_blocks=65536, page=2048, ws_bytes=1 << 40) == 2
 
 
 def test_varlen_fwd_rejects_on_host(lib):
