@@ -474,12 +474,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             break;
           sm100::tc_fence_after();
           if (it.n0 > jb && lo[0] == jb) {
-            if (!(ok = s_slot_free(0))) break;
+            ok = s_slot_free(0);
+            if (!ok) break;
             issue_s(0, ks);
             commit(&s_full[0]);
           }
           if (it.n1 > jb && lo[1] == jb) {
-            if (!(ok = s_slot_free(1))) break;
+            ok = s_slot_free(1);
+            if (!ok) break;
             issue_s(1, ks);
             commit(&s_full[1]);
           }
