@@ -32,12 +32,14 @@ CASES = [
     # B, Hq, Hkv, Lmax, d, k_lens
     (3, 8, 2, 3000, 128, [2500, 1, 2048]),        # chunk boundary, single key, exact chunk
     (1, 4, 1, 5000, 128, [4097]),                 # three chunks, the last holding one key
-    (2, 4, 4, 2100, 128, [2049, 2100]),           # G = 1 (padded to 4 lanes' heads)
+    (2, 4, 4, 2100, 128, [2049, 2100]),           # G = 1
     (2, 16, 2, 1500, 128, [1500, 777]),           # G = 8
     (2, 4, 2, 1300, 64, [1300, 65]),              # d = 64, G = 2
     (2, 8, 2, 1200, 128, [0, 1200]),              # an empty sequence
     (1, 4, 1, 70, 128, [70]),                     # shorter than one stage
     (2, 4, 2, 2200, 128, [128, 2177]),            # G = 2; one whole 128-key block; a chunk of 129 keys
+    (2, 16, 2, 4500, 64, [4500, 2049]),           # d = 64, G = 8: three chunks, the last of one key
+    (2, 4, 4, 2100, 64, [0, 2100]),               # d = 64, G = 1: an empty sequence, two chunks
 ]
 
 

@@ -54,6 +54,7 @@ CASES = [
     (2, 8, 2, 1200, 128, [0, 1200], 128),          # an empty sequence
     (1, 4, 1, 5000, 128, [4097], 1024),            # three chunks inside large pages
     (2, 4, 2, 2200, 128, [128, 2177], 32),         # G = 2; a chunk of 129 keys over 32-row pages
+    (2, 16, 2, 4200, 64, [4200, 2048], 16),        # d = 64, G = 8: three chunks over 16-row pages
 ]
 
 
