@@ -61,12 +61,12 @@ def bwd_flops(c):
 
 def peaks():
     p = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
-         "source": "fallback"}
+         "source": "fallback peaks (MEASURED_PEAKS.json absent)"}
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             m = json.load(f)
         p.update({k: float(m[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")})
-        p["source"] = "measured"
+        p["source"] = "measured peaks (MEASURED_PEAKS.json)"
     except Exception:
         pass
     return p
@@ -999,7 +999,7 @@ def main():
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
                      "traffic": traffic_per_launch("attn_fwd_impl::fwd_kernel<128>"),
-                     "peak_source": f"{pk['source']} burst bf16 (MEASURED_PEAKS.json)",
+                     "peak_source": f"{pk['source']}: burst bf16",
                      "kernel": "attn_fwd_impl::fwd_kernel<128>"},
         "e2e": {"value": world * flops / (t_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -1035,7 +1035,7 @@ def main():
         "roofline": {"bound": "tensor", "achieved": ach8, "peak": peak8, "unit": "TFLOP/s",
                      "frac": ach8 / peak8,
                      "traffic": traffic_per_launch("attn_fwd_impl::fwd_kernel<128,MODE_FP8>"),
-                     "peak_source": f"{pk['source']} burst bf16 x 2 (the nominal 8-bit:bf16 "
+                     "peak_source": f"{pk['source']}: burst bf16 x 2 (the nominal 8-bit:bf16 "
                                     f"dense ratio, 4.5 : 2.25 PFLOP/s)",
                      "kernel": "attn_fwd_impl::fwd_kernel<128,MODE_FP8>"},
     }
