@@ -15,6 +15,10 @@ The functions carry the C entry points' names:
 * ``attn_fwd_sliding`` / ``attn_bwd_sliding``: the same with a sliding-window causal mask
 * ``attn_fwd_fp8(Q8, K8, V8, q_scale, k_scale, v_scale, ...) -> (O, LSE)``: E4M3 inputs with
   one scale per 128-row tile
+* ``attn_fwd_splitkv_decode_noalloc``: the split decode without a workspace (a fixed
+  device array of ``ATTN_NOALLOC_SCRATCH_BYTES``)
+* ``attn_fwd_merge``, ``attn_merge_partial``, ``attn_accumulate``: the folds of ring
+  attention's partial results (``exact_io_aware_46_b200.ring`` drives them)
 * the ``*_workspace_size`` queries and the device-status helpers.
 """
 
