@@ -500,8 +500,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             break;
           sm100::tc_fence_after();
           // one query tile's step: O_t += P_t V_j, then S_t = Q_t K_{j+1}^T
-          // (d = 64: S_t = Q_t K_{j+1}^T first, then O_t += P_t V_j)
-          auto step = [&](int t, int n_t, uint32_t& pc) -> bool {
+          auto step = [&](int t, int n_t, uint32_t& pc, bool pv, bool sn) -> bool {
             auto do_pv = [&]() -> bool {
               if (lo[t] <= j && j < n_t) {
                 if (j == lo[t] && !sm100::mbar_wait(&o_empty[t], oe_par, abort_flag, p.status))
@@ -530,11 +529,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               }
               return true;
             };
-            if constexpr (C::SEP_P) return do_s() && do_pv();
-            else return do_pv() && do_s();
+            return (!pv || do_pv()) && (!sn || do_s());
           };
-          if (!(ok = step(0, it.n0, pc0))) break;
-          if (!(ok = step(1, it.n1, pc1))) break;
+          if constexpr (C::SEP_P) {
+            // d = 64 (P has columns of its own): both tiles' next S go in as soon
+            // as the softmax has read the current one, ahead of either PV, so
+            // neither tile's softmax waits behind the other tile's P
+            if (!(ok = step(0, it.n0, pc0, false, true) && step(1, it.n1, pc1, false, true) &&
+                       step(0, it.n0, pc0, true, false) && step(1, it.n1, pc1, true, false)))
+              break;
+          } else {
+            // P overwrites S: each tile's next S follows its PV
+            if (!(ok = step(0, it.n0, pc0, true, true))) break;
+            if (!(ok = step(1, it.n1, pc1, true, true))) break;
+          }
           if (k_ready) commit(&kv_empty[ks]);
           commit(&kv_empty[vs]);
           if (j + 2 == it.nmax) commit(q_empty);  // S_t(nmax - 1) were the last S
