@@ -222,6 +222,21 @@ __device__ __forceinline__ Item get_item(const Params& p, int w, bool* bad) {
   return it;
 }
 
+// 32-byte global store / load of eight 32-bit words (one whole sector per lane);
+// the address must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t* v) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+__device__ __forceinline__ void ld_global_v8(const void* p, uint32_t* v) {
+  asm volatile("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                 "=r"(v[6]), "=r"(v[7])
+               : "l"(p)
+               : "memory");
+}
+
 // Polynomial (FMA-pipe) instead of MUFU exp2 for column pairs whose index
 // cp = c / 2 satisfies cp % 8 >= 6 (bf16 at d = 128: a quarter of the
 // exponentials) or cp % 8 == 7 (8-bit inputs, and d = 64: an eighth; at d = 64,
@@ -775,6 +790,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         float* arow = p.o_acc + rix * D + DH * hf;
         __nv_bfloat16* orow = p.O ? p.O + rix * D + DH * hf : nullptr;
+        // 32-byte loads and stores when both rows start on 32-byte boundaries
+        const bool wide = ((reinterpret_cast<uintptr_t>(p.o_acc) |
+                            reinterpret_cast<uintptr_t>(p.O)) & 31) == 0;
 #pragma unroll 1
         for (int c = 0; c < DH / 16; ++c) {
           uint32_t o[16];
@@ -787,25 +805,51 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
           if (live) {
             float4* a4 = reinterpret_cast<float4*>(arow + c * 16);
-            float res[16];
+            uint32_t res[16];  // fp32 bits
+            if (wide) {  // 32-byte accesses: whole sectors of this thread's row
+              if (wa != 0.f) {
+                ld_global_v8(arow + c * 16, &res[0]);
+                ld_global_v8(arow + c * 16 + 8, &res[8]);
+              } else {
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const float4 a = (wa != 0.f) ? a4[v] : make_float4(0.f, 0.f, 0.f, 0.f);
-              res[4 * v] = wa * a.x + wb * __uint_as_float(o[4 * v]);
-              res[4 * v + 1] = wa * a.y + wb * __uint_as_float(o[4 * v + 1]);
-              res[4 * v + 2] = wa * a.z + wb * __uint_as_float(o[4 * v + 2]);
-              res[4 * v + 3] = wa * a.w + wb * __uint_as_float(o[4 * v + 3]);
+                for (int e = 0; e < 16; ++e) res[e] = 0u;
+              }
+            } else {
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                const float4 a = (wa != 0.f) ? a4[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+                res[4 * v] = __float_as_uint(a.x);
+                res[4 * v + 1] = __float_as_uint(a.y);
+                res[4 * v + 2] = __float_as_uint(a.z);
+                res[4 * v + 3] = __float_as_uint(a.w);
+              }
             }
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              a4[v] = make_float4(res[4 * v], res[4 * v + 1], res[4 * v + 2], res[4 * v + 3]);
+            for (int e = 0; e < 16; ++e)
+              res[e] = __float_as_uint(wa * __uint_as_float(res[e]) + wb * __uint_as_float(o[e]));
+            if (wide) {
+              st_global_v8(arow + c * 16, &res[0]);
+              st_global_v8(arow + c * 16 + 8, &res[8]);
+            } else {
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                a4[v] = make_float4(__uint_as_float(res[4 * v]), __uint_as_float(res[4 * v + 1]),
+                                    __uint_as_float(res[4 * v + 2]),
+                                    __uint_as_float(res[4 * v + 3]));
+            }
             if (orow) {
               uint32_t pk[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) pk[e] = sm100::pack_bf16x2(res[2 * e], res[2 * e + 1]);
-              uint4* dst = reinterpret_cast<uint4*>(orow + c * 16);
-              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+              for (int e = 0; e < 8; ++e)
+                pk[e] = sm100::pack_bf16x2(__uint_as_float(res[2 * e]),
+                                           __uint_as_float(res[2 * e + 1]));
+              if (wide) {
+                st_global_v8(orow + c * 16, pk);
+              } else {
+                uint4* dst = reinterpret_cast<uint4*>(orow + c * 16);
+                dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+              }
             }
           }
         }
@@ -821,6 +865,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       else
         orow = p.O + ((static_cast<size_t>(it.b) * p.Hq + it.h) * p.Lq + (live ? row : 0)) * D +
                DH * hf;
+      // each thread writes its own row, so a warp's store touches 32 rows: 32-byte
+      // stores fill whole sectors (measured on B200, causal B4 H16 L4096 d128:
+      // the O stores alone cost ~6 % of the kernel with 16-byte stores)
+      const bool o_v8 = (reinterpret_cast<uintptr_t>(p.O) & 31) == 0;
       if (n_t > 0) {
 #pragma unroll 1
         for (int c = 0; c < DH / 32; ++c) {
@@ -833,10 +881,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             pk[e] = sm100::pack_bf16x2(__uint_as_float(o[2 * e]) * inv,
                                        __uint_as_float(o[2 * e + 1]) * inv);
           if (live) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+            if (o_v8) {  // a row's 64 bytes as two full sectors
+              st_global_v8(orow + c * 32, &pk[0]);
+              st_global_v8(orow + c * 32 + 16, &pk[8]);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+              for (int v = 0; v < 4; ++v)
+                dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
           }
         }
       } else if (live) {

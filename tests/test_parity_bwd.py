@@ -99,6 +99,32 @@ def test_bwd_d64_matches_oracle(B, Hq, Hkv, Lq, Lk, causal, k_lens):
     _check(to_f64(dv), rV, "dV")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_bwd_gradients_aligned_to_16_bytes_only(d):
+    """dK and dV 16-byte but not 32-byte aligned (the boundary asks for 16): dK and
+    dV are bit-identical to buffers at 32-byte boundaries and match the oracle."""
+    import torch
+
+    attn = _lib()
+    B, H, L = 1, 2, 300
+    Q, K, V, dO = (synth.normal_bf16(4700 + d + i, (B, H, L, d)) for i in range(4))
+    q, k, v, do = (dev_bf16(t) for t in (Q, K, V, dO))
+    O, Lse = attn.attn_fwd(q, k, v, causal=True)
+    _, dk1, dv1 = attn.attn_bwd(q, k, v, O, do, Lse, causal=True)
+    n = B * H * L * d
+    kb = torch.empty(n + 8, dtype=torch.bfloat16, device="cuda")
+    vb = torch.empty(n + 8, dtype=torch.bfloat16, device="cuda")
+    dk2, dv2 = kb[8:].view(B, H, L, d), vb[8:].view(B, H, L, d)
+    assert dk2.data_ptr() % 32 == 16 and dv2.data_ptr() % 32 == 16
+    dq2, _, _ = attn.attn_bwd(q, k, v, O, do, Lse, causal=True, dK=dk2, dV=dv2)
+    torch.cuda.synchronize()
+    assert torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
+    rQ, rK, rV = oracle.bwd(Q, K, V, dO, 1.0 / math.sqrt(d), causal=True)
+    _check(to_f64(dq2), rQ, "dQ")
+    _check(to_f64(dk2), rK, "dK")
+    _check(to_f64(dv2), rV, "dV")
+
+
 def test_bwd_full_size_sampled():
     """B=2, H=16, L=8192, d=128, causal: sampled rows of dQ and keys of dK, dV."""
     import torch

@@ -113,6 +113,29 @@ def test_fwd_deterministic():
     assert torch.equal(O1, O2) and torch.equal(L1, L2)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_fwd_output_aligned_to_16_bytes_only(d):
+    """O may be 16-byte aligned without being 32-byte aligned (the boundary asks for 16):
+    the epilogue then stores 16 bytes at a time; the result is bit-identical to an
+    output buffer at a 32-byte boundary, and matches the oracle."""
+    import torch
+
+    attn = _lib()
+    B, H, L = 2, 3, 300
+    Q, K, V = _inputs(77 + d, B, H, H, L, L, d)
+    q, k, v = dev_bf16(Q), dev_bf16(K), dev_bf16(V)
+    O1, L1 = attn.attn_fwd(q, k, v, causal=True)
+    big = torch.empty(B * H * L * d + 8, dtype=torch.bfloat16, device="cuda")
+    O2 = big[8:].view(B, H, L, d)  # 16 bytes past the allocation's start
+    assert O2.data_ptr() % 32 == 16
+    _, L2 = attn.attn_fwd(q, k, v, causal=True, O=O2)
+    torch.cuda.synchronize()
+    assert torch.equal(O1, O2) and torch.equal(L1, L2)
+    Oref, Lref = oracle.fwd(Q, K, V, 1 / math.sqrt(d), causal=True)
+    assert_out_close(to_f64(O2), Oref)
+    assert_lse_close(to_f64(L2), Lref)
+
+
 def test_bad_k_len_sets_status_and_zeroes():
     import torch
 

@@ -142,6 +142,39 @@ def test_fwd_merge_rows_without_keys_keep_the_accumulator():
     assert torch.all(acc == 0) and torch.all(O == 0) and torch.all(torch.isneginf(lacc))
 
 
+def test_fwd_merge_buffers_aligned_to_16_bytes_only():
+    """The fused fold with O_acc and O_out 16-byte but not 32-byte aligned (the
+    boundary asks for 16): the epilogue then moves 16 bytes at a time; the results
+    are bit-identical to buffers at 32-byte boundaries."""
+    import torch
+
+    attn = _lib()
+    B, H, Lq, LA, LB, d = 1, 2, 200, 260, 140, 128
+    Q = synth.normal_bf16(9311, (B, H, Lq, d))
+    KA, VA = synth.normal_bf16(9312, (B, H, LA, d)), synth.normal_bf16(9313, (B, H, LA, d))
+    KB, VB = synth.normal_bf16(9314, (B, H, LB, d)), synth.normal_bf16(9315, (B, H, LB, d))
+    q = dev_bf16(Q)
+    n = B * H * Lq * d
+    outs = []
+    for shift in (0, 4):  # 0 or 4 fp32 (16 bytes) past a 32-byte boundary
+        acc_big = torch.empty(n + 8, dtype=torch.float32, device="cuda")
+        o_big = torch.empty(n + 16, dtype=torch.bfloat16, device="cuda")
+        acc = acc_big[shift:shift + n].view(B, H, Lq, d)
+        O = o_big[2 * shift:2 * shift + n].view(B, H, Lq, d)
+        assert acc.data_ptr() % 32 == 4 * shift and O.data_ptr() % 32 == 4 * shift
+        lacc = torch.empty((B, H, Lq), dtype=torch.float32, device="cuda")
+        attn.attn_fwd_merge(q, dev_bf16(KA), dev_bf16(VA), acc, lacc, init=True)
+        attn.attn_fwd_merge(q, dev_bf16(KB), dev_bf16(VB), acc, lacc, init=False, O_out=O)
+        torch.cuda.synchronize()
+        outs.append((acc.clone(), lacc.clone(), O.clone()))
+    for a, b in zip(outs[0], outs[1]):
+        assert torch.equal(a, b)
+    Oref, Lref = oracle.fwd(Q, np.concatenate([KA, KB], axis=2), np.concatenate([VA, VB], axis=2),
+                            1.0 / math.sqrt(d))
+    assert_out_close(to_f64(outs[1][2]), Oref)
+    assert_lse_close(to_f64(outs[1][1]), Lref)
+
+
 def test_accumulate_kernel():
     import torch
 
