@@ -56,6 +56,25 @@ def test_decode_matches_oracle(B, Hq, Hkv, Lmax, d, k_lens):
     assert_lse_close(L, Lref[:, :, 0])
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_large_logits(d):
+    """Scale 1 (scores of size ~sqrt(d)): each head's probabilities concentrate on a
+    few keys across several 2048-key chunks, so the chunks' partial maxima differ by
+    tens of log2 units in the combine.  |O| then reaches ~4, so the absolute O bar is
+    scaled by max(1, |O_ref|) as in the forward's large-logit test."""
+    B, Hq, Hkv, Lmax = 2, 8, 2, 4600
+    k_lens = [4600, 2100]
+    Q = synth.normal_bf16(9900 + d, (B, Hq, 1, d))
+    K = synth.normal_bf16(9910 + d, (B, Hkv, Lmax, d))
+    V = synth.normal_bf16(9920 + d, (B, Hkv, Lmax, d))
+    O, L = _run(Q, K, V, k_lens, 1.0)
+    Oref, Lref = oracle.fwd(Q, K, V, 1.0, causal=False, k_lens=k_lens)
+    err = np.abs(O - Oref)
+    bound = 1e-2 * np.maximum(1.0, np.abs(Oref))
+    assert np.all(err <= bound), f"max err/bound {np.max(err / bound):.3f}"
+    assert_lse_close(L, Lref[:, :, 0])
+
+
 def test_decode_deterministic_and_status():
     import torch
 
