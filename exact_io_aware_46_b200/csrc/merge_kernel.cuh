@@ -12,7 +12,10 @@
 //
 // HBM-bound elementwise work: per row, 4d bytes of accumulator read and
 // written, 2d bytes of bf16 partial read, 12 bytes of LSE.  One thread per 8
-// elements of a row (16-byte loads), rows laid out back to back.
+// elements of a row, rows laid out back to back: the thread's 32 bytes of the
+// fp32 accumulator move as one 32-byte access (whole sectors) when the
+// accumulator is 32-byte aligned (measured on B200, 131,072 rows of d = 128:
+// 4.6-4.8 TB/s with two 16-byte accesses).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -33,6 +36,19 @@ struct Params {
 
 constexpr int NTHREADS = 256;
 
+__device__ __forceinline__ void ld_global_v8(const void* p, uint32_t* v) {
+  asm volatile("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                 "=r"(v[6]), "=r"(v[7])
+               : "l"(p)
+               : "memory");
+}
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t* v) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
 __global__ void __launch_bounds__(NTHREADS) merge_kernel(const Params p) {
   const int tpr = p.d / 8;  // threads per row
   const int rows_per_block = NTHREADS / tpr;
@@ -42,6 +58,7 @@ __global__ void __launch_bounds__(NTHREADS) merge_kernel(const Params p) {
   const unsigned row_mask =
       (tpr == 32 ? 0xffffffffu : ((1u << tpr) - 1u)) << ((threadIdx.x & 31) - lane);
   if (sub >= rows_per_block) return;
+  const bool wide = (reinterpret_cast<uintptr_t>(p.O_acc) & 31) == 0;
   for (long long row = static_cast<long long>(blockIdx.x) * rows_per_block + sub; row < p.rows;
        row += static_cast<long long>(gridDim.x) * rows_per_block) {
     const size_t off = static_cast<size_t>(row) * p.d + lane * 8;
@@ -63,6 +80,11 @@ __global__ void __launch_bounds__(NTHREADS) merge_kernel(const Params p) {
     if (p.init) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) o[e] = 0.f;
+    } else if (wide) {
+      uint32_t a[8];
+      ld_global_v8(p.O_acc + off, a);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = __uint_as_float(a[e]);
     } else {
       const float4 a0 = *reinterpret_cast<const float4*>(p.O_acc + off);
       const float4 a1 = *reinterpret_cast<const float4*>(p.O_acc + off + 4);
@@ -75,8 +97,15 @@ __global__ void __launch_bounds__(NTHREADS) merge_kernel(const Params p) {
       o[2 * e] = wa * o[2 * e] + wb * f.x;
       o[2 * e + 1] = wa * o[2 * e + 1] + wb * f.y;
     }
-    *reinterpret_cast<float4*>(p.O_acc + off) = make_float4(o[0], o[1], o[2], o[3]);
-    *reinterpret_cast<float4*>(p.O_acc + off + 4) = make_float4(o[4], o[5], o[6], o[7]);
+    if (wide) {
+      uint32_t a[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) a[e] = __float_as_uint(o[e]);
+      st_global_v8(p.O_acc + off, a);
+    } else {
+      *reinterpret_cast<float4*>(p.O_acc + off) = make_float4(o[0], o[1], o[2], o[3]);
+      *reinterpret_cast<float4*>(p.O_acc + off + 4) = make_float4(o[4], o[5], o[6], o[7]);
+    }
     if (p.O_out) {
       uint4 ob;
       __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&ob);
