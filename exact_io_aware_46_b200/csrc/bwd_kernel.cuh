@@ -25,12 +25,13 @@
 //     dV and dK accumulate in TMEM across the item (256 columns); S^T/P^T and
 //     dP^T take the other 256, and dQ^T reuses the dP^T columns once dS has
 //     been formed.  Tensor memory holds one query tile at a time, so the
-//     issue order S^T(t), dP^T(t), dV(t), dQ^T(t), dK(t), S^T(t+1) gives each
-//     hand-off one MMA group of cover: P(t) forms while dP^T(t) runs, dS(t)
-//     while dV(t) runs, and the drain of dQ^T(t) while dK(t) and S^T(t+1) run.
-//     Warps 0-7 form P and dS (one key row per thread, two warps per row, 64
-//     query rows each), warps 8-11 drain dQ^T into the fp32 accumulator with
-//     bulk reduce-adds, warp 12 feeds TMA, warp 13 issues MMAs.
+//     issue order S^T(t), dK(t-1), dP^T(t), dV(t), dQ^T(t), S^T(t+1), dK(t), ...
+//     gives each hand-off one MMA group of cover: P(t) forms while dK(t-1) and
+//     dP^T(t) run, dS(t) while dV(t) runs, and the drain of dQ^T(t) while
+//     S^T(t+1) and dK(t) run.  Warps 0-7 form P and dS (one key row per thread,
+//     two warps per row, 64 query rows each), warps 8-11 drain dQ^T into the
+//     fp32 accumulator (d = 128: coalesced reductions and bulk reduce-adds;
+//     d = 64: tensor reduce-adds), warp 12 feeds TMA, warp 13 issues MMAs.
 //  3. convert: dQ = bf16(scale * accumulator).
 #pragma once
 
