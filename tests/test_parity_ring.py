@@ -175,6 +175,40 @@ def test_fwd_merge_buffers_aligned_to_16_bytes_only():
     assert_lse_close(to_f64(outs[1][1]), Lref)
 
 
+def test_merge_and_accumulate_accumulators_aligned_to_16_bytes_only():
+    """attn_merge_partial and attn_accumulate with fp32 accumulators 16-byte but not
+    32-byte aligned (the boundary asks for 16): bit-identical results to accumulators
+    at 32-byte boundaries (the kernels then move 16 bytes at a time)."""
+    import torch
+
+    attn = _lib()
+    rows, d = 700, 128
+    Ob = dev_bf16(synth.normal_bf16(9500, (rows, d)))
+    lb = torch.from_numpy((np.random.default_rng(9501).standard_normal(rows) * 3)
+                          .astype(np.float32)).cuda()
+    A0 = torch.from_numpy(np.random.default_rng(9502).standard_normal((rows, d))
+                          .astype(np.float32)).cuda()
+    l0 = torch.from_numpy(np.random.default_rng(9503).standard_normal(rows)
+                          .astype(np.float32)).cuda()
+    parts = [dev_bf16(synth.normal_bf16(9510 + i, (rows, d))) for i in range(2)]
+    results = []
+    for shift in (0, 4):  # fp32 elements past a 32-byte boundary
+        big = torch.empty(rows * d + 8, dtype=torch.float32, device="cuda")
+        acc = big[shift:shift + rows * d].view(rows, d)
+        assert acc.data_ptr() % 32 == 4 * shift
+        acc.copy_(A0)
+        lacc = l0.clone()
+        attn.attn_merge_partial(Ob, lb, acc, lacc, init=False)
+        merged = acc.clone()
+        attn.attn_accumulate(parts[0], acc, init=True)
+        attn.attn_accumulate(parts[1], acc, init=False)
+        torch.cuda.synchronize()
+        results.append((merged, lacc.clone(), acc.clone()))
+    for a, b in zip(results[0], results[1]):
+        assert torch.equal(a, b)
+    assert torch.equal(results[1][2], parts[0].float() + parts[1].float())
+
+
 def test_accumulate_kernel():
     import torch
 
